@@ -1,0 +1,512 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle.
+
+Each test ties one oracle function to something independent of it: a value
+set printed for the method, a closed form evaluated with exact rationals, a
+library routine (numpy's binary16 cast, torch's fp64 matmul), brute force
+over tiny inputs, or an algebraic identity.  A plausible slip in the oracle
+(wrong bias, dropped subnormal, wrong tie rule, swapped nibbles, a wrong
+sign or index in the GEMM) fails at least one of them.
+"""
+import math
+import os
+from fractions import Fraction as Fr
+
+import numpy as np
+import pytest
+import torch
+
+from w4a16_gemm_fp4_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+# (e, m) of the three 4-bit formats; bias b = 2^(e-1) - 1 (IEEE-style)
+FMT_EM = {0: (1, 2), 1: (2, 1), 2: (3, 0)}
+
+
+# ----------------------------------------------------------- independent helpers
+
+def value_exact(fmt, code):
+    """Closed form of the ExMy value, as exact rationals."""
+    e, m = FMT_EM[fmt]
+    b = 2 ** (e - 1) - 1
+    s = (code >> 3) & 1
+    p = (code >> m) & ((1 << e) - 1)
+    d = code & ((1 << m) - 1)
+    frac = Fr(d, 1 << m)
+    v = (frac * Fr(2) ** (1 - b)) if p == 0 else ((1 + frac) * Fr(2) ** (p - b))
+    return -v if s else v
+
+
+def mags_exact(fmt):
+    return [value_exact(fmt, i) for i in range(8)]
+
+
+def nearest_exact(q, mags):
+    """Nearest magnitude of |q| (a Fraction), ties to the even index,
+    saturating at the top of the grid."""
+    a = abs(q)
+    if a >= mags[7]:
+        return 7
+    dists = [abs(a - v) for v in mags]
+    best = min(dists)
+    cands = [i for i, dd in enumerate(dists) if dd == best]
+    if len(cands) == 1:
+        return cands[0]
+    assert len(cands) == 2 and cands[1] == cands[0] + 1
+    return cands[0] if cands[0] % 2 == 0 else cands[1]
+
+
+def f32(x):
+    return np.float32(x)
+
+
+def bf16_rne_exact(x: np.float32) -> int:
+    """bf16 bits of a finite float by exact rational rounding."""
+    xf = float(x)
+    if xf == 0.0:
+        return 0x8000 if math.copysign(1.0, xf) < 0 else 0
+    sign = 0x8000 if xf < 0 else 0
+    a = Fr(abs(xf))
+    E = math.frexp(abs(xf))[1] - 1          # binade 2^E
+    E = max(E, -126)
+    ulp = Fr(2) ** (E - 7)
+    q = a / ulp
+    r = math.floor(q)
+    rem = q - r
+    if rem > Fr(1, 2) or (rem == Fr(1, 2) and r % 2 == 1):
+        r += 1
+    y = float(r * ulp)
+    bits = np.array([y], np.float32).view(np.uint32)[0] >> 16
+    return int(bits) | sign
+
+
+def scale_ref(A, j, fmt, sdt):
+    """Reading R3 with numpy float32 arithmetic (IEEE, RNE)."""
+    qmax = f32(float(mags_exact(fmt)[7]))
+    cj = c_exact_f32(j)
+    t = f32(f32(A) * cj)
+    s32 = f32(t / qmax)
+    if sdt == "f16":
+        return np.float32(np.float16(s32))
+    return s32
+
+
+def c_exact_f32(j):
+    """fl32(2^(-j/8)) from a 60-digit decimal evaluation."""
+    from decimal import Decimal, getcontext
+    getcontext().prec = 60
+    v = Decimal(2) ** (Decimal(-j) / Decimal(8))
+    # correctly round the 60-digit value to binary32 via Fraction
+    fr = Fr(v)
+    lo = np.float32(float(fr))
+    # float(fr) is correctly rounded to binary64; step to the nearest binary32
+    cands = [np.nextafter(lo, np.float32(-1)), lo, np.nextafter(lo, np.float32(2))]
+    return min(cands, key=lambda c: (abs(Fr(float(c)) - fr), int(np.array([c]).view(np.uint32)[0]) & 1))
+
+
+def quantize_bruteforce(W, g, fmt, j, sdt):
+    """Pure-Python reference of readings R3-R5 for tiny tensors."""
+    N, K = W.shape
+    mags = mags_exact(fmt)
+    codes = np.zeros((N, K), np.int64)
+    scales = np.zeros((N, K // g), np.float32)
+    sse = Fr(0)
+    for n in range(N):
+        for gi in range(K // g):
+            seg = W[n, gi * g:(gi + 1) * g]
+            A = np.max(np.abs(seg)).astype(np.float32)
+            s = scale_ref(A, j, fmt, sdt)
+            scales[n, gi] = s
+            for t in range(g):
+                x = seg[t]
+                idx = 0
+                if s != 0:
+                    q = f32(x / s)
+                    idx = nearest_exact(Fr(float(q)), mags)
+                sign = 1 if math.copysign(1.0, float(x)) < 0 else 0
+                codes[n, gi * g + t] = (sign << 3) | idx
+                v = -mags[idx] if sign else mags[idx]
+                sse += (Fr(float(x)) - v * Fr(float(s))) ** 2
+    return codes, scales, sse
+
+
+def unpack(packed):
+    lo = packed & 0x0F
+    hi = packed >> 4
+    out = np.empty((packed.shape[0], packed.shape[1] * 2), np.int64)
+    out[:, 0::2] = lo
+    out[:, 1::2] = hi
+    return out
+
+
+def dequant_independent(packed, scales, fmt, g):
+    codes = unpack(packed)
+    vals = np.array([float(value_exact(fmt, c)) for c in range(16)])
+    s = np.repeat(scales.astype(np.float64), g, axis=1)
+    return vals[codes] * s
+
+
+# --------------------------------------------------------------------- format table
+
+def test_e2m1_value_set_matches_printed_set(oracle_mod):
+    """E2M1 magnitudes = the set printed for the method, from golden file."""
+    path = os.path.join(GOLDEN, "e2m1_values.txt")
+    printed = [float(t) for t in open(path).read().split("#")[0].split()]
+    mags, qmax = oracle_mod.format_table(oracle_mod.E2M1)
+    assert list(mags) == printed
+    assert qmax == 6.0
+
+
+@pytest.mark.parametrize("fmt", [0, 1, 2])
+def test_code_values_closed_form_all_16(oracle_mod, fmt):
+    """All 16 codes of every format equal the closed form (exact)."""
+    for code in range(16):
+        assert Fr(oracle_mod.code_value(fmt, code)) == value_exact(fmt, code)
+    mags, qmax = oracle_mod.format_table(fmt)
+    assert all(mags[i] < mags[i + 1] for i in range(7)), "magnitude index must be monotone"
+    for i in range(8):
+        assert oracle_mod.code_value(fmt, 8 + i) == -mags[i] or (i == 0 and mags[0] == 0.0)
+    assert oracle_mod.format_bias(fmt) == 2 ** (FMT_EM[fmt][0] - 1) - 1
+
+
+def test_other_format_tables():
+    """E1M2 is uniform in steps of 1/2; E3M0 is 0 and powers of two."""
+    assert [float(v) for v in mags_exact(0)] == [0, .5, 1, 1.5, 2, 2.5, 3, 3.5]
+    assert [float(v) for v in mags_exact(2)] == [0, .25, .5, 1, 2, 4, 8, 16]
+
+
+def test_bias_factors_correctly_rounded(oracle_mod):
+    for j in range(8):
+        assert oracle_mod.bias_factor(j) == c_exact_f32(j), j
+    assert oracle_mod.bias_factor(0) == np.float32(1.0)
+
+
+# ------------------------------------------------------------------ float rounding
+
+def test_f16_rounding_matches_numpy(oracle_mod):
+    rng = np.random.default_rng(11)
+    x = np.concatenate([
+        rng.standard_normal(3000).astype(np.float32) * np.float32(1e-3),
+        (rng.standard_normal(1000) * 1e4).astype(np.float32),
+        np.array([0.0, -0.0, 65504.0, 65519.0, 65520.0, 1e9, 6.1e-5, 5.96e-8, 2.98e-8, 2.99e-8,
+                  1e-12, -3.0e-6, 1.0009765625, 1.00048828125, 1.00146484375], np.float32),
+    ])
+    ours = oracle_mod.f32_to_f16(x)
+    with np.errstate(over="ignore"):
+        ref = x.astype(np.float16).view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+def test_bf16_rounding_matches_exact(oracle_mod):
+    rng = np.random.default_rng(12)
+    x = np.concatenate([rng.standard_normal(2000).astype(np.float32),
+                        np.array([1.00390625, 1.005859375, 1.0078125 + 2 ** -9, -0.0, 3e-39, 1.1754944e-38],
+                                 np.float32)])
+    ours = oracle_mod.f32_to_bf16(x)
+    ref = np.array([bf16_rne_exact(v) for v in x], np.uint16)
+    assert np.array_equal(ours, ref)
+    # torch's cast is a second, library reference
+    tref = synth.to_bf16_bits(x)
+    assert np.array_equal(ours, tref)
+
+
+# ---------------------------------------------------------------- nearest / RNE
+
+@pytest.mark.parametrize("fmt", [0, 1, 2])
+def test_nearest_index_every_midpoint(oracle_mod, fmt):
+    mags = mags_exact(fmt)
+    pts = set()
+    for i in range(7):
+        mid = (mags[i] + mags[i + 1]) / 2
+        pts.update([mid, mags[i], mags[i + 1]])
+    pts.update([mags[7] * 2, Fr(0)])
+    for p in sorted(pts):
+        for eps in (Fr(0), Fr(1, 1 << 20), -Fr(1, 1 << 20)):
+            q = p + eps
+            if q < 0:
+                continue
+            assert oracle_mod.nearest_index(float(q), fmt) == nearest_exact(q, mags), (fmt, q)
+
+
+@pytest.mark.parametrize("fmt,sdt", [(1, "f32"), (1, "f16"), (0, "f16"), (2, "f32")])
+def test_quantize_bruteforce_tiny(oracle_mod, fmt, sdt):
+    """Codes, scales and SSE of a tiny tensor equal a pure-Python quantizer."""
+    rng = np.random.default_rng(5 + fmt)
+    W = (rng.standard_normal((3, 64)) * 0.05).astype(np.float32)
+    # constructed group: absmax 6 * s with every midpoint, zeros of both signs
+    s0 = np.float32(0.25)
+    mags = [float(v) for v in mags_exact(fmt)]
+    qmax = mags[7]
+    row = [qmax * s0] + [((mags[i] + mags[i + 1]) / 2) * s0 for i in range(7)]
+    row += [-v for v in row[1:]] + [0.0, -0.0, 1e-9, -1e-9]
+    W[2, :32] = np.array(row + [0.0] * (32 - len(row)), np.float32)
+    for j in (0, 3, 7):
+        packed, scales, sse = oracle_mod.quantize_fixed(W, 32, fmt, j, None, sdt)
+        codes, sref, sse_ref = quantize_bruteforce(W, 32, fmt, j, sdt)
+        assert np.array_equal(unpack(packed), codes), (fmt, sdt, j)
+        assert np.array_equal(scales.astype(np.float32), sref)
+        assert abs(Fr(sse) - sse_ref) <= sse_ref * Fr(1, 10 ** 12) + Fr(1, 10 ** 300)
+
+
+def test_negative_zero_and_small_negatives_keep_sign(oracle_mod):
+    W = np.zeros((1, 32), np.float32)
+    W[0, 0] = 6.0
+    W[0, 1] = -0.0
+    W[0, 2] = -0.2   # |q| = 0.2 -> magnitude 0, sign kept
+    W[0, 3] = 0.2
+    packed, _, _ = oracle_mod.quantize_fixed(W, 32, 1, 0, None, "f32")
+    c = unpack(packed)[0]
+    assert c[0] == 7 and c[1] == 8 and c[2] == 8 and c[3] == 0
+
+
+def test_zero_group_gives_zero_scale_and_code(oracle_mod):
+    W = np.zeros((2, 64), np.float32)
+    W[1, 32:] = -0.0
+    packed, scales, sse = oracle_mod.quantize_fixed(W, 32, 1, 0, None, "f16")
+    assert np.all(scales == 0)
+    assert np.all(unpack(packed)[0] == 0)
+    assert np.all(unpack(packed)[1, 32:] == 8)
+    assert sse == 0.0
+
+
+def test_fp16_scale_underflow_gives_code_zero(oracle_mod):
+    W = np.zeros((1, 32), np.float32)
+    W[0, :4] = [1e-9, -1e-9, 5e-10, 0]
+    packed, scales, sse = oracle_mod.quantize_fixed(W, 32, 1, 0, None, "f16")
+    assert scales[0, 0] == 0
+    assert list(unpack(packed)[0, :4]) == [0, 8, 0, 0]
+    assert sse == pytest.approx(float(np.sum(W.astype(np.float64) ** 2)))
+
+
+def test_fp16_scale_overflow_is_an_error(oracle_mod):
+    W = np.zeros((1, 32), np.float32)
+    W[0, 0] = 1e6   # 1e6 / 6 > 65504
+    with pytest.raises(oracle_mod.OracleError):
+        oracle_mod.quantize_fixed(W, 32, 1, 0, None, "f16")
+
+
+def test_nonfinite_input_is_an_error(oracle_mod):
+    W = np.zeros((1, 32), np.float32)
+    W[0, 5] = np.nan
+    with pytest.raises(oracle_mod.OracleError):
+        oracle_mod.quantize_fixed(W, 32, 1, 0, None, "f32")
+
+
+@pytest.mark.parametrize("fmt", [0, 1, 2])
+def test_idempotence_on_grid_values(oracle_mod, fmt):
+    """quantize(dequantize(c)) == c for every code, incl. 0x8 (-0)."""
+    rng = np.random.default_rng(21 + fmt)
+    N, K, g = 8, 256, 128
+    codes = rng.integers(0, 16, size=(N, K))
+    codes[:, ::g] = 7                           # every group reaches Qmax
+    # power-of-two scales keep Qmax*s exact so the recomputed scale is s
+    sexp = rng.integers(-12, -2, size=(N, K // g))
+    s = np.ldexp(np.ones_like(sexp, dtype=np.float64), sexp).astype(np.float32)
+    vals = np.array([float(value_exact(fmt, c)) for c in range(16)])
+    W = (vals[codes] * np.repeat(s.astype(np.float64), g, axis=1)).astype(np.float32)
+    W[codes == 8] = -0.0
+    packed, scales, sse = oracle_mod.quantize_fixed(W, g, fmt, 0, None, "f32")
+    assert np.array_equal(unpack(packed), codes)
+    assert np.array_equal(scales, s)
+    assert sse == 0.0
+
+
+# -------------------------------------------------------------------------- pack
+
+def test_pack_low_nibble_first(oracle_mod):
+    """codes (1, 2) -> byte 0x21: element k even in the low nibble."""
+    W = np.zeros((1, 32), np.float32)
+    W[0, 0] = 0.5    # E2M1 index 1 with s = 1 (absmax 6)
+    W[0, 1] = 1.0    # index 2
+    W[0, 2] = 6.0
+    packed, _, _ = oracle_mod.quantize_fixed(W, 32, 1, 0, None, "f32")
+    assert packed[0, 0] == 0x21
+    assert packed[0, 1] == 0x07
+
+
+def test_pack_roundtrip(oracle_mod):
+    W, _ = synth.random_case(3, 16, 256, 1)
+    packed, scales, _ = oracle_mod.quantize_fixed(W, 128, 1, 0, None, "f16")
+    codes = unpack(packed)
+    repacked = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+    assert np.array_equal(repacked, packed)
+
+
+# ------------------------------------------------------------------------ search
+
+def exact_sse_all(W, g, sdt):
+    out = {}
+    for f in range(3):
+        for j in range(8):
+            _, _, sse = quantize_bruteforce(W, g, f, j, sdt)
+            out[(f, j)] = sse
+    return out
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_search_is_mse_optimal_tiny(oracle_mod, seed):
+    rng = np.random.default_rng(100 + seed)
+    W = (rng.standard_t(5, size=(2, 64)) * 0.015).astype(np.float32)
+    res = oracle_mod.quantize(W, 32, oracle_mod.AUTO, True, None, "f16")
+    exact = exact_sse_all(W, 32, "f16")
+    best = min(exact.values())
+    f, j = res["choice"]
+    assert exact[(f, j)] == best
+    # first strict minimum in (format, j) order
+    first = min((k for k, v in exact.items() if v == best))
+    assert (f, j) == first
+    for (ff, jj), v in exact.items():
+        assert abs(Fr(res["sse"][ff * 8 + jj]) - v) <= v * Fr(1, 10 ** 12) + Fr(1, 10 ** 300)
+
+
+def test_search_tie_rule_first_candidate(oracle_mod):
+    """All-zero tensor: every candidate has SSE 0 -> (E1M2, j=0)."""
+    res = oracle_mod.quantize(np.zeros((2, 64), np.float32), 32, oracle_mod.AUTO, True)
+    assert res["choice"] == (0, 0)
+    # one value per group at +-absmax: the three j=0 candidates are exact
+    W = np.zeros((2, 64), np.float32)
+    W[:, 0] = 168 * 2.0 ** -10     # /3.5, /6 and /16 are all exact in fp16
+    W[:, 32] = -84 * 2.0 ** -10
+    res = oracle_mod.quantize(W, 32, oracle_mod.AUTO, True)
+    assert res["choice"] == (0, 0)
+    assert res["sse"][0] == 0.0 and res["sse"][8] == 0.0 and res["sse"][16] == 0.0
+
+
+def test_search_modes(oracle_mod):
+    W, _ = synth.random_case(4, 4, 128, 1, dist="t")
+    r_fixed = oracle_mod.quantize(W, 128, 1, False)
+    assert r_fixed["choice"] == (1, 0)
+    assert np.isnan(r_fixed["sse"][0]) and not np.isnan(r_fixed["sse"][8])
+    r_bias = oracle_mod.quantize(W, 128, 1, True)
+    assert r_bias["choice"][0] == 1
+    assert np.all(np.isnan(r_bias["sse"][:8])) and np.all(~np.isnan(r_bias["sse"][8:16]))
+    r_fmt = oracle_mod.quantize(W, 128, oracle_mod.AUTO, False)
+    assert r_fmt["choice"][1] == 0
+    assert np.all(~np.isnan(r_fmt["sse"][[0, 8, 16]]))
+
+
+# ------------------------------------------------------------------------- fold
+
+def test_fold_equals_prescaled_weights(oracle_mod):
+    """quantize(W, shift) == quantize(W * 2^shift) (numpy float32 multiply)."""
+    W, _ = synth.random_case(6, 8, 256, 1)
+    rng = np.random.default_rng(7)
+    shift = rng.integers(-9, 1, size=256).astype(np.int8)
+    Wp = (W * np.ldexp(np.float32(1), shift.astype(np.int32)).astype(np.float32)).astype(np.float32)
+    a = oracle_mod.quantize(W, 128, 1, True, shift, "f16")
+    b = oracle_mod.quantize(Wp, 128, 1, True, None, "f16")
+    assert a["choice"] == b["choice"]
+    assert np.array_equal(a["packed"], b["packed"])
+    assert np.array_equal(a["scales"], b["scales"])
+
+
+def test_fold_identity_fp64(oracle_mod):
+    """X.W^T == (X*2^-e).(W*2^e)^T bitwise in fp64 (power-of-two scaling
+    commutes exactly with every product), and the prologue output times rho
+    reproduces X*2^-e within bf16 rounding."""
+    rng = np.random.default_rng(8)
+    X, idx = synth.outlier_activations(rng, 16, 256)
+    W = synth.normal_weights(rng, 12, 256)
+    shift, rho = oracle_mod.preshift_calibrate(X)
+    x = synth.bf16_bits_to_f32(X).astype(np.float64)
+    p = np.ldexp(1.0, shift.astype(np.int32))
+    lhs = np.zeros((16, 12))
+    rhs = np.zeros((16, 12))
+    for m in range(16):
+        for n in range(12):
+            a = 0.0
+            b = 0.0
+            for k in range(256):
+                a += x[m, k] * float(W[n, k])
+                b += (x[m, k] / p[k]) * (float(W[n, k]) * p[k])
+            lhs[m, n] = a
+            rhs[m, n] = b
+    assert np.array_equal(lhs, rhs)
+    Xt = oracle_mod.preshift_apply(X, shift, rho)
+    xt = synth.bf16_bits_to_f32(Xt).astype(np.float64)
+    assert np.max(np.abs(xt)) <= 1.0
+    np.testing.assert_allclose(xt * float(rho), x / p, rtol=2 ** -8, atol=0)
+
+
+def test_calibration_exponents_bruteforce(oracle_mod):
+    rng = np.random.default_rng(9)
+    X, idx = synth.outlier_activations(rng, 32, 512)
+    Xf = synth.bf16_bits_to_f32(X)
+    X2 = X.copy()
+    X2[:, 7] = 0          # an all-zero channel
+    for Xb in (X, X2):
+        shift, rho = oracle_mod.preshift_calibrate(Xb)
+        c = np.max(np.abs(synth.bf16_bits_to_f32(Xb)), axis=0)
+        assert rho == np.max(c)
+        for k in range(Xb.shape[1]):
+            e = int(shift[k])
+            assert -126 <= e <= 0
+            if c[k] == 0:
+                assert e == 0
+                continue
+            r = Fr(float(c[k])) / Fr(float(rho))
+            assert Fr(2) ** (e - 1) < r <= Fr(2) ** e, (k, e, r)
+    # the 50x outlier channels carry the tensor maximum: their shift is 0 or -1
+    assert np.all(shift[idx] >= -1)
+
+
+def test_preshift_apply_matches_float32_steps(oracle_mod):
+    rng = np.random.default_rng(10)
+    X, _ = synth.outlier_activations(rng, 8, 256)
+    shift, rho = oracle_mod.preshift_calibrate(X)
+    Xt = oracle_mod.preshift_apply(X, shift, rho)
+    x = synth.bf16_bits_to_f32(X)
+    y = (x * np.ldexp(np.float32(1), -shift.astype(np.int32)).astype(np.float32)).astype(np.float32)
+    z = (y / np.float32(rho)).astype(np.float32)
+    assert np.array_equal(Xt, synth.to_bf16_bits(z))
+
+
+def test_calibrate_all_zero_rho_one(oracle_mod):
+    shift, rho = oracle_mod.preshift_calibrate(np.zeros((4, 64), np.uint16))
+    assert rho == 1.0 and np.all(shift == 0)
+
+
+# -------------------------------------------------------------------------- GEMM
+
+@pytest.mark.parametrize("fmt,sdt", [(1, "f32"), (1, "f16"), (0, "f16"), (2, "f16")])
+def test_gemm_matches_torch_fp64(oracle_mod, fmt, sdt):
+    """Oracle GEMM == torch.matmul in fp64 on an independently dequantized W."""
+    W, X = synth.random_case(13, 40, 384, 5)
+    packed, scales, _ = oracle_mod.quantize_fixed(W, 128, fmt, 0, None, sdt)
+    What = dequant_independent(packed, scales, fmt, 128)
+    assert np.array_equal(oracle_mod.dequantize(packed, scales, fmt, 128), What)
+    x = synth.bf16_bits_to_f32(X).astype(np.float64)
+    ref = torch.matmul(torch.from_numpy(x), torch.from_numpy(What).T).numpy()
+    Y = oracle_mod.gemm(X, packed, scales, fmt, 128)
+    np.testing.assert_allclose(Y, ref, rtol=1e-12, atol=1e-12 * np.max(np.abs(ref)))
+    rho = np.float32(3.25)
+    Y2 = oracle_mod.gemm(X, packed, scales, fmt, 128, rho)
+    np.testing.assert_allclose(Y2, ref * 3.25, rtol=1e-12, atol=1e-12 * np.max(np.abs(ref)))
+    ms = np.array([0, 4, 2], np.int32)
+    ns = np.array([39, 0, 17], np.int32)
+    Ys = oracle_mod.gemm_sampled(X, packed, scales, fmt, 128, ms, ns)
+    assert np.array_equal(Ys, Y[ms, ns])
+
+
+def test_gemm_quantization_error_is_small(oracle_mod):
+    """Sanity: the quantized product stays close to the fp64 product."""
+    W, X = synth.random_case(14, 64, 512, 4)
+    r = oracle_mod.quantize(W, 128, 1)
+    Y = oracle_mod.gemm(X, r["packed"], r["scales"], 1, 128)
+    x = synth.bf16_bits_to_f32(X).astype(np.float64)
+    ref = x @ W.astype(np.float64).T
+    cos = np.sum(Y * ref) / np.linalg.norm(Y) / np.linalg.norm(ref)
+    assert cos > 0.98
+
+
+def test_golden_tiny_digest(oracle_mod):
+    """The tiny workload's oracle outputs match the committed digest."""
+    import hashlib
+    import json
+    d = json.load(open(os.path.join(GOLDEN, "tiny_oracle_digest.json")))
+    case = synth.tiny()
+    r = oracle_mod.quantize(case["W"], 128, 1, False, None, "f32")
+    assert hashlib.sha256(r["packed"].tobytes()).hexdigest() == d["packed_sha256"]
+    assert hashlib.sha256(r["scales"].tobytes()).hexdigest() == d["scales_sha256"]
+    Y = oracle_mod.gemm(case["X"], r["packed"], r["scales"], 1, 128)
+    np.testing.assert_allclose(Y[0, :8], d["y_first8"], rtol=1e-15, atol=0)
