@@ -1,0 +1,472 @@
+"""Benchmark of the FP4 W4A16 decode GEMM on the LLaMA-7B-shaped decode
+workload (three weight matrices 4096x4096, 11008x4096, 4096x11008, E2M1,
+group 128, fp16 scales; activations with M in {1, 8, 16, 64} rows).
+
+One step = the decode sweep: fp4_gemm for every (M, matrix) pair, 12 calls,
+on weights already quantized and resident in HBM.  The metric is weight
+GB/s: packed codes + scales streamed per step / step time (all ranks).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Also measured in the same run and reported under "parts": the quantize
+pass (GB/s), the prefill GEMM at M = 2048 (TFLOP/s) on the LLaMA-7B
+prefill workload with the pre-shift, and the format/bias search on a
+LLaMA-13B-shaped 5120x5120 matrix.  ``--impl reference`` times the CPU
+oracle on a bounded sample of the same workload, in the same unit.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fp4_gemm decode weight-GB/s vs HBM peak; prefill TFLOP/s vs bf16 tensor peak"
+SHAPES = ((4096, 4096), (11008, 4096), (4096, 11008))
+MS = (1, 8, 16, 64)
+GROUP = 128
+
+
+def weight_bytes(N, K, group=GROUP, scale_bytes=2):
+    return N * K // 2 + N * (K // group) * scale_bytes
+
+
+def step_weight_bytes():
+    return sum(weight_bytes(N, K) for (N, K) in SHAPES) * len(MS)
+
+
+def read_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------- distributed
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, value):
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------- our arm
+
+def build_workload(api, torch, copies):
+    """Quantize the three matrices once, then replicate the packed weights
+    into `copies` buffers so that consecutive steps read different memory
+    (total > L2)."""
+    from w4a16_gemm_fp4_b200 import synth
+    cases = synth.llama7b_decode()
+    mats = []
+    for (N, K), case in zip(SHAPES, cases):
+        W = torch.from_numpy(case["W"]).cuda()
+        q = api.quantize(W, GROUP, api.E2M1, False, None, "f16")
+        del W
+        reps = [(q["packed"].clone(), q["scales"].clone()) for _ in range(copies)]
+        xs = {M: torch.from_numpy(case["X"][M].view(np.int16)).cuda().view(torch.bfloat16) for M in MS}
+        mats.append({"N": N, "K": K, "reps": reps, "X": xs})
+    return mats, cases
+
+
+def run_ours(args, world, rank):
+    import torch
+    from w4a16_gemm_fp4_b200 import api, build
+    build.build()
+    api.lib()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peaks = read_peaks()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    per_copy = sum(weight_bytes(N, K) for (N, K) in SHAPES)
+    copies = max(4, int(np.ceil(4 * l2 / per_copy)))
+    mats, cases = build_workload(api, torch, copies)
+    outs = {(i, M): torch.empty((M, m["N"]), dtype=torch.bfloat16, device=dev) for i, m in enumerate(mats)
+            for M in MS}
+    wss = {}
+    for i, m in enumerate(mats):
+        for M in MS:
+            nb = api.gemm_workspace_size(M, m["N"], m["K"])
+            wss[(i, M)] = torch.zeros(max(nb, 16), dtype=torch.uint8, device=dev) if nb else None
+    stream = torch.cuda.current_stream()
+
+    def step(s, events=None):
+        c = s % copies
+        for M in MS:
+            for i, m in enumerate(mats):
+                packed, scales = m["reps"][c]
+                if events is not None:
+                    events[(i, M)][0].record(stream)
+                api.gemm(m["X"][M], packed, scales, api.E2M1, GROUP, out=outs[(i, M)], workspace=wss[(i, M)],
+                         stream=stream)
+                if events is not None:
+                    events[(i, M)][1].record(stream)
+
+    for s in range(args.warmup):
+        step(s)
+    torch.cuda.synchronize()
+    api.device_status(clear=True)
+
+    # timed region: per-launch events inside, outer events around
+    ev = {k: [] for k in outs}
+    per = {}
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for s in range(args.steps):
+        evs = {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for k in outs}
+        step(args.warmup + s, evs)
+        for k in outs:
+            ev[k].append(evs[k])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    ms_local = t0.elapsed_time(t1)
+    ms = max_over_ranks(world, ms_local)
+    st = api.device_status(clear=True)
+    if st:
+        raise RuntimeError("device status %#x during the timed region" % st)
+    for k, lst in ev.items():
+        per[k] = sum(a.elapsed_time(b) for a, b in lst) / len(lst)
+
+    total_bytes = step_weight_bytes() * args.steps * world
+    value = total_bytes / (ms * 1e-3) / 1e9
+
+    # dominant kernel (largest share of the step): roofline
+    groups = {}
+    for (i, M), t in per.items():
+        eng = "decode" if M <= 8 else "tensor"
+        g = groups.setdefault((eng, M), {"ms": 0.0, "bytes": 0.0, "launches": 0})
+        N, K = mats[i]["N"], mats[i]["K"]
+        g["ms"] += t
+        g["bytes"] += weight_bytes(N, K) + M * K * 2 + M * N * 2
+        g["launches"] += 1
+    dom = max(groups.items(), key=lambda kv: kv[1]["ms"])
+    (eng, Mdom), g = dom
+    achieved = g["bytes"] / (g["ms"] * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                "kernel": "gemm_%s_kernel (M=%d, 3 matrices)" % ("decode" if eng == "decode" else "tc", Mdom),
+                "peak_source": peaks["source"]}
+    per_m = {}
+    for (eng_, M), gg in sorted(groups.items(), key=lambda kv: kv[0][1]):
+        per_m[str(M)] = {"engine": eng_, "us_per_3_matrices": round(gg["ms"] * 1e3, 2),
+                         "weight_gbs": round(sum(weight_bytes(N, K) for (N, K) in SHAPES) / (gg["ms"] * 1e-3) / 1e9,
+                                             1)}
+
+    # e2e: activations copied from pinned host memory each step, outputs read back
+    e2e = run_e2e(api, torch, mats, args, stream, world)
+
+    parts = {}
+    if not args.no_parts and rank == 0:
+        parts = run_parts(api, torch, peaks, dev)
+    return {
+        "value": value, "ms_per_step": ms / args.steps, "roofline": roofline, "clocks": clk, "e2e": e2e,
+        "gpu_launches": len(outs) * args.steps, "per_m": per_m, "parts": parts, "copies": copies,
+        "copy_bytes": per_copy * copies, "l2_bytes": l2,
+    }
+
+
+def run_e2e(api, torch, mats, args, stream, world):
+    """Same sweep through the public API with host buffers: every step
+    copies X (pinned) to the device and reads every Y back."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    hx, hy, dx, dy = {}, {}, {}, {}
+    h2d = d2h = 0
+    for i, m in enumerate(mats):
+        for M in MS:
+            hx[(i, M)] = m["X"][M].cpu().pin_memory()
+            hy[(i, M)] = torch.empty((M, m["N"]), dtype=torch.bfloat16).pin_memory()
+            dx[(i, M)] = torch.empty_like(m["X"][M])
+            dy[(i, M)] = torch.empty((M, m["N"]), dtype=torch.bfloat16, device=dev)
+            h2d += hx[(i, M)].numel() * 2
+            d2h += hy[(i, M)].numel() * 2
+
+    def step(s):
+        c = s % len(mats[0]["reps"])
+        for M in MS:
+            for i, m in enumerate(mats):
+                dx[(i, M)].copy_(hx[(i, M)], non_blocking=True)
+                packed, scales = m["reps"][c]
+                api.gemm(dx[(i, M)], packed, scales, api.E2M1, GROUP, out=dy[(i, M)], stream=stream)
+                hy[(i, M)].copy_(dy[(i, M)], non_blocking=True)
+
+    for s in range(args.warmup):
+        step(s)
+    torch.cuda.synchronize()
+    barrier(world)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for s in range(args.steps):
+        step(s)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(world, t0.elapsed_time(t1))
+    v = step_weight_bytes() * args.steps * world / (ms * 1e-3) / 1e9
+    return {"value": round(v, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def time_fn(torch, fn, iters, warm=3):
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(iters):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / iters
+
+
+def run_parts(api, torch, peaks, dev):
+    from w4a16_gemm_fp4_b200 import synth
+    out = {}
+    # quantize pass (E2M1, group 128, fp16 scales) over the three decode matrices
+    rng = np.random.default_rng(1)
+    Ws = [torch.from_numpy(synth.lognormal_row_weights(rng, N, K)).cuda() for (N, K) in SHAPES]
+    outs = [api.quantize(W, GROUP, api.E2M1) for W in Ws]
+
+    def qpass():
+        for W, o in zip(Ws, outs):
+            api.quantize_into(W, o["packed"], o["scales"], o["choice"], GROUP, api.E2M1)
+    ms = time_fn(torch, qpass, 10)
+    qbytes = sum(N * K * 4 + weight_bytes(N, K) for (N, K) in SHAPES)
+    out["quantize"] = {"workload": "3 LLaMA-7B decode matrices, E2M1 g128 fp16 scales", "ms": round(ms, 4),
+                       "gbs": round(qbytes / (ms * 1e-3) / 1e9, 1),
+                       "frac_hbm": round(qbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
+    del Ws, outs
+    # prefill with the pre-shift: calibrate + apply + GEMM M = 2048 on 4096x4096 and 11008x4096
+    case = synth.llama7b_prefill()
+    X = torch.from_numpy(case["X"].view(np.int16)).cuda().view(torch.bfloat16)
+    shift, rho = api.preshift_calibrate(X)
+    Xt = api.preshift_apply(X, shift, rho)
+    qs = [api.quantize(torch.from_numpy(W).cuda(), GROUP, api.E2M1, False, shift) for W in case["W"]]
+    ys = [torch.empty((X.shape[0], W.shape[0]), dtype=torch.bfloat16, device=dev) for W in case["W"]]
+
+    def prefill():
+        for q, y in zip(qs, ys):
+            api.gemm(Xt, q["packed"], q["scales"], api.E2M1, GROUP, x_scale=rho, out=y)
+    ms = time_fn(torch, prefill, 10)
+    flops = sum(2.0 * X.shape[0] * N * K for (N, K) in ((4096, 4096), (11008, 4096)))
+    tf = flops / (ms * 1e-3) / 1e12
+    out["prefill"] = {"workload": "LLaMA-7B prefill X 2048x4096 (1% outlier channels x50), pre-shift on",
+                      "ms": round(ms, 4), "tflops": round(tf, 1), "peak_tflops": peaks["bf16_tflops"],
+                      "frac": round(tf / peaks["bf16_tflops"], 4)}
+    ms_pro = time_fn(torch, lambda: api.preshift_apply(X, shift, rho, out=Xt), 10)
+    out["preshift_apply"] = {"ms": round(ms_pro, 4),
+                             "gbs": round(2 * 2 * X.numel() / (ms_pro * 1e-3) / 1e9, 1)}
+    del X, Xt, qs, ys
+    # format / bias search on 5120x5120 Student-t weights
+    W = torch.from_numpy(synth.student_t_weights(np.random.default_rng(3), 5120, 5120)).cuda()
+    ms = time_fn(torch, lambda: api.quantize(W, GROUP, api.AUTO, True), 3, warm=1)
+    out["search"] = {"workload": "5120x5120 Student-t(5)*0.015, 3 formats x 8 bias candidates + pack",
+                     "ms": round(ms, 3), "candidate_evals_per_s": round(24 * W.numel() / (ms * 1e-3), 0)}
+    return out
+
+
+# ----------------------------------------------------------- CPU oracle
+
+def oracle_sample(budget_s=12.0):
+    """Time the CPU oracle (fp64 GEMM on dequantized weights) over the
+    decode sweep, matrix by matrix and M by M, until the budget is spent.
+    Returns (weight GB/s in the step's unit, cores, description)."""
+    import oracle
+    from w4a16_gemm_fp4_b200 import synth
+    oracle.build()
+    cores = oracle.num_threads()
+    cases = synth.llama7b_decode()
+    quant = [oracle.quantize(c["W"], GROUP, oracle.E2M1) for c in cases]
+    done_bytes = 0
+    t_total = 0.0
+    done = []
+    for M in MS:
+        for (N, K), c, q in zip(SHAPES, cases, quant):
+            t0 = time.perf_counter()
+            oracle.gemm(c["X"][M], q["packed"], q["scales"], oracle.E2M1, GROUP)
+            dt = time.perf_counter() - t0
+            t_total += dt
+            done_bytes += weight_bytes(N, K)
+            done.append("%dx%d@M=%d" % (N, K, M))
+            if t_total >= budget_s:
+                break
+        if t_total >= budget_s:
+            break
+    gbs = done_bytes / t_total / 1e9
+    return gbs, cores, "oracle fp64 GEMM on %d of 12 sweep calls (%s), %.1f s" % (len(done), ", ".join(done),
+                                                                                   t_total)
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    import oracle
+    oracle.build()
+    # each step is one bounded sample of the sweep
+    vals = []
+    desc = ""
+    cores = 1
+    for s in range(args.warmup + args.steps):
+        gbs, cores, desc = oracle_sample(budget_s=4.0)
+        if s >= args.warmup:
+            vals.append(gbs)
+    v = statistics.median(vals)
+    return {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_weight_bytes() / (v * 1e9) * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded PCG64 draws standing in for LLaMA-7B weights/activations)",
+            "config": {"workload": "llama7b_decode: W 4096x4096, 11008x4096, 4096x11008 E2M1 g128 fp16 "
+                                   "scales; M in {1,8,16,64}", "l2": "n/a (CPU)"},
+            "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc},
+            "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-parts", action="store_true", help="skip the quantize/prefill/search legs")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        line = run_reference(args, world, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    world, rank, local = dist_setup(args)
+    res = run_ours(args, world, rank)
+    if rank == 0:
+        cpu = None
+        if not args.no_cpu_baseline:
+            gbs, cores, desc = oracle_sample()
+            cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc}
+        line = {
+            "metric": METRIC, "value": round(res["value"], 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(res["ms_per_step"], 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded PCG64 draws standing in for LLaMA-7B weights/activations)",
+            "config": {"workload": "llama7b_decode: W 4096x4096, 11008x4096, 4096x11008 E2M1 g128 fp16 scales; "
+                                   "M in {1,8,16,64}; one step = 12 fp4_gemm calls",
+                       "global_batch": sum(MS), "parallelism": "replicas" if world > 1 else "single",
+                       "l2": "weights rotate over %d copies (%.0f MB) > 4x L2 (%d MB)" % (
+                           res["copies"], res["copy_bytes"] / 1e6, res["l2_bytes"] // 2 ** 20)},
+            "roofline": res["roofline"], "cpu_baseline": cpu, "e2e": res["e2e"], "gpu_launches": res["gpu_launches"],
+            "clocks": res["clocks"], "per_m": res["per_m"], "parts": res["parts"],
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,210 @@
+/*
+ * fp4w4a16.h -- C interface of the B200 (sm_100a) FP4 weight-quantization
+ * and W4A16 GEMM library (libfp4w4a16.so).
+ *
+ * Method: 4-bit floating-point (ExMy) post-training quantization of linear
+ * layer weights and the matrix multiply that consumes them, as described on
+ * the LLM-FP4 summary page "首个支持4-bit浮点量化的LLM来了" (sections on the
+ * floating-point number formula, scale-and-clip, compare-and-quantize, the
+ * efficient matrix multiplication, the format/range search, and the
+ * pre-shifted exponent bias) with two codes packed per byte as in the
+ * "为什么我们需要4-bit浮点量化" tutorial, section 2.2.
+ *
+ * Conventions for every entry point:
+ *  - Tensor arguments are DEVICE pointers allocated and owned by the caller.
+ *    The library never allocates or frees device memory; scratch space is
+ *    passed in as `workspace`.
+ *  - Layouts are row-major and contiguous.  bf16 and fp16 tensors are passed
+ *    as uint16_t bit patterns.  Tensor base pointers must be 16-byte
+ *    aligned (FP4_ERR_MISALIGNED otherwise); scale arrays 4-byte aligned.
+ *  - Argument errors are detected on the host before anything is launched
+ *    and returned synchronously; nothing is written in that case.
+ *  - Work is enqueued on `stream` and is asynchronous; a launch failure
+ *    returns FP4_ERR_CUDA.  Problems only the GPU can see (a non-finite
+ *    input, an fp16 scale overflow, a pipeline wait that timed out) set bits
+ *    of a per-device status word read by fp4_get_device_status().
+ *  - Empty problems (a zero dimension) succeed without launching, except
+ *    that fp4_gemm with K == 0 writes zeros to Y.
+ *  - Weight layouts produced by fp4_quantize and read by fp4_gemm:
+ *      packed [N][K/2] uint8: element k of row n is nibble (k & 1) of byte
+ *                             k/2, low nibble first (even k in bits 0..3);
+ *      scales [N][K/group]    fp32 or fp16, one per (row, group of `group`
+ *                             consecutive k).
+ *    Code = sign<<3 | exponent<<m | mantissa; magnitude index = code & 7.
+ */
+#ifndef FP4W4A16_H
+#define FP4W4A16_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define FP4_API __attribute__((visibility("default")))
+#else
+#define FP4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum fp4_status {
+    FP4_OK = 0,
+    FP4_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad enum  */
+    FP4_ERR_UNSUPPORTED_SHAPE = 2, /* K % group, K % 32, group not 32/64/128 */
+    FP4_ERR_MISALIGNED = 3,        /* a tensor pointer is not 16-byte aligned */
+    FP4_ERR_WORKSPACE = 4,         /* workspace missing or too small          */
+    FP4_ERR_CUDA = 5,              /* a CUDA call or launch failed            */
+    FP4_ERR_DEVICE_STATUS = 6      /* fp4_get_device_status found a flag set  */
+} fp4_status;
+
+/* 4-bit formats (exponent bits / mantissa bits, bias 2^(e-1)-1):
+ *   E1M2 {0,.5,1,1.5,2,2.5,3,3.5}   E2M1 {0,.5,1,1.5,2,3,4,6}
+ *   E3M0 {0,.25,.5,1,2,4,8,16}  (magnitudes of codes 0..7; codes 8..15 are
+ *   the negatives).  FP4_FMT_AUTO asks fp4_quantize to search the format. */
+typedef enum fp4_format { FP4_E1M2 = 0, FP4_E2M1 = 1, FP4_E3M0 = 2, FP4_FMT_AUTO = -1 } fp4_format;
+
+typedef enum fp4_scale_dtype { FP4_SCALE_F32 = 0, FP4_SCALE_F16 = 1 } fp4_scale_dtype;
+
+/* GEMM engine selection for fp4_gemm_ex (fp4_gemm always uses AUTO). */
+typedef enum fp4_engine { FP4_ENGINE_AUTO = 0, FP4_ENGINE_DECODE = 1, FP4_ENGINE_TENSOR = 2 } fp4_engine;
+
+/* Bits of the device status word. */
+#define FP4_DEV_NONFINITE_INPUT 0x1 /* NaN/Inf met in W or X                   */
+#define FP4_DEV_SCALE_OVERFLOW 0x2  /* a group scale does not fit in fp16       */
+#define FP4_DEV_WAIT_TIMEOUT 0x4    /* a pipeline wait gave up; output invalid  */
+
+/* Version of this interface (major * 100 + minor). */
+FP4_API int fp4_abi_version(void);
+
+/* Human-readable name of a status code (static string). */
+FP4_API const char *fp4_status_string(fp4_status s);
+
+/* ------------------------------------------------------------------------
+ * fp4_quantize -- scale-and-clip, optional format / range search,
+ * compare-and-quantize, pack.  (LLM-FP4 summary page: scale-and-clip,
+ * eq. (2)-(4); compare-and-quantize, eq. (5); format and range search;
+ * pre-shifted exponent bias folded into the weights.)
+ *
+ * For every row n and group gi of `group` consecutive k:
+ *   W'[n,k] = W[n,k] * 2^chan_shift[k]            (chan_shift NULL: W' = W)
+ *   A       = max |W'| over the group              (fp32)
+ *   s       = R(fl32(fl32(A * c_j) / Qmax_f))      R = identity (fp32 scales)
+ *                                                  or fp16 round-to-nearest-even
+ *   c_j     = fl32(2^(-j/8)), j = 0..7: a real-valued exponent bias acting as
+ *             a scale (j = 0 is plain absmax scaling)
+ *   code    = signbit(W') << 3 | nearest magnitude index of fl32(|W'| / s),
+ *             ties to the even index, saturating at index 7; s == 0 gives
+ *             index 0.
+ * Search: the candidates are formats {fmt} (or all three if fmt ==
+ * FP4_FMT_AUTO) times j in {0} (or 0..7 if bias_search != 0).  The chosen
+ * candidate minimises SSE = sum (W' - v*s)^2 over the whole tensor (fp64);
+ * the first strict minimum in (format, j) order wins.
+ *
+ *   W          [N][K] fp32, device.
+ *   group      32, 64 or 128; K % group == 0 and K % 32 == 0.
+ *   chan_shift [K] int8 device (values in [-126, 0]) or NULL.
+ *   sdt        scale storage type.
+ *   packed     [N][K/2] uint8 out.   scales [N][K/group] fp32/fp16 out.
+ *   choice     device int32[2] out: {format, j}.  Required.
+ *   sse        device double[24] out or NULL: SSE of candidate f*8+j for the
+ *              candidates evaluated; NaN for the others.
+ *   workspace  device scratch of fp4_quantize_workspace_size(...) bytes
+ *              (may be NULL when that size is 0).  Its contents need no
+ *              initialisation and are undefined afterwards.
+ * Device status: FP4_DEV_NONFINITE_INPUT, FP4_DEV_SCALE_OVERFLOW.
+ * ---------------------------------------------------------------------- */
+FP4_API size_t fp4_quantize_workspace_size(int N, int K, int group, fp4_format fmt, int bias_search);
+FP4_API fp4_status fp4_quantize(const float *W, int N, int K, int group, fp4_format fmt, int bias_search,
+                        const int8_t *chan_shift, fp4_scale_dtype sdt, uint8_t *packed, void *scales,
+                        int32_t *choice, double *sse, void *workspace, size_t ws_bytes,
+                        cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * fp4_dequantize -- W_hat[n,k] = fl32(v(code[n,k]) * s[n, k/group]), the
+ * weights the GEMM multiplies by (test aid).  W_hat [N][K] fp32 out.
+ * ---------------------------------------------------------------------- */
+FP4_API fp4_status fp4_dequantize(const uint8_t *packed, const void *scales, fp4_scale_dtype sdt,
+                          fp4_format fmt, int N, int K, int group, float *W_hat, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Pre-shifted exponent bias (LLM-FP4 summary page, section on the
+ * pre-shifted exponent bias): a per-channel activation maximum from
+ * calibration data is split into one per-tensor real factor rho times a
+ * per-channel power of two 2^e_k; 2^e_k is folded into the weights
+ * (pass it as chan_shift to fp4_quantize), rho stays with the activations.
+ *
+ * fp4_preshift_calibrate:
+ *   c_k = max_m |X[m,k]|, rho = max_k c_k (1 if X is all zero),
+ *   e_k = ceil(log2(c_k / rho)) clamped to [-126, 0], 0 when c_k == 0.
+ *   X [M][K] bf16; shift [K] int8 out; rho device float out.
+ *   workspace: fp4_preshift_workspace_size(M, K) bytes, no initialisation.
+ *   Device status: FP4_DEV_NONFINITE_INPUT.
+ * fp4_preshift_apply:
+ *   Xt[m,k] = bf16_rne(fl32(fl32(X[m,k] * 2^-e_k) / rho)), |Xt| <= 1.
+ *   Xt may not alias X.  The GEMM then takes x_scale = rho.
+ * ---------------------------------------------------------------------- */
+FP4_API size_t fp4_preshift_workspace_size(int M, int K);
+FP4_API fp4_status fp4_preshift_calibrate(const uint16_t *X, int M, int K, int8_t *shift, float *rho,
+                                  void *workspace, size_t ws_bytes, cudaStream_t stream);
+FP4_API fp4_status fp4_preshift_apply(const uint16_t *X, int M, int K, const int8_t *shift, const float *rho,
+                              uint16_t *Xt, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * fp4_gemm -- Y = bf16( x_scale * X . dequant(W)^T ), fp32 accumulation.
+ * (LLM-FP4 summary page, efficient matrix multiplication: the per-group
+ * scales are applied outside the 4-bit products.)
+ *
+ *   Y[m,n] = bf16_rne( rho * sum_k X[m,k] * v(code[n,k]) * s[n, k/group] )
+ *
+ *   X        [M][K] bf16 device.   packed/scales as written by fp4_quantize.
+ *   fmt      the format the weights were quantized in (not AUTO).
+ *   x_scale  device float (rho from fp4_preshift_calibrate) or NULL for 1.
+ *   Y        [M][N] bf16 out; must not alias the inputs.
+ *   workspace device scratch of fp4_gemm_workspace_size(M, N, K) bytes.  It
+ *            must be ZERO-FILLED before its first use; every call leaves it
+ *            ready for the next one.  Calls that may run concurrently need
+ *            separate workspaces.  NULL (with ws_bytes 0) is accepted and
+ *            disables split-K, which is slower for skinny problems.
+ * Engines: M <= 8 uses the decode engine (streams the packed weights with
+ * 128-bit loads, dequantizes in registers, warp-level MMAs); larger M uses
+ * the tensor engine (TMA-staged tiles, tcgen05 MMAs into tensor memory).
+ * Device status: FP4_DEV_WAIT_TIMEOUT.
+ * ---------------------------------------------------------------------- */
+FP4_API size_t fp4_gemm_workspace_size(int M, int N, int K);
+FP4_API fp4_status fp4_gemm(const uint16_t *X, const uint8_t *packed, const void *scales,
+                    fp4_scale_dtype sdt, fp4_format fmt, int M, int N, int K, int group,
+                    const float *x_scale, uint16_t *Y, void *workspace, size_t ws_bytes,
+                    cudaStream_t stream);
+
+/* fp4_gemm with an explicit engine and split-K count (0 = automatic);
+ * meant for tests and tuning.  The decode engine accepts M <= 8 only. */
+FP4_API fp4_status fp4_gemm_ex(const uint16_t *X, const uint8_t *packed, const void *scales,
+                       fp4_scale_dtype sdt, fp4_format fmt, int M, int N, int K, int group,
+                       const float *x_scale, uint16_t *Y, void *workspace, size_t ws_bytes,
+                       fp4_engine engine, int splits, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * fp4_get_device_status -- synchronises `stream`, copies the current
+ * device's status word (FP4_DEV_* bits) to *host_code and, when `clear` is
+ * non-zero, resets it.  Returns FP4_ERR_DEVICE_STATUS when a bit is set.
+ * ---------------------------------------------------------------------- */
+FP4_API fp4_status fp4_get_device_status(int32_t *host_code, int clear, cudaStream_t stream);
+
+/* Test knob: bound, in microseconds, of every pipeline wait in the tensor
+ * engine (default 2,000,000).  Values < 1 restore the default.  A test sets
+ * it small to check that a wait which cannot complete reports
+ * FP4_DEV_WAIT_TIMEOUT instead of hanging. */
+FP4_API void fp4_set_wait_timeout_us(long long us);
+
+/* Failure-detection check: launches one CTA that waits, with the bound
+ * timeout_us (1 .. 10,000,000), on a barrier nothing arrives on.  The wait
+ * must give up and set FP4_DEV_WAIT_TIMEOUT; no fault, trap or hang.  The
+ * page has no counterpart: this only tests the library's bounded waits. */
+FP4_API fp4_status fp4_selftest_bounded_wait(long long timeout_us, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FP4W4A16_H */

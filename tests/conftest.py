@@ -11,6 +11,7 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long-running oracle case")
+    config.addinivalue_line("markers", "expect_status: the test sets device status bits on purpose")
 
 
 @pytest.fixture(scope="session")

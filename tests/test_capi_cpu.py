@@ -1,0 +1,113 @@
+"""Host-side checks of the C interface that need no GPU: the library loads,
+exports every entry point the header declares, and rejects bad arguments
+before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from w4a16_gemm_fp4_b200 import api
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp4w4a16.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from w4a16_gemm_fp4_b200 import build
+    build.build()
+    return api.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^FP4_API\s+[\w\s\*]*?\b(fp4_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_interface():
+    names = declared_functions()
+    assert "fp4_quantize" in names and "fp4_gemm" in names and "fp4_preshift_calibrate" in names
+    assert set(names) == set(api.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    # and they are real dynamic exports, not just resolvable names
+    out = os.popen("nm -D --defined-only %s" % api.LIB_PATH).read()
+    for name in declared_functions():
+        assert re.search(r" T %s$" % name, out, flags=re.M), name
+
+
+def test_version_and_strings(L):
+    assert L.fp4_abi_version() == 100
+    assert L.fp4_status_string(0) == b"ok"
+    assert b"workspace" in L.fp4_status_string(4)
+
+
+FAKE = ctypes.c_void_p(1 << 20)          # 16-byte aligned, never dereferenced
+MIS = ctypes.c_void_p((1 << 20) + 8)     # misaligned
+
+
+def q(L, W=FAKE, N=4, K=128, group=128, fmt=1, bias=0, shift=None, sdt=1, packed=FAKE, scales=FAKE,
+      choice=FAKE, sse=None, ws=None, wsb=0):
+    return L.fp4_quantize(W, N, K, group, fmt, bias, shift, sdt, packed, scales, choice, sse, ws, wsb, None)
+
+
+def test_quantize_argument_errors(L):
+    assert q(L, group=48) == 2
+    assert q(L, K=96, group=64) == 2
+    assert q(L, N=-1) == 1
+    assert q(L, fmt=3) == 1
+    assert q(L, fmt=-2) == 1
+    assert q(L, sdt=2) == 1
+    assert q(L, choice=None) == 1
+    assert q(L, W=None) == 1
+    assert q(L, W=MIS) == 3
+    assert q(L, packed=MIS) == 3
+    assert q(L, shift=MIS) == 3
+    # search needs a workspace
+    assert q(L, fmt=-1, bias=1) == 4
+    need = L.fp4_quantize_workspace_size(4, 128, 128, -1, 1)
+    assert need > 0
+    assert q(L, fmt=-1, bias=1, ws=FAKE, wsb=need - 8) == 4
+
+
+def test_gemm_argument_errors(L):
+    Xp, Pp, Sp, Yp = (ctypes.c_void_p(a << 20) for a in (1, 2, 3, 4))
+
+    def g(X=Xp, packed=Pp, scales=Sp, sdt=1, fmt=1, M=4, N=64, K=256, group=128, Y=Yp, engine=0,
+          splits=0):
+        return L.fp4_gemm_ex(X, packed, scales, sdt, fmt, M, N, K, group, None, Y, None, 0, engine, splits, None)
+    assert g(group=256) == 2
+    assert g(K=192) == 2
+    assert g(fmt=-1) == 1
+    assert g(M=-1) == 1
+    assert g(Y=None) == 1
+    assert g(X=MIS) == 3
+    assert g(Y=MIS) == 3
+    assert g(engine=7) == 1
+    assert g(splits=-1) == 1
+    assert g(M=9, engine=1) == 2          # decode engine takes M <= 8
+    assert g(Y=Xp) == 1                   # output aliases the input
+    # empty problems succeed without touching the device
+    assert g(M=0) == 0
+    assert g(N=0) == 0
+
+
+def test_preshift_argument_errors(L):
+    assert L.fp4_preshift_calibrate(FAKE, 4, 12, FAKE, FAKE, FAKE, 1 << 20, None) == 2
+    assert L.fp4_preshift_calibrate(FAKE, 4, 64, FAKE, None, FAKE, 1 << 20, None) == 1
+    assert L.fp4_preshift_calibrate(FAKE, 4, 64, FAKE, FAKE, None, 0, None) == 4
+    assert L.fp4_preshift_apply(FAKE, 4, 64, FAKE, FAKE, FAKE, None) == 1   # in place
+    assert L.fp4_preshift_apply(FAKE, 4, 64, FAKE, FAKE, MIS, None) == 3
+    assert L.fp4_preshift_apply(FAKE, 0, 64, FAKE, FAKE, FAKE, None) == 0
+
+
+def test_workspace_sizes(L):
+    assert L.fp4_gemm_workspace_size(1, 4096, 4096) == 0        # decode engine: none
+    assert L.fp4_gemm_workspace_size(64, 4096, 4096) > 0        # skinny tensor problem: split-K
+    assert L.fp4_gemm_workspace_size(2048, 4096, 4096) == 0     # enough tiles: no split
+    assert L.fp4_quantize_workspace_size(4096, 4096, 128, 1, 0) >= 8
+    assert L.fp4_preshift_workspace_size(2048, 4096) >= 4096 * 4

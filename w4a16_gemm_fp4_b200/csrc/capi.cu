@@ -1,0 +1,293 @@
+// capi.cu -- the extern "C" entry points of libfp4w4a16.so: argument
+// validation (before anything is launched), the per-format value tables,
+// engine dispatch and the per-device status word.  See include/fp4w4a16.h
+// for the contract of each call.
+#include <math.h>
+#include <stdio.h>
+
+#include "common.cuh"
+
+namespace fp4 {
+// kernels (quantize.cu, preshift.cu, gemm_decode.cu, gemm_tc.cu)
+size_t quantize_ws_bytes(long long total, bool search, bool want_sse);
+cudaError_t launch_quantize(const float* W, int N, int K, int group, int fmt, int bias_search,
+                            const int8_t* shift, int sdt, uint8_t* packed, void* scales, int32_t* choice,
+                            double* sse, void* ws, const FmtTables& tabs, int* status, cudaStream_t st);
+cudaError_t launch_dequantize(const uint8_t* packed, const void* scales, int sdt, const FmtTable& t, int N, int K,
+                              int group, float* out, cudaStream_t st);
+size_t preshift_ws_bytes(int M, int K);
+cudaError_t launch_calibrate(const uint16_t* X, int M, int K, int8_t* shift, float* rho, void* ws, int* status,
+                             cudaStream_t st);
+cudaError_t launch_apply(const uint16_t* X, int M, int K, const int8_t* shift, const float* rho, uint16_t* Xt,
+                         cudaStream_t st);
+cudaError_t launch_gemm_decode(const uint16_t* X, const uint8_t* packed, const void* scales, int sdt,
+                               const FmtTable& t, int M, int N, int K, int group, const float* x_scale,
+                               uint16_t* Y, cudaStream_t st);
+size_t tc_ws_bytes(int M, int N, int K);
+cudaError_t launch_gemm_tc(const uint16_t* X, const uint8_t* packed, const void* scales, int sdt, const FmtTable& t,
+                           int M, int N, int K, int group, const float* x_scale, uint16_t* Y, void* ws,
+                           size_t ws_bytes, int splits, int* status, unsigned long long timeout_ns,
+                           cudaStream_t st);
+cudaError_t launch_bounded_wait_probe(int* status, unsigned long long timeout_ns, cudaStream_t st);
+}  // namespace fp4
+
+using namespace fp4;
+
+// The status word lives in this module; each device holds its own copy.
+__device__ int g_fp4_status;
+
+namespace {
+
+constexpr int kDecodeMaxM = 8;
+constexpr int kMaxDevices = 64;
+long long g_timeout_us = 2000000;
+
+// Value of magnitude index i (code & 7) of the format with e exponent and m
+// mantissa bits and bias b = 2^(e-1) - 1: exponent field p = i >> m,
+// mantissa d = i & (2^m - 1); p == 0 is the subnormal binade.
+float magnitude(int e, int m, int i) {
+    const int b = (1 << (e - 1)) - 1;
+    const int p = i >> m, d = i & ((1 << m) - 1);
+    if (p == 0) return ldexpf((float)d, 1 - b - m);
+    return ldexpf((float)((1 << m) + d), p - b - m);
+}
+
+const FmtTables& tables() {
+    static FmtTables T;
+    static bool init = false;
+    if (!init) {
+        const int em[3][2] = {{1, 2}, {2, 1}, {3, 0}};
+        for (int f = 0; f < 3; ++f) {
+            for (int i = 0; i < 8; ++i) T.f[f].mag[i] = magnitude(em[f][0], em[f][1], i);
+            for (int i = 0; i < 7; ++i) T.f[f].mid[i] = 0.5f * (T.f[f].mag[i] + T.f[f].mag[i + 1]);
+            T.f[f].qmax = T.f[f].mag[7];
+        }
+        for (int j = 0; j < 8; ++j) T.cj[j] = (float)exp2(-(double)j / 8.0);
+        init = true;
+    }
+    return T;
+}
+
+int* status_ptr() {
+    static int* ptrs[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    if (!ptrs[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_fp4_status) != cudaSuccess) return nullptr;
+        ptrs[dev] = reinterpret_cast<int*>(p);
+    }
+    return ptrs[dev];
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+fp4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA; }
+
+fp4_status check_group(int K, int group) {
+    if (group != 32 && group != 64 && group != 128) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if (K % group != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
+    return FP4_OK;
+}
+
+fp4_status check_weights(const uint8_t* packed, const void* scales, fp4_scale_dtype sdt, fp4_format fmt, int N,
+                         int K, int group) {
+    if (N < 0 || K < 0) return FP4_ERR_INVALID_ARG;
+    if (fmt < FP4_E1M2 || fmt > FP4_E3M0) return FP4_ERR_INVALID_ARG;
+    if (sdt != FP4_SCALE_F32 && sdt != FP4_SCALE_F16) return FP4_ERR_INVALID_ARG;
+    fp4_status s = check_group(K, group);
+    if (s != FP4_OK) return s;
+    if ((long long)N * K > 0) {
+        if (!packed || !scales) return FP4_ERR_INVALID_ARG;
+        if (!aligned(packed, 16) || !aligned(scales, 4)) return FP4_ERR_MISALIGNED;
+    }
+    return FP4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fp4_abi_version(void) { return 100; }
+
+const char* fp4_status_string(fp4_status s) {
+    switch (s) {
+        case FP4_OK: return "ok";
+        case FP4_ERR_INVALID_ARG: return "invalid argument";
+        case FP4_ERR_UNSUPPORTED_SHAPE: return "unsupported shape (group must be 32/64/128 and divide K)";
+        case FP4_ERR_MISALIGNED: return "tensor pointer not 16-byte aligned";
+        case FP4_ERR_WORKSPACE: return "workspace missing or too small";
+        case FP4_ERR_CUDA: return "CUDA error";
+        case FP4_ERR_DEVICE_STATUS: return "device status flag set";
+    }
+    return "unknown status";
+}
+
+void fp4_set_wait_timeout_us(long long us) { g_timeout_us = us < 1 ? 2000000 : us; }
+
+size_t fp4_quantize_workspace_size(int N, int K, int group, fp4_format fmt, int bias_search) {
+    (void)group;
+    if (N <= 0 || K <= 0) return 0;
+    const bool search = fmt == FP4_FMT_AUTO || bias_search != 0;
+    return quantize_ws_bytes((long long)N * K, search, true);
+}
+
+fp4_status fp4_quantize(const float* W, int N, int K, int group, fp4_format fmt, int bias_search,
+                        const int8_t* chan_shift, fp4_scale_dtype sdt, uint8_t* packed, void* scales,
+                        int32_t* choice, double* sse, void* workspace, size_t ws_bytes, cudaStream_t stream) {
+    if (N < 0 || K < 0) return FP4_ERR_INVALID_ARG;
+    if (fmt < FP4_FMT_AUTO || fmt > FP4_E3M0) return FP4_ERR_INVALID_ARG;
+    if (sdt != FP4_SCALE_F32 && sdt != FP4_SCALE_F16) return FP4_ERR_INVALID_ARG;
+    fp4_status s = check_group(K, group);
+    if (s != FP4_OK) return s;
+    if (!choice) return FP4_ERR_INVALID_ARG;
+    if (!aligned(choice, 4) || (sse && !aligned(sse, 8))) return FP4_ERR_MISALIGNED;
+    const long long total = (long long)N * K;
+    const bool search = fmt == FP4_FMT_AUTO || bias_search != 0;
+    if (total > 0) {
+        if (!W || !packed || !scales) return FP4_ERR_INVALID_ARG;
+        if (!aligned(W, 16) || !aligned(packed, 16) || !aligned(scales, 4)) return FP4_ERR_MISALIGNED;
+        if (chan_shift && !aligned(chan_shift, 16)) return FP4_ERR_MISALIGNED;
+        const size_t need = quantize_ws_bytes(total, search, sse != nullptr);
+        if (need > 0 && (!workspace || ws_bytes < need)) return FP4_ERR_WORKSPACE;
+        if (workspace && !aligned(workspace, 16)) return FP4_ERR_MISALIGNED;
+    }
+    int* st = status_ptr();
+    if (!st) return FP4_ERR_CUDA;
+    if (total == 0) {
+        // nothing to quantize: every candidate has SSE 0, the first one wins
+        const int f = fmt == FP4_FMT_AUTO ? 0 : (int)fmt;
+        const int32_t host_choice[2] = {f, 0};
+        cudaError_t e = cudaMemcpyAsync(choice, host_choice, sizeof(host_choice), cudaMemcpyHostToDevice, stream);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+        if (e == cudaSuccess && sse) {
+            double host_sse[24];
+            const int f1 = fmt == FP4_FMT_AUTO ? 2 : f;
+            const int jn = bias_search ? 8 : 1;
+            for (int ff = 0; ff < 3; ++ff)
+                for (int j = 0; j < 8; ++j) host_sse[ff * 8 + j] = (ff >= f && ff <= f1 && j < jn) ? 0.0 : NAN;
+            e = cudaMemcpyAsync(sse, host_sse, sizeof(host_sse), cudaMemcpyHostToDevice, stream);
+            if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+        }
+        return cuda_status(e);
+    }
+    return cuda_status(launch_quantize(W, N, K, group, (int)fmt, bias_search, chan_shift, (int)sdt, packed, scales,
+                                       choice, sse, workspace, tables(), st, stream));
+}
+
+fp4_status fp4_dequantize(const uint8_t* packed, const void* scales, fp4_scale_dtype sdt, fp4_format fmt, int N,
+                          int K, int group, float* W_hat, cudaStream_t stream) {
+    fp4_status s = check_weights(packed, scales, sdt, fmt, N, K, group);
+    if (s != FP4_OK) return s;
+    if ((long long)N * K == 0) return FP4_OK;
+    if (!W_hat) return FP4_ERR_INVALID_ARG;
+    if (!aligned(W_hat, 16)) return FP4_ERR_MISALIGNED;
+    return cuda_status(launch_dequantize(packed, scales, (int)sdt, tables().f[fmt], N, K, group, W_hat, stream));
+}
+
+size_t fp4_preshift_workspace_size(int M, int K) {
+    if (M <= 0 || K <= 0) return 0;
+    return preshift_ws_bytes(M, K);
+}
+
+fp4_status fp4_preshift_calibrate(const uint16_t* X, int M, int K, int8_t* shift, float* rho, void* workspace,
+                                  size_t ws_bytes, cudaStream_t stream) {
+    if (M < 0 || K < 0) return FP4_ERR_INVALID_ARG;
+    if (K % 8 != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if (!rho || (K > 0 && !shift)) return FP4_ERR_INVALID_ARG;
+    if (!aligned(rho, 4) || (shift && !aligned(shift, 16))) return FP4_ERR_MISALIGNED;
+    if ((long long)M * K == 0) {
+        // rho = 1, every shift 0
+        const float one = 1.0f;
+        cudaError_t e = cudaMemcpyAsync(rho, &one, sizeof(one), cudaMemcpyHostToDevice, stream);
+        if (e == cudaSuccess && K > 0) e = cudaMemsetAsync(shift, 0, (size_t)K, stream);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+        return cuda_status(e);
+    }
+    if (!X) return FP4_ERR_INVALID_ARG;
+    if (!aligned(X, 16)) return FP4_ERR_MISALIGNED;
+    const size_t need = preshift_ws_bytes(M, K);
+    if (!workspace || ws_bytes < need) return FP4_ERR_WORKSPACE;
+    if (!aligned(workspace, 16)) return FP4_ERR_MISALIGNED;
+    int* st = status_ptr();
+    if (!st) return FP4_ERR_CUDA;
+    return cuda_status(launch_calibrate(X, M, K, shift, rho, workspace, st, stream));
+}
+
+fp4_status fp4_preshift_apply(const uint16_t* X, int M, int K, const int8_t* shift, const float* rho, uint16_t* Xt,
+                              cudaStream_t stream) {
+    if (M < 0 || K < 0) return FP4_ERR_INVALID_ARG;
+    if (K % 8 != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if ((long long)M * K == 0) return FP4_OK;
+    if (!X || !shift || !rho || !Xt || X == Xt) return FP4_ERR_INVALID_ARG;
+    if (!aligned(X, 16) || !aligned(Xt, 16) || !aligned(shift, 16) || !aligned(rho, 4)) return FP4_ERR_MISALIGNED;
+    return cuda_status(launch_apply(X, M, K, shift, rho, Xt, stream));
+}
+
+size_t fp4_gemm_workspace_size(int M, int N, int K) {
+    if (M <= 0 || N <= 0 || K <= 0) return 0;
+    if (M <= kDecodeMaxM) return 0;
+    return tc_ws_bytes(M, N, K);
+}
+
+fp4_status fp4_gemm_ex(const uint16_t* X, const uint8_t* packed, const void* scales, fp4_scale_dtype sdt,
+                       fp4_format fmt, int M, int N, int K, int group, const float* x_scale, uint16_t* Y,
+                       void* workspace, size_t ws_bytes, fp4_engine engine, int splits, cudaStream_t stream) {
+    if (M < 0) return FP4_ERR_INVALID_ARG;
+    fp4_status s = check_weights(packed, scales, sdt, fmt, N, K, group);
+    if (s != FP4_OK) return s;
+    if (engine != FP4_ENGINE_AUTO && engine != FP4_ENGINE_DECODE && engine != FP4_ENGINE_TENSOR)
+        return FP4_ERR_INVALID_ARG;
+    if (splits < 0) return FP4_ERR_INVALID_ARG;
+    if ((long long)M * N == 0) return FP4_OK;
+    if (!Y) return FP4_ERR_INVALID_ARG;
+    if (!aligned(Y, 16)) return FP4_ERR_MISALIGNED;
+    if (x_scale && !aligned(x_scale, 4)) return FP4_ERR_MISALIGNED;
+    if (workspace && !aligned(workspace, 16)) return FP4_ERR_MISALIGNED;
+    if (K == 0) return cuda_status(cudaMemsetAsync(Y, 0, (size_t)M * N * sizeof(uint16_t), stream));
+    if (!X) return FP4_ERR_INVALID_ARG;
+    if (!aligned(X, 16)) return FP4_ERR_MISALIGNED;
+    if ((const void*)Y == (const void*)X || (const void*)Y == (const void*)packed) return FP4_ERR_INVALID_ARG;
+    if (engine == FP4_ENGINE_AUTO) engine = M <= kDecodeMaxM ? FP4_ENGINE_DECODE : FP4_ENGINE_TENSOR;
+    const FmtTable& t = tables().f[fmt];
+    if (engine == FP4_ENGINE_DECODE) {
+        if (M > kDecodeMaxM) return FP4_ERR_UNSUPPORTED_SHAPE;
+        return cuda_status(launch_gemm_decode(X, packed, scales, (int)sdt, t, M, N, K, group, x_scale, Y, stream));
+    }
+    int* st = status_ptr();
+    if (!st) return FP4_ERR_CUDA;
+    return cuda_status(launch_gemm_tc(X, packed, scales, (int)sdt, t, M, N, K, group, x_scale, Y, workspace,
+                                      ws_bytes, splits, st, (unsigned long long)g_timeout_us * 1000ull, stream));
+}
+
+fp4_status fp4_gemm(const uint16_t* X, const uint8_t* packed, const void* scales, fp4_scale_dtype sdt,
+                    fp4_format fmt, int M, int N, int K, int group, const float* x_scale, uint16_t* Y,
+                    void* workspace, size_t ws_bytes, cudaStream_t stream) {
+    return fp4_gemm_ex(X, packed, scales, sdt, fmt, M, N, K, group, x_scale, Y, workspace, ws_bytes,
+                       FP4_ENGINE_AUTO, 0, stream);
+}
+
+fp4_status fp4_get_device_status(int32_t* host_code, int clear, cudaStream_t stream) {
+    if (!host_code) return FP4_ERR_INVALID_ARG;
+    int* st = status_ptr();
+    if (!st) return FP4_ERR_CUDA;
+    int v = 0;
+    cudaError_t e = cudaMemcpyAsync(&v, st, sizeof(int), cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e == cudaSuccess && clear) {
+        e = cudaMemsetAsync(st, 0, sizeof(int), stream);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    }
+    if (e != cudaSuccess) return FP4_ERR_CUDA;
+    *host_code = v;
+    return v ? FP4_ERR_DEVICE_STATUS : FP4_OK;
+}
+
+fp4_status fp4_selftest_bounded_wait(long long timeout_us, cudaStream_t stream) {
+    if (timeout_us < 1 || timeout_us > 10000000) return FP4_ERR_INVALID_ARG;
+    int* st = status_ptr();
+    if (!st) return FP4_ERR_CUDA;
+    return cuda_status(launch_bounded_wait_probe(st, (unsigned long long)timeout_us * 1000ull, stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,289 @@
+// common.cuh -- helpers shared by the sm_100a kernels of libfp4w4a16:
+// format tables, the device status word, bf16 nibble dequantization, and
+// thin inline-PTX wrappers for mbarrier, TMA and tcgen05 (tensor memory).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/fp4w4a16.h"
+
+namespace fp4 {
+
+// ------------------------------------------------------------ format table
+// Magnitudes of codes 0..7 of one 4-bit ExMy format (the value formula of
+// the LLM-FP4 summary page: p == 0 subnormal 2^(1-b) * 0.d, otherwise
+// 2^(p-b) * 1.d, bias b = 2^(e-1)-1), their midpoints and Qmax.  Built on
+// the host (capi.cu) and passed to kernels by value.
+struct FmtTable {
+    float mag[8];
+    float mid[7];  // mid[i] = (mag[i] + mag[i+1]) / 2, exact in fp32
+    float qmax;
+};
+
+struct FmtTables {
+    FmtTable f[3];
+    float cj[8];  // fl32(2^(-j/8)): real-valued exponent-bias candidates
+};
+
+// Device status word bits (mirrors FP4_DEV_* of the public header).
+constexpr int kStatusNonfinite = FP4_DEV_NONFINITE_INPUT;
+constexpr int kStatusScaleOverflow = FP4_DEV_SCALE_OVERFLOW;
+constexpr int kStatusTimeout = FP4_DEV_WAIT_TIMEOUT;
+
+__device__ __forceinline__ void raise_status(int* status, int bits) {
+    if (status) atomicOr(status, bits);
+}
+
+// Nearest magnitude index of a = |q| (q = fl32(x / s)): count the
+// midpoints below a; at an exact midpoint mid[i] (between i and i+1) the
+// even index wins.  |q| >= Qmax is index 7 (a > mid[6]).
+__device__ __forceinline__ int nearest_index(float a, const FmtTable& t) {
+    int idx = 0;
+#pragma unroll
+    for (int i = 0; i < 7; ++i) {
+        // strictly above the midpoint -> at least i+1; equal -> i+1 only if
+        // i+1 is even (i odd)
+        idx += (a > t.mid[i]) || ((a == t.mid[i]) && (i & 1));
+    }
+    return idx;
+}
+
+// ---------------------------------------------------- bf16 nibble dequant
+// A 16-entry code -> bf16 table held in four registers as split byte
+// planes: lo0/hi0 = low/high bytes of the bf16 values of magnitude indices
+// 0..3, lo1/hi1 = indices 4..7.  The sign is applied separately, because
+// bf16(-v) differs from bf16(v) only in bit 15.
+struct Bf16Lut {
+    uint32_t lo0, lo1, hi0, hi1;
+};
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// LUT of bf16(mag[i] * s) (s = 1 gives the exact magnitudes).
+__device__ __forceinline__ Bf16Lut make_lut(const float* mag, float s) {
+    uint32_t b01 = pack_bf16x2(__fmul_rn(mag[0], s), __fmul_rn(mag[1], s));
+    uint32_t b23 = pack_bf16x2(__fmul_rn(mag[2], s), __fmul_rn(mag[3], s));
+    uint32_t b45 = pack_bf16x2(__fmul_rn(mag[4], s), __fmul_rn(mag[5], s));
+    uint32_t b67 = pack_bf16x2(__fmul_rn(mag[6], s), __fmul_rn(mag[7], s));
+    Bf16Lut l;
+    l.lo0 = prmt(b01, b23, 0x6420);
+    l.hi0 = prmt(b01, b23, 0x7531);
+    l.lo1 = prmt(b45, b67, 0x6420);
+    l.hi1 = prmt(b45, b67, 0x7531);
+    return l;
+}
+
+// Dequantize one 32-bit word of packed codes (nibble i = element i, low
+// nibble first) into four bf16x2 words p[j] = (elem 2j, elem 2j+1), low
+// half = lower k.  15 integer ops for 8 elements:
+//  - the magnitude index (code & 7) selects a byte of each byte plane;
+//  - prmt in sign-replicate mode (selector bit 3) turns each code's sign bit
+//    into a 0x00/0xFF byte, and bit 7 of it is OR-ed into the high byte.
+__device__ __forceinline__ void dequant8(uint32_t w, const Bf16Lut& l, uint32_t p[4]) {
+    const uint32_t m = w & 0x77777777u;
+    const uint32_t w4 = w << 4;
+    const uint32_t mh = m >> 16;
+    {
+        uint32_t lo = prmt(l.lo0, l.lo1, m);
+        uint32_t hi = prmt(l.hi0, l.hi1, m);
+        uint32_t sg = prmt(w, w4, 0x9D8Cu);  // sign bytes of elements 0..3
+        hi |= sg & 0x80808080u;
+        p[0] = prmt(lo, hi, 0x5140u);
+        p[1] = prmt(lo, hi, 0x7362u);
+    }
+    {
+        uint32_t lo = prmt(l.lo0, l.lo1, mh);
+        uint32_t hi = prmt(l.hi0, l.hi1, mh);
+        uint32_t sg = prmt(w, w4, 0xBFAEu);  // sign bytes of elements 4..7
+        hi |= sg & 0x80808080u;
+        p[2] = prmt(lo, hi, 0x5140u);
+        p[3] = prmt(lo, hi, 0x7362u);
+    }
+}
+
+__device__ __forceinline__ float load_scale(const void* scales, int sdt, size_t idx) {
+    if (sdt == FP4_SCALE_F16) return __half2float(__ldg(reinterpret_cast<const __half*>(scales) + idx));
+    return __ldg(reinterpret_cast<const float*>(scales) + idx);
+}
+
+// ------------------------------------------------------------- PTX: misc
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ uint32_t elect_one() {
+    uint32_t pred = 0;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "elect.sync _|p, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(pred));
+    return pred;
+}
+
+// --------------------------------------------------------- PTX: mbarrier
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.release.cta.shared::cta.b64 st, [%0];\n\t}" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile(
+        "{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.release.cta.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(
+            smem_u32(bar)),
+        "r"(bytes)
+        : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait: returns false (and the caller must give up) after
+// `timeout_ns` of global time.  Every wait in the library goes through here.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 32; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer_ns() - t0 > timeout_ns) return false;
+    }
+}
+
+// -------------------------------------------------------------- PTX: TMA
+// 2D tiled bulk tensor load global -> shared, completion on an mbarrier.
+// No multicast.  c0 = innermost coordinate (elements), c1 = row.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ---------------------------------------------------------- PTX: tcgen05
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16 (bf16 inputs, fp32
+// accumulate).  Issued by one thread.
+__device__ __forceinline__ void tc_mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive on an mbarrier once all previously issued tcgen05.mma of this
+// thread have completed.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+
+// 32 lanes x 32 bit, 16 consecutive columns per thread.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t r[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor, K-major operand with the 128-byte
+// swizzle: rows of 128 B, 8-row atoms of 1024 B stacked at a stride of
+// 1024 B (SBO), base 1024-byte aligned, descriptor version 1.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1u << 16;            // leading byte offset (unused here)
+    d |= (uint64_t)(1024u >> 4) << 32;  // stride byte offset
+    d |= (uint64_t)1u << 46;            // version
+    d |= (uint64_t)2u << 61;            // layout: 128-byte swizzle
+    return d;
+}
+
+// Instruction descriptor: kind::f16, A = B = bf16 (K-major), D = fp32,
+// shape M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
+    return (1u << 4)                       // D format fp32
+           | (1u << 7)                     // A format bf16
+           | (1u << 10)                    // B format bf16
+           | ((uint32_t)(N >> 3) << 17)    // N / 8
+           | ((uint32_t)(M >> 4) << 24);   // M / 16
+}
+
+}  // namespace fp4

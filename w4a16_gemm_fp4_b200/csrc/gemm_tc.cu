@@ -1,0 +1,393 @@
+// gemm_tc.cu -- W4A16 GEMM on the sm_100a tensor cores (tcgen05 + TMEM).
+//
+// Y[m,n] = bf16( rho * sum_k X[m,k] * v(code[n,k]) * s[n, k/g] )
+// (LLM-FP4 summary page "首个支持4-bit浮点量化的LLM来了", efficient matrix
+// multiplication; the group scale is applied while dequantizing, before the
+// bf16 product, so the tensor cores see plain bf16 operands.)
+//
+// CTA tile: 128 weight rows (MMA M) x BT activation rows (MMA N) x 64 k per
+// pipeline stage.  The product is computed transposed, D[n][m] = W . X^T,
+// so the 128 weight rows map onto the 128 TMEM lanes and the dequantizing
+// thread of row r is the thread that owns TMEM lane r.
+//
+// Warp roles (192 threads):
+//   warp 0      TMA producer: X tile (bf16, 128-byte swizzle) and the packed
+//               code tile (uint8 [128][32]) into a ring of smem stages;
+//   warp 1      TMEM allocator and MMA issuer: one thread issues 4
+//               tcgen05.mma (K = 16 each) per stage into an fp32 TMEM
+//               accumulator and commits the stage back to the producer;
+//   warps 2..5  dequantize the stage's codes into a bf16 K-major tile with
+//               the 128-byte swizzle (byte-plane LUT of bf16(v*s), 16-byte
+//               stores), then, after the last stage, run the epilogue:
+//               tcgen05.ld -> * rho -> bf16 -> global (or fp32 split-K
+//               partials, reduced in fixed order by the last CTA of a tile).
+// Every mbarrier wait is bounded; a wait that gives up sets
+// FP4_DEV_WAIT_TIMEOUT in the status word and the CTA winds down normally
+// (outstanding copies awaited, TMEM freed).  No multicast is used.
+#include "common.cuh"
+
+namespace fp4 {
+
+struct TcParams {
+    const void* scales;
+    int sdt;
+    FmtTable t;
+    int M, N, K, group;
+    const float* x_scale;
+    uint16_t* Y;
+    float* part;         // [splits][M][N] fp32 partials (splits > 1)
+    unsigned* counters;  // one per output tile (splits > 1)
+    int splits;
+    int* status;
+    unsigned long long timeout_ns;
+};
+
+template <int BT>
+struct TcCfg {
+    static constexpr int BW = 128;              // weight rows per tile (MMA M)
+    static constexpr int BK = 64;               // k per stage (one 128-byte swizzle row of bf16)
+    static constexpr int XBYTES = BT * 128;     // activation tile
+    static constexpr int WBYTES = BW * 128;     // dequantized weight tile
+    static constexpr int PBYTES = BW * 32;      // packed code tile
+    static constexpr int STAGE = XBYTES + WBYTES + PBYTES;
+    static constexpr int STAGES = (220 * 1024) / STAGE > 8 ? 8 : (220 * 1024) / STAGE;
+    static constexpr int TMEM_COLS = BT < 32 ? 32 : BT;
+    static constexpr int SMEM = STAGES * STAGE + 1024 + 256;
+};
+
+template <int BT>
+__global__ void __launch_bounds__(192, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, TcParams p) {
+    using C = TcCfg<BT>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* xs = smem;                                   // STAGES x XBYTES
+    uint8_t* ws = smem + C::STAGES * C::XBYTES;           // STAGES x WBYTES
+    uint8_t* ps = ws + C::STAGES * C::WBYTES;             // STAGES x PBYTES
+    uint64_t* bars = reinterpret_cast<uint64_t*>(ps + C::STAGES * C::PBYTES);
+    uint64_t* full = bars;                                // TMA landed
+    uint64_t* dq = bars + C::STAGES;                      // weight tile dequantized
+    uint64_t* empty = bars + 2 * C::STAGES;               // MMA done with the stage
+    uint64_t* accf = bars + 3 * C::STAGES;                // accumulator complete
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * C::STAGES + 1);
+    int* last_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * C::BW, m0 = blockIdx.y * BT, split = blockIdx.z;
+    const int kblocks = (p.K + C::BK - 1) / C::BK;
+    const int kb0 = (int)((long long)split * kblocks / p.splits);
+    const int kb1 = (int)((long long)(split + 1) * kblocks / p.splits);
+    const int nkb = kb1 - kb0;
+    const uint64_t to = p.timeout_ns;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&dq[s], 128);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(accf, 1);
+        fence_mbar_init();
+        prefetch_tmap(&tmX);
+        prefetch_tmap(&tmW);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ producer
+        if (elect_one()) {
+            int issued = 0;
+            for (int i = 0; i < nkb; ++i) {
+                const int s = i % C::STAGES;
+                const uint32_t ph = (uint32_t)(i / C::STAGES) & 1u;
+                if (!mbar_wait(&empty[s], ph ^ 1u, to)) {
+                    raise_status(p.status, kStatusTimeout);
+                    break;
+                }
+                mbar_arrive_expect_tx(&full[s], C::XBYTES + C::PBYTES);
+                tma_load_2d(xs + s * C::XBYTES, &tmX, (kb0 + i) * C::BK, m0, &full[s]);
+                tma_load_2d(ps + s * C::PBYTES, &tmW, (kb0 + i) * (C::BK / 2), n0, &full[s]);
+                issued = i + 1;
+            }
+            // wait until every copy this thread issued has landed
+            for (int i = issued - C::STAGES < 0 ? 0 : issued - C::STAGES; i < issued; ++i) {
+                if (!mbar_wait(&full[i % C::STAGES], (uint32_t)(i / C::STAGES) & 1u, to)) {
+                    raise_status(p.status, kStatusTimeout);
+                    break;
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ----------------------------------------------------- MMA issuer
+        if (elect_one()) {
+            const uint32_t idesc = idesc_bf16_f32(C::BW, BT);
+            for (int i = 0; i < nkb; ++i) {
+                const int s = i % C::STAGES;
+                const uint32_t ph = (uint32_t)(i / C::STAGES) & 1u;
+                if (!mbar_wait(&dq[s], ph, to) || !mbar_wait(&full[s], ph, to)) {
+                    raise_status(p.status, kStatusTimeout);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t wa = smem_u32(ws + s * C::WBYTES);
+                const uint32_t xa = smem_u32(xs + s * C::XBYTES);
+#pragma unroll
+                for (int kk = 0; kk < C::BK / 16; ++kk)
+                    tc_mma_f16(tmem, sw128_desc(wa + kk * 32), sw128_desc(xa + kk * 32), idesc,
+                               (i > 0 || kk > 0) ? 1u : 0u);
+                tc_commit(&empty[s]);
+            }
+            tc_commit(accf);  // arrives once every MMA issued above is complete
+            // TMEM is freed below: make sure no MMA is still writing it
+            if (!mbar_wait(accf, 0, to)) raise_status(p.status, kStatusTimeout);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------- dequant + epilogue
+        const int q = warp & 3;        // TMEM lane quadrant of this warp
+        const int r = q * 32 + lane;   // weight row within the tile == TMEM lane
+        const int n = n0 + r;
+        const bool nvalid = n < p.N;
+        const int G = p.K / p.group;
+        int lut_group = -1;
+        Bf16Lut lut_a = make_lut(p.t.mag, 0.f), lut_b = lut_a;
+        bool ok = true;
+        for (int i = 0; i < nkb; ++i) {
+            const int s = i % C::STAGES;
+            const uint32_t ph = (uint32_t)(i / C::STAGES) & 1u;
+            const int k0 = (kb0 + i) * C::BK;
+            const int ga = k0 / p.group, gb = (k0 + 32) / p.group;
+            if (ga != lut_group) {
+                const float sa = (nvalid && k0 < p.K) ? load_scale(p.scales, p.sdt, (size_t)n * G + ga) : 0.f;
+                lut_a = make_lut(p.t.mag, sa);
+                lut_group = ga;
+            }
+            if (gb != ga) {
+                const float sb = (nvalid && k0 + 32 < p.K) ? load_scale(p.scales, p.sdt, (size_t)n * G + gb) : 0.f;
+                lut_b = make_lut(p.t.mag, sb);
+            } else {
+                lut_b = lut_a;
+            }
+            if (!mbar_wait(&full[s], ph, to)) {
+                raise_status(p.status, kStatusTimeout);
+                ok = false;
+                break;
+            }
+            const uint4* prow = reinterpret_cast<const uint4*>(ps + s * C::PBYTES + r * 32);
+            const uint4 w0 = prow[0], w1 = prow[1];
+            uint8_t* wrow = ws + s * C::WBYTES + r * 128;
+            const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                uint32_t v[4];
+                dequant8(words[c], c < 4 ? lut_a : lut_b, v);
+                *reinterpret_cast<uint4*>(wrow + ((c ^ (r & 7)) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&dq[s]);
+        }
+        // epilogue
+        if (ok && !mbar_wait(accf, 0, to)) {
+            raise_status(p.status, kStatusTimeout);
+            ok = false;
+        }
+        tc_fence_after();
+        const float rho = p.x_scale ? *p.x_scale : 1.f;
+        const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
+        for (int c0 = 0; c0 < BT; c0 += 16) {
+            uint32_t v[16];
+            tmem_ld16(trow + c0, v);
+            tmem_ld_wait();
+            if (!ok || !nvalid) continue;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int m = m0 + c0 + j;
+                if (m >= p.M) break;
+                const float a = __uint_as_float(v[j]);
+                if (p.splits == 1) {
+                    __nv_bfloat16 y = __float2bfloat16_rn(rho * a);
+                    p.Y[(size_t)m * p.N + n] = *reinterpret_cast<uint16_t*>(&y);
+                } else {
+                    p.part[((size_t)split * p.M + m) * p.N + n] = a;
+                }
+            }
+        }
+        if (p.splits > 1) {
+            // the last CTA of this output tile sums the partials in split order
+            __threadfence();
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            const unsigned tile = blockIdx.y * gridDim.x + blockIdx.x;
+            if (threadIdx.x == 64) {
+                const unsigned old = atomicAdd(&p.counters[tile], 1u);
+                *last_flag = (old == (unsigned)p.splits - 1u) ? 1 : 0;
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (*last_flag) {
+                __threadfence();
+                if (nvalid) {
+                    const int mend = min(p.M, m0 + BT);
+                    for (int m = m0; m < mend; ++m) {
+                        float a = 0.f;
+                        for (int z = 0; z < p.splits; ++z) a += __ldcg(&p.part[((size_t)z * p.M + m) * p.N + n]);
+                        __nv_bfloat16 y = __float2bfloat16_rn(rho * a);
+                        p.Y[(size_t)m * p.N + n] = *reinterpret_cast<uint16_t*>(&y);
+                    }
+                }
+                if (threadIdx.x == 64) p.counters[tile] = 0u;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+// ----------------------------------------------------------- host launch
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+static bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, int elem_bytes, const void* base, uint64_t inner,
+                      uint64_t outer, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+    EncodeTiledFn fn = get_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {inner * (uint64_t)elem_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int tc_token_tile(int M) {
+    if (M <= 32) return 32;
+    if (M <= 64) return 64;
+    if (M <= 128) return 128;
+    return 256;
+}
+
+int tc_splits(int M, int N, int K) {
+    const int BT = tc_token_tile(M);
+    const long long tiles = (long long)((N + 127) / 128) * ((M + BT - 1) / BT);
+    const int kblocks = (K + 63) / 64;
+    if (tiles >= 148 || tiles > 4096) return 1;
+    int s = (int)((2 * 148 + tiles - 1) / tiles);
+    s = s > kblocks / 4 ? kblocks / 4 : s;
+    if (s > 16) s = 16;
+    return s < 1 ? 1 : s;
+}
+
+size_t tc_ws_bytes(int M, int N, int K) {
+    const int s = tc_splits(M, N, K);
+    if (s <= 1) return 0;
+    return 4096 * sizeof(unsigned) + (size_t)s * M * N * sizeof(float);
+}
+
+template <int BT>
+static cudaError_t launch_tc_bt(const CUtensorMap& mx, const CUtensorMap& mw, const TcParams& p, cudaStream_t st) {
+    using C = TcCfg<BT>;
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    dim3 grid((p.N + C::BW - 1) / C::BW, (p.M + BT - 1) / BT, p.splits);
+    gemm_tc_kernel<BT><<<grid, 192, C::SMEM, st>>>(mx, mw, p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_tc(const uint16_t* X, const uint8_t* packed, const void* scales, int sdt, const FmtTable& t,
+                           int M, int N, int K, int group, const float* x_scale, uint16_t* Y, void* ws,
+                           size_t ws_bytes, int splits, int* status, unsigned long long timeout_ns,
+                           cudaStream_t st) {
+    const int BT = tc_token_tile(M);
+    const int kblocks = (K + 63) / 64;
+    if (splits <= 0) splits = tc_splits(M, N, K);
+    if (splits > kblocks) splits = kblocks;
+    const long long tiles = (long long)((N + 127) / 128) * ((M + BT - 1) / BT);
+    if (splits > 1) {
+        const size_t need = 4096 * sizeof(unsigned) + (size_t)splits * M * N * sizeof(float);
+        if (!ws || ws_bytes < need || tiles > 4096) splits = 1;
+    }
+    CUtensorMap mx, mw;
+    if (!encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, (uint64_t)K, (uint64_t)M, 64, (uint32_t)BT,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    if (!encode_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, packed, (uint64_t)K / 2, (uint64_t)N, 32, 128,
+                   CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    TcParams p;
+    p.scales = scales;
+    p.sdt = sdt;
+    p.t = t;
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.group = group;
+    p.x_scale = x_scale;
+    p.Y = Y;
+    p.counters = splits > 1 ? reinterpret_cast<unsigned*>(ws) : nullptr;
+    p.part = splits > 1 ? reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + 4096 * sizeof(unsigned)) : nullptr;
+    p.splits = splits;
+    p.status = status;
+    p.timeout_ns = timeout_ns;
+    switch (BT) {
+        case 32: return launch_tc_bt<32>(mx, mw, p, st);
+        case 64: return launch_tc_bt<64>(mx, mw, p, st);
+        case 128: return launch_tc_bt<128>(mx, mw, p, st);
+        default: return launch_tc_bt<256>(mx, mw, p, st);
+    }
+}
+
+}  // namespace fp4
+
+// ------------------------------------------------------- bounded-wait check
+namespace fp4 {
+
+// Waits on an mbarrier that nothing ever arrives on; the bounded wait must
+// give up after timeout_ns and raise FP4_DEV_WAIT_TIMEOUT.  Used by the
+// failure-detection test: it exercises the timeout path without any fault.
+__global__ void bounded_wait_probe_kernel(int* status, unsigned long long timeout_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && !mbar_wait(&bar, 0, timeout_ns)) raise_status(status, kStatusTimeout);
+}
+
+cudaError_t launch_bounded_wait_probe(int* status, unsigned long long timeout_ns, cudaStream_t st) {
+    bounded_wait_probe_kernel<<<1, 32, 0, st>>>(status, timeout_ns);
+    return cudaGetLastError();
+}
+
+}  // namespace fp4

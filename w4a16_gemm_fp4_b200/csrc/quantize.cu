@@ -1,0 +1,370 @@
+// quantize.cu -- FP4 (ExMy) weight quantization on sm_100a.
+//
+// Implements scale-and-clip, compare-and-quantize and the format / range
+// search of the LLM-FP4 summary page ("首个支持4-bit浮点量化的LLM来了",
+// sections on scale-and-clip, eq. (2)-(4), compare-and-quantize, eq. (5),
+// and the search over exponent/mantissa split and quantization range), the
+// fold of the pre-shifted exponent bias into the weights (same page), and
+// the 2-codes-per-byte packing of the "为什么我们需要4-bit浮点量化" tutorial,
+// section 2.2.
+//
+// Data layout: W is walked as a flat array of N*K fp32 (rows contiguous,
+// K % group == 0, so groups never straddle rows).  One warp handles a unit
+// of 128 consecutive elements (4 per lane, one 16-byte load per lane), i.e.
+// 128/group groups; the group absmax is a shuffle reduction over group/4
+// lanes.  The pass is HBM-bound: 4 B read + 0.5 B + (2|4)/group B written
+// per weight.
+//
+// Arithmetic that decides a code is IEEE binary32 with round-to-nearest
+// (__fmul_rn / __fdiv_rn, never contracted), so codes and scales are
+// bit-identical to the CPU oracle.
+#include "common.cuh"
+
+namespace fp4 {
+
+constexpr int kQuantThreads = 256;
+constexpr int kSearchBlocksMax = 1184;  // fixed (shape-only) grid cap => deterministic SSE order
+
+struct QuantParams {
+    const float* W;
+    const int8_t* shift;  // [K] or null
+    long long total;      // N*K
+    int K;
+    int group;
+    int sdt;
+    uint8_t* packed;
+    void* scales;
+    int* status;
+};
+
+__device__ __forceinline__ float pow2i(int e) {  // 2^e for e in [-126, 127], exact
+    return __int_as_float((127 + e) << 23);
+}
+
+// Load the 4 elements of this lane (folded by 2^shift).  Returns false for
+// lanes past the end of the tensor.
+__device__ __forceinline__ bool load4(const QuantParams& p, long long base, float w[4]) {
+    long long off = base + 4 * (threadIdx.x & 31);
+    if (off >= p.total) {
+        w[0] = w[1] = w[2] = w[3] = 0.f;
+        return false;
+    }
+    float4 v = __ldg(reinterpret_cast<const float4*>(p.W + off));
+    w[0] = v.x;
+    w[1] = v.y;
+    w[2] = v.z;
+    w[3] = v.w;
+    if (p.shift) {
+        int k0 = (int)(off % p.K);
+        char4 s = __ldg(reinterpret_cast<const char4*>(p.shift + k0));
+        w[0] = __fmul_rn(w[0], pow2i(s.x));
+        w[1] = __fmul_rn(w[1], pow2i(s.y));
+        w[2] = __fmul_rn(w[2], pow2i(s.z));
+        w[3] = __fmul_rn(w[3], pow2i(s.w));
+    }
+    return true;
+}
+
+// Max over the group/4 lanes that hold one group.
+__device__ __forceinline__ float group_absmax(float a, int lanes_per_group) {
+    for (int o = 1; o < lanes_per_group; o <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    return a;
+}
+
+// Stored scale (fp32, or fp16 round-to-nearest-even widened back) for
+// group absmax A, bias factor cj and format maximum qmax.
+__device__ __forceinline__ float stored_scale(float A, float cj, float qmax, int sdt, bool* overflow,
+                                              uint32_t* raw) {
+    float s32 = __fdiv_rn(__fmul_rn(A, cj), qmax);
+    if (sdt == FP4_SCALE_F16) {
+        __half h = __float2half_rn(s32);
+        *raw = __half_as_ushort(h);
+        float s = __half2float(h);
+        *overflow = isinf(s);
+        return s;
+    }
+    *raw = __float_as_uint(s32);
+    *overflow = !isfinite(s32);
+    return s32;
+}
+
+__device__ __forceinline__ int code_of(float w, float s, const FmtTable& t, float* v_signed) {
+    int idx = 0;
+    if (s != 0.f) idx = nearest_index(fabsf(__fdiv_rn(w, s)), t);
+    const bool neg = signbit(w);
+    const float v = t.mag[idx];
+    *v_signed = neg ? -v : v;
+    return (neg ? 8 : 0) | idx;
+}
+
+// Fused pass: group absmax -> scale -> codes -> pack, for a fixed
+// candidate (format, j) taken from kernel arguments or, when `choice` is
+// non-null, from device memory (written by the search).  Optionally
+// accumulates SSE per block into ws_sse[block] (fp64).
+__global__ void __launch_bounds__(kQuantThreads) quantize_kernel(QuantParams p, FmtTables tabs, int fmt, int j,
+                                                                 const int32_t* choice, int32_t* choice_out,
+                                                                 double* ws_sse) {
+    if (choice) {
+        fmt = choice[0];
+        j = choice[1];
+    }
+    const FmtTable& t = tabs.f[fmt];
+    const float cj = tabs.cj[j];
+    const int lane = threadIdx.x & 31;
+    const int lpg = p.group >> 2;  // lanes per group
+    const long long units = (p.total + 127) / 128;
+    const long long wid = (long long)blockIdx.x * (kQuantThreads / 32) + (threadIdx.x >> 5);
+    const long long nw = (long long)gridDim.x * (kQuantThreads / 32);
+    if (choice_out && blockIdx.x == 0 && threadIdx.x == 0) {
+        choice_out[0] = fmt;
+        choice_out[1] = j;
+    }
+    double sse = 0.0;
+    bool bad = false, ovf = false;
+    for (long long u = wid; u < units; u += nw) {
+        const long long base = u * 128;
+        float w[4];
+        const bool valid = load4(p, base, w);
+        float a = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            bad |= valid && !isfinite(w[i]);
+            a = fmaxf(a, fabsf(w[i]));
+        }
+        const float A = group_absmax(a, lpg);
+        bool o;
+        uint32_t raw;
+        const float s = stored_scale(A, cj, t.qmax, p.sdt, &o, &raw);
+        if (!valid) continue;
+        ovf |= o;
+        uint32_t codes = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float v;
+            const int c = code_of(w[i], s, t, &v);
+            codes |= (uint32_t)c << (4 * i);
+            if (ws_sse) {
+                const double d = (double)w[i] - (double)v * (double)s;
+                sse = fma(d, d, sse);
+            }
+        }
+        const long long off = base + 4 * lane;
+        *reinterpret_cast<uint16_t*>(p.packed + off / 2) = (uint16_t)codes;
+        if ((lane & (lpg - 1)) == 0) {
+            const long long gi = off / p.group;
+            if (p.sdt == FP4_SCALE_F16)
+                reinterpret_cast<uint16_t*>(p.scales)[gi] = (uint16_t)raw;
+            else
+                reinterpret_cast<uint32_t*>(p.scales)[gi] = raw;
+        }
+    }
+    if (bad) raise_status(p.status, kStatusNonfinite);
+    if (ovf) raise_status(p.status, kStatusScaleOverflow);
+    if (ws_sse) {
+        // fixed-order block reduction: warp shuffles, then warps in order
+        __shared__ double red[kQuantThreads / 32];
+        for (int o = 16; o > 0; o >>= 1) sse += __shfl_xor_sync(0xffffffffu, sse, o);
+        if (lane == 0) red[threadIdx.x >> 5] = sse;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            double acc = 0.0;
+            for (int i = 0; i < kQuantThreads / 32; ++i) acc += red[i];
+            ws_sse[blockIdx.x] = acc;
+        }
+    }
+}
+
+// Search pass: for every candidate (f, j) in the set, SSE of quantizing
+// the whole tensor with it; per-block fp64 partials into ws[block][24].
+// Every element is loaded once and evaluated for all candidates from
+// registers (the pass is ALU-bound: one IEEE division per element and
+// candidate).
+__global__ void __launch_bounds__(kQuantThreads) search_kernel(QuantParams p, FmtTables tabs, int f0, int f1,
+                                                               int jn, double* ws) {
+    const int lane = threadIdx.x & 31;
+    const int lpg = p.group >> 2;
+    const long long units = (p.total + 127) / 128;
+    const long long wid = (long long)blockIdx.x * (kQuantThreads / 32) + (threadIdx.x >> 5);
+    const long long nw = (long long)gridDim.x * (kQuantThreads / 32);
+    double sse[24];
+#pragma unroll
+    for (int c = 0; c < 24; ++c) sse[c] = 0.0;
+    bool bad = false;
+    for (long long u = wid; u < units; u += nw) {
+        float w[4];
+        const bool valid = load4(p, u * 128, w);
+        float a = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            bad |= valid && !isfinite(w[i]);
+            a = fmaxf(a, fabsf(w[i]));
+        }
+        const float A = group_absmax(a, lpg);
+        if (!valid) continue;
+#pragma unroll
+        for (int f = 0; f < 3; ++f) {
+            if (f < f0 || f > f1) continue;
+            const FmtTable& t = tabs.f[f];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                if (j >= jn) continue;
+                bool o;
+                uint32_t raw;
+                const float s = stored_scale(A, tabs.cj[j], t.qmax, p.sdt, &o, &raw);
+                double acc = 0.0;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float v;
+                    code_of(w[i], s, t, &v);
+                    const double d = (double)w[i] - (double)v * (double)s;
+                    acc = fma(d, d, acc);
+                }
+                sse[f * 8 + j] += acc;
+            }
+        }
+    }
+    if (bad) raise_status(p.status, kStatusNonfinite);
+    __shared__ double red[kQuantThreads / 32][24];
+#pragma unroll
+    for (int c = 0; c < 24; ++c) {
+        double v = sse[c];
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) red[threadIdx.x >> 5][c] = v;
+    }
+    __syncthreads();
+    if (threadIdx.x < 24) {
+        double acc = 0.0;
+        for (int i = 0; i < kQuantThreads / 32; ++i) acc += red[i][threadIdx.x];
+        ws[(size_t)blockIdx.x * 24 + threadIdx.x] = acc;
+    }
+}
+
+// Sum the per-block partials in block order, pick the first strict minimum
+// in (format, j) order, write choice and sse (NaN for candidates outside
+// the searched set).  One block.
+__global__ void search_finalize_kernel(const double* ws, int nblocks, int f0, int f1, int jn, int32_t* choice,
+                                       double* sse_out) {
+    __shared__ double tot[24];
+    const int c = threadIdx.x;
+    if (c < 24) {
+        double acc = 0.0;
+        for (int b = 0; b < nblocks; ++b) acc += ws[(size_t)b * 24 + c];
+        tot[c] = acc;
+    }
+    __syncthreads();
+    if (c == 0) {
+        int bf = f0, bj = 0;
+        double best = INFINITY;
+        for (int f = f0; f <= f1; ++f)
+            for (int j = 0; j < jn; ++j)
+                if (tot[f * 8 + j] < best) {
+                    best = tot[f * 8 + j];
+                    bf = f;
+                    bj = j;
+                }
+        if (choice) {
+            choice[0] = bf;
+            choice[1] = bj;
+        }
+        if (sse_out) {
+            for (int f = 0; f < 3; ++f)
+                for (int j = 0; j < 8; ++j) {
+                    const bool in = f >= f0 && f <= f1 && j < jn;
+                    sse_out[f * 8 + j] = in ? tot[f * 8 + j] : __longlong_as_double(0x7ff8000000000000LL);
+                }
+        }
+    }
+}
+
+// SSE of a single fixed candidate (no search): per-block partials written
+// by quantize_kernel, summed in block order.
+__global__ void sse_single_finalize_kernel(const double* ws, int nblocks, int fmt, int j, double* sse_out) {
+    if (threadIdx.x != 0) return;
+    double acc = 0.0;
+    for (int b = 0; b < nblocks; ++b) acc += ws[b];
+    for (int c = 0; c < 24; ++c) sse_out[c] = __longlong_as_double(0x7ff8000000000000LL);
+    sse_out[fmt * 8 + j] = acc;
+}
+
+// ----------------------------------------------------------- host launch
+
+int quantize_grid_blocks(long long total) {
+    const long long units = (total + 127) / 128;
+    long long blocks = (units + (kQuantThreads / 32) - 1) / (kQuantThreads / 32);
+    if (blocks > kSearchBlocksMax) blocks = kSearchBlocksMax;
+    if (blocks < 1) blocks = 1;
+    return (int)blocks;
+}
+
+size_t quantize_ws_bytes(long long total, bool search, bool want_sse) {
+    if (!search && !want_sse) return 0;
+    return (size_t)quantize_grid_blocks(total) * 24 * sizeof(double);
+}
+
+cudaError_t launch_quantize(const float* W, int N, int K, int group, int fmt, int bias_search,
+                            const int8_t* shift, int sdt, uint8_t* packed, void* scales, int32_t* choice,
+                            double* sse, void* ws, const FmtTables& tabs, int* status, cudaStream_t st) {
+    QuantParams p;
+    p.W = W;
+    p.shift = shift;
+    p.total = (long long)N * K;
+    p.K = K;
+    p.group = group;
+    p.sdt = sdt;
+    p.packed = packed;
+    p.scales = scales;
+    p.status = status;
+    const int f0 = fmt < 0 ? 0 : fmt, f1 = fmt < 0 ? 2 : fmt;
+    const int jn = bias_search ? 8 : 1;
+    const bool search = (f0 != f1) || jn > 1;
+    const int blocks = quantize_grid_blocks(p.total);
+    double* wsd = reinterpret_cast<double*>(ws);
+    if (search) {
+        search_kernel<<<blocks, kQuantThreads, 0, st>>>(p, tabs, f0, f1, jn, wsd);
+        search_finalize_kernel<<<1, 32, 0, st>>>(wsd, blocks, f0, f1, jn, choice, sse);
+        quantize_kernel<<<blocks, kQuantThreads, 0, st>>>(p, tabs, 0, 0, choice, nullptr, nullptr);
+    } else {
+        quantize_kernel<<<blocks, kQuantThreads, 0, st>>>(p, tabs, f0, 0, nullptr, choice, sse ? wsd : nullptr);
+        if (sse) sse_single_finalize_kernel<<<1, 32, 0, st>>>(wsd, blocks, f0, 0, sse);
+    }
+    return cudaGetLastError();
+}
+
+// --------------------------------------------------------------- dequant
+// W_hat[n,k] = fl32(v(code) * s): one thread per 8 elements (one 32-bit
+// word of codes).
+__global__ void dequantize_kernel(const uint32_t* packed, const void* scales, int sdt, FmtTable t,
+                                  long long words, int K, int group, float* out) {
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < words;
+         i += (long long)gridDim.x * blockDim.x) {
+        const uint32_t w = packed[i];
+        const long long e0 = i * 8;
+        const long long row = e0 / K;
+        const int k0 = (int)(e0 % K);
+        const int G = K / group;
+        const float s = load_scale(scales, sdt, (size_t)row * G + k0 / group);
+        float r[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int c = (w >> (4 * q)) & 15;
+            const float v = t.mag[c & 7];
+            r[q] = __fmul_rn((c & 8) ? -v : v, s);
+        }
+        float4* o = reinterpret_cast<float4*>(out + e0);
+        o[0] = make_float4(r[0], r[1], r[2], r[3]);
+        o[1] = make_float4(r[4], r[5], r[6], r[7]);
+    }
+}
+
+cudaError_t launch_dequantize(const uint8_t* packed, const void* scales, int sdt, const FmtTable& t, int N,
+                              int K, int group, float* out, cudaStream_t st) {
+    const long long words = (long long)N * K / 8;
+    long long blocks = (words + 255) / 256;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks < 1) blocks = 1;
+    dequantize_kernel<<<(int)blocks, 256, 0, st>>>(reinterpret_cast<const uint32_t*>(packed), scales, sdt, t,
+                                                   words, K, group, out);
+    return cudaGetLastError();
+}
+
+}  // namespace fp4
