@@ -164,6 +164,14 @@ def build_workload(api, torch, copies):
     return mats, cases
 
 
+def capture(torch, fn, stream):
+    """Capture fn() (a sequence of library calls) into a CUDA graph."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    return g
+
+
 def run_ours(args, world, rank):
     import torch
     from w4a16_gemm_fp4_b200 import api, build
@@ -175,63 +183,74 @@ def run_ours(args, world, rank):
     per_copy = sum(weight_bytes(N, K) for (N, K) in SHAPES)
     copies = max(4, int(np.ceil(4 * l2 / per_copy)))
     mats, cases = build_workload(api, torch, copies)
-    outs = {(i, M): torch.empty((M, m["N"]), dtype=torch.bfloat16, device=dev) for i, m in enumerate(mats)
-            for M in MS}
+    keys = [(i, M) for M in MS for i in range(len(mats))]
+    outs = {(i, M): torch.empty((M, mats[i]["N"]), dtype=torch.bfloat16, device=dev) for (i, M) in keys}
     wss = {}
-    for i, m in enumerate(mats):
-        for M in MS:
-            nb = api.gemm_workspace_size(M, m["N"], m["K"])
-            wss[(i, M)] = torch.zeros(max(nb, 16), dtype=torch.uint8, device=dev) if nb else None
-    stream = torch.cuda.current_stream()
+    for (i, M) in keys:
+        nb = api.gemm_workspace_size(M, mats[i]["N"], mats[i]["K"])
+        wss[(i, M)] = torch.zeros(max(nb, 16), dtype=torch.uint8, device=dev) if nb else None
+    stream = torch.cuda.Stream()
 
-    def step(s, events=None):
-        c = s % copies
-        for M in MS:
-            for i, m in enumerate(mats):
-                packed, scales = m["reps"][c]
-                if events is not None:
-                    events[(i, M)][0].record(stream)
-                api.gemm(m["X"][M], packed, scales, api.E2M1, GROUP, out=outs[(i, M)], workspace=wss[(i, M)],
-                         stream=stream)
-                if events is not None:
-                    events[(i, M)][1].record(stream)
+    def sweep(c, events=None):
+        for (i, M) in keys:
+            packed, scales = mats[i]["reps"][c]
+            if events is not None:
+                events[(i, M)][0].record()
+            api.gemm(mats[i]["X"][M], packed, scales, api.E2M1, GROUP, out=outs[(i, M)], workspace=wss[(i, M)])
+            if events is not None:
+                events[(i, M)][1].record()
 
-    for s in range(args.warmup):
-        step(s)
+    with torch.cuda.stream(stream):
+        for s in range(args.warmup):          # eager warm-up (also loads modules, sets attributes)
+            sweep(s % copies)
+    torch.cuda.synchronize()
+    # one graph per weight copy; each holds the 12 launches and an event pair around each launch
+    graphs, gevents = [], []
+    for c in range(copies):
+        evs = {k: (torch.cuda.Event(enable_timing=True, external=True),
+                   torch.cuda.Event(enable_timing=True, external=True)) for k in keys}
+        graphs.append(capture(torch, lambda c=c, evs=evs: sweep(c, evs), stream))
+        gevents.append(evs)
+    with torch.cuda.stream(stream):
+        for s in range(args.warmup):
+            graphs[s % copies].replay()
     torch.cuda.synchronize()
     api.device_status(clear=True)
 
-    # timed region: per-launch events inside, outer events around
-    ev = {k: [] for k in outs}
-    per = {}
+    # clock sampler: soak ~1.5 s of the same replays so that nvidia-smi has
+    # samples under this load, then the timed region
     clocks = ClockSampler(dev.index)
     clocks.start()
+    t_end = time.time() + args.soak_s
+    with torch.cuda.stream(stream):
+        s = 0
+        while time.time() < t_end:
+            for _ in range(50):
+                graphs[s % copies].replay()
+                s += 1
+            stream.synchronize()
     barrier(world)
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for s in range(args.steps):
-        evs = {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for k in outs}
-        step(args.warmup + s, evs)
-        for k in outs:
-            ev[k].append(evs[k])
-    t1.record(stream)
+    with torch.cuda.stream(stream):
+        t0.record()
+        for s in range(args.steps):
+            graphs[s % copies].replay()
+        t1.record()
     torch.cuda.synchronize()
     barrier(world)
     clk = clocks.stop()
-    ms_local = t0.elapsed_time(t1)
-    ms = max_over_ranks(world, ms_local)
+    ms = max_over_ranks(world, t0.elapsed_time(t1))
     st = api.device_status(clear=True)
     if st:
         raise RuntimeError("device status %#x during the timed region" % st)
-    for k, lst in ev.items():
-        per[k] = sum(a.elapsed_time(b) for a, b in lst) / len(lst)
+    # per-launch durations: the last replay of every graph (the final `copies` steps of the timed region)
+    per = {k: statistics.mean(ev[k][0].elapsed_time(ev[k][1]) for ev in gevents) for k in keys}
 
     total_bytes = step_weight_bytes() * args.steps * world
     value = total_bytes / (ms * 1e-3) / 1e9
 
-    # dominant kernel (largest share of the step): roofline
     groups = {}
     for (i, M), t in per.items():
         eng = "decode" if M <= 8 else "tensor"
@@ -240,87 +259,100 @@ def run_ours(args, world, rank):
         g["ms"] += t
         g["bytes"] += weight_bytes(N, K) + M * K * 2 + M * N * 2
         g["launches"] += 1
-    dom = max(groups.items(), key=lambda kv: kv[1]["ms"])
-    (eng, Mdom), g = dom
+    (eng, Mdom), g = max(groups.items(), key=lambda kv: kv[1]["ms"])
     achieved = g["bytes"] / (g["ms"] * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
-                "kernel": "gemm_%s_kernel (M=%d, 3 matrices)" % ("decode" if eng == "decode" else "tc", Mdom),
-                "peak_source": peaks["source"]}
+                "kernel": "%s (M=%d, 3 matrices)" % ("gemm_decode_kernel" if eng == "decode" else "gemm_tc_kernel",
+                                                     Mdom),
+                "peak_source": peaks["source"], "share_of_step": round(g["ms"] / sum(per.values()), 3)}
     per_m = {}
     for (eng_, M), gg in sorted(groups.items(), key=lambda kv: kv[0][1]):
         per_m[str(M)] = {"engine": eng_, "us_per_3_matrices": round(gg["ms"] * 1e3, 2),
                          "weight_gbs": round(sum(weight_bytes(N, K) for (N, K) in SHAPES) / (gg["ms"] * 1e-3) / 1e9,
-                                             1)}
+                                             1),
+                         "us_per_launch": [round(per[(i, M)] * 1e3, 2) for i in range(len(mats))]}
 
-    # e2e: activations copied from pinned host memory each step, outputs read back
-    e2e = run_e2e(api, torch, mats, args, stream, world)
-
+    e2e = None if args.no_e2e else run_e2e(api, torch, mats, args, stream, world)
     parts = {}
     if not args.no_parts and rank == 0:
-        parts = run_parts(api, torch, peaks, dev)
+        parts = run_parts(api, torch, peaks, dev, stream)
     return {
         "value": value, "ms_per_step": ms / args.steps, "roofline": roofline, "clocks": clk, "e2e": e2e,
-        "gpu_launches": len(outs) * args.steps, "per_m": per_m, "parts": parts, "copies": copies,
+        "gpu_launches": len(keys) * args.steps, "per_m": per_m, "parts": parts, "copies": copies,
         "copy_bytes": per_copy * copies, "l2_bytes": l2,
     }
 
 
 def run_e2e(api, torch, mats, args, stream, world):
-    """Same sweep through the public API with host buffers: every step
-    copies X (pinned) to the device and reads every Y back."""
+    """The same sweep through the public API with host buffers: every step
+    copies each X from pinned host memory to the device and reads every Y
+    back (captured once into graphs, replayed per step)."""
     dev = torch.device("cuda", torch.cuda.current_device())
+    keys = [(i, M) for M in MS for i in range(len(mats))]
     hx, hy, dx, dy = {}, {}, {}, {}
     h2d = d2h = 0
-    for i, m in enumerate(mats):
-        for M in MS:
-            hx[(i, M)] = m["X"][M].cpu().pin_memory()
-            hy[(i, M)] = torch.empty((M, m["N"]), dtype=torch.bfloat16).pin_memory()
-            dx[(i, M)] = torch.empty_like(m["X"][M])
-            dy[(i, M)] = torch.empty((M, m["N"]), dtype=torch.bfloat16, device=dev)
-            h2d += hx[(i, M)].numel() * 2
-            d2h += hy[(i, M)].numel() * 2
+    for (i, M) in keys:
+        hx[(i, M)] = mats[i]["X"][M].cpu().pin_memory()
+        hy[(i, M)] = torch.empty((M, mats[i]["N"]), dtype=torch.bfloat16).pin_memory()
+        dx[(i, M)] = torch.empty_like(mats[i]["X"][M])
+        dy[(i, M)] = torch.empty((M, mats[i]["N"]), dtype=torch.bfloat16, device=dev)
+        h2d += hx[(i, M)].numel() * 2
+        d2h += hy[(i, M)].numel() * 2
+    copies = len(mats[0]["reps"])
+    wss = {k: (lambda nb: torch.zeros(max(nb, 16), dtype=torch.uint8, device=dev) if nb else None)(
+        api.gemm_workspace_size(k[1], mats[k[0]]["N"], mats[k[0]]["K"])) for k in keys}
 
-    def step(s):
-        c = s % len(mats[0]["reps"])
-        for M in MS:
-            for i, m in enumerate(mats):
-                dx[(i, M)].copy_(hx[(i, M)], non_blocking=True)
-                packed, scales = m["reps"][c]
-                api.gemm(dx[(i, M)], packed, scales, api.E2M1, GROUP, out=dy[(i, M)], stream=stream)
-                hy[(i, M)].copy_(dy[(i, M)], non_blocking=True)
+    def step(c):
+        for (i, M) in keys:
+            dx[(i, M)].copy_(hx[(i, M)], non_blocking=True)
+            packed, scales = mats[i]["reps"][c]
+            api.gemm(dx[(i, M)], packed, scales, api.E2M1, GROUP, out=dy[(i, M)], workspace=wss[(i, M)])
+            hy[(i, M)].copy_(dy[(i, M)], non_blocking=True)
 
-    for s in range(args.warmup):
-        step(s)
+    with torch.cuda.stream(stream):
+        for s in range(args.warmup):
+            step(s % copies)
+    torch.cuda.synchronize()
+    graphs = [capture(torch, lambda c=c: step(c), stream) for c in range(copies)]
+    with torch.cuda.stream(stream):
+        for s in range(args.warmup):
+            graphs[s % copies].replay()
     torch.cuda.synchronize()
     barrier(world)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for s in range(args.steps):
-        step(s)
-    t1.record(stream)
+    with torch.cuda.stream(stream):
+        t0.record()
+        for s in range(args.steps):
+            graphs[s % copies].replay()
+        t1.record()
     torch.cuda.synchronize()
     ms = max_over_ranks(world, t0.elapsed_time(t1))
     v = step_weight_bytes() * args.steps * world / (ms * 1e-3) / 1e9
     return {"value": round(v, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 
-def time_fn(torch, fn, iters, warm=3):
-    for _ in range(warm):
-        fn()
+def time_graph(torch, fn, stream, iters, warm=3):
+    """Mean time of fn() replayed from a CUDA graph (no host overhead)."""
+    with torch.cuda.stream(stream):
+        for _ in range(warm):
+            fn()
     torch.cuda.synchronize()
-    a = torch.cuda.Event(enable_timing=True)
-    b = torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(iters):
-        fn()
-    b.record()
+    g = capture(torch, fn, stream)
+    with torch.cuda.stream(stream):
+        g.replay()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(iters):
+            g.replay()
+        b.record()
     torch.cuda.synchronize()
     return a.elapsed_time(b) / iters
 
 
-def run_parts(api, torch, peaks, dev):
+def run_parts(api, torch, peaks, dev, stream):
     from w4a16_gemm_fp4_b200 import synth
     out = {}
     # quantize pass (E2M1, group 128, fp16 scales) over the three decode matrices
@@ -331,13 +363,13 @@ def run_parts(api, torch, peaks, dev):
     def qpass():
         for W, o in zip(Ws, outs):
             api.quantize_into(W, o["packed"], o["scales"], o["choice"], GROUP, api.E2M1)
-    ms = time_fn(torch, qpass, 10)
+    ms = time_graph(torch, qpass, stream, 20)
     qbytes = sum(N * K * 4 + weight_bytes(N, K) for (N, K) in SHAPES)
     out["quantize"] = {"workload": "3 LLaMA-7B decode matrices, E2M1 g128 fp16 scales", "ms": round(ms, 4),
                        "gbs": round(qbytes / (ms * 1e-3) / 1e9, 1),
                        "frac_hbm": round(qbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
     del Ws, outs
-    # prefill with the pre-shift: calibrate + apply + GEMM M = 2048 on 4096x4096 and 11008x4096
+    # prefill with the pre-shift: GEMM M = 2048 on 4096x4096 and 11008x4096
     case = synth.llama7b_prefill()
     X = torch.from_numpy(case["X"].view(np.int16)).cuda().view(torch.bfloat16)
     shift, rho = api.preshift_calibrate(X)
@@ -348,19 +380,21 @@ def run_parts(api, torch, peaks, dev):
     def prefill():
         for q, y in zip(qs, ys):
             api.gemm(Xt, q["packed"], q["scales"], api.E2M1, GROUP, x_scale=rho, out=y)
-    ms = time_fn(torch, prefill, 10)
+    ms = time_graph(torch, prefill, stream, 20)
     flops = sum(2.0 * X.shape[0] * N * K for (N, K) in ((4096, 4096), (11008, 4096)))
     tf = flops / (ms * 1e-3) / 1e12
-    out["prefill"] = {"workload": "LLaMA-7B prefill X 2048x4096 (1% outlier channels x50), pre-shift on",
-                      "ms": round(ms, 4), "tflops": round(tf, 1), "peak_tflops": peaks["bf16_tflops"],
-                      "frac": round(tf / peaks["bf16_tflops"], 4)}
-    ms_pro = time_fn(torch, lambda: api.preshift_apply(X, shift, rho, out=Xt), 10)
-    out["preshift_apply"] = {"ms": round(ms_pro, 4),
-                             "gbs": round(2 * 2 * X.numel() / (ms_pro * 1e-3) / 1e9, 1)}
-    del X, Xt, qs, ys
+    out["prefill"] = {"workload": "LLaMA-7B prefill X 2048x4096 (1% outlier channels x50), pre-shift on, "
+                                  "W 4096x4096 + 11008x4096", "ms": round(ms, 4), "tflops": round(tf, 1),
+                      "peak_tflops": peaks["bf16_tflops"], "frac": round(tf / peaks["bf16_tflops"], 4)}
+    ws_cal = torch.zeros(api.lib().fp4_preshift_workspace_size(*X.shape), dtype=torch.uint8, device=dev)
+    ms_pro = time_graph(torch, lambda: api.preshift_apply(X, shift, rho, out=Xt), stream, 20)
+    out["preshift_apply"] = {"ms": round(ms_pro, 4), "gbs": round(2 * 2 * X.numel() / (ms_pro * 1e-3) / 1e9, 1)}
+    del X, Xt, qs, ys, ws_cal
     # format / bias search on 5120x5120 Student-t weights
     W = torch.from_numpy(synth.student_t_weights(np.random.default_rng(3), 5120, 5120)).cuda()
-    ms = time_fn(torch, lambda: api.quantize(W, GROUP, api.AUTO, True), 3, warm=1)
+    o = api.quantize(W, GROUP, api.AUTO, True)
+    ms = time_graph(torch, lambda: api.quantize_into(W, o["packed"], o["scales"], o["choice"], GROUP, api.AUTO,
+                                                     True), stream, 5, warm=1)
     out["search"] = {"workload": "5120x5120 Student-t(5)*0.015, 3 formats x 8 bias candidates + pack",
                      "ms": round(ms, 3), "candidate_evals_per_s": round(24 * W.numel() / (ms * 1e-3), 0)}
     return out
@@ -425,11 +459,14 @@ def run_reference(args, world, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-parts", action="store_true", help="skip the quantize/prefill/search legs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg")
+    ap.add_argument("--soak-s", type=float, default=1.5,
+                    help="seconds of untimed replays before the timed region (clock sampling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
