@@ -123,8 +123,11 @@ class Workspace:
 _ws = {}
 
 
-def _workspace(device):
-    key = (device.type, device.index)
+def _workspace(device, kind="scratch"):
+    """Per-device buffers.  "gemm" is reserved for fp4_gemm, whose split-K
+    tile counters must stay zero between calls; "scratch" serves the calls
+    whose workspace needs no initialisation (quantize, calibrate)."""
+    key = (device.type, device.index, kind)
     if key not in _ws:
         _ws[key] = Workspace(device)
     return _ws[key]
@@ -225,7 +228,7 @@ def gemm(X, packed, scales, fmt=E2M1, group=128, x_scale=None, out=None, engine=
         need = L.fp4_gemm_workspace_size(M, N, K)
         if splits > 0:
             need = max(need, 16384 + splits * M * N * 4)
-        ws, wsb = _workspace(X.device).get(need)
+        ws, wsb = _workspace(X.device, "gemm").get(need)
     else:
         ws, wsb = workspace, workspace.numel() * workspace.element_size()
     _check(L.fp4_gemm_ex(_ptr(_bits(X)), _ptr(packed), _ptr(scales), sdt, fmt, M, N, K, group, _ptr(x_scale),

@@ -21,7 +21,7 @@ cudaError_t launch_calibrate(const uint16_t* X, int M, int K, int8_t* shift, flo
 cudaError_t launch_apply(const uint16_t* X, int M, int K, const int8_t* shift, const float* rho, uint16_t* Xt,
                          cudaStream_t st);
 cudaError_t launch_gemm_decode(const uint16_t* X, const uint8_t* packed, const void* scales, int sdt,
-                               const FmtTable& t, int M, int N, int K, int group, const float* x_scale,
+                               const FmtTable& t, int fmt, int M, int N, int K, int group, const float* x_scale,
                                uint16_t* Y, cudaStream_t st);
 size_t tc_ws_bytes(int M, int N, int K);
 cudaError_t launch_gemm_tc(const uint16_t* X, const uint8_t* packed, const void* scales, int sdt, const FmtTable& t,
@@ -252,7 +252,8 @@ fp4_status fp4_gemm_ex(const uint16_t* X, const uint8_t* packed, const void* sca
     const FmtTable& t = tables().f[fmt];
     if (engine == FP4_ENGINE_DECODE) {
         if (M > kDecodeMaxM) return FP4_ERR_UNSUPPORTED_SHAPE;
-        return cuda_status(launch_gemm_decode(X, packed, scales, (int)sdt, t, M, N, K, group, x_scale, Y, stream));
+        return cuda_status(
+            launch_gemm_decode(X, packed, scales, (int)sdt, t, (int)fmt, M, N, K, group, x_scale, Y, stream));
     }
     int* st = status_ptr();
     if (!st) return FP4_ERR_CUDA;

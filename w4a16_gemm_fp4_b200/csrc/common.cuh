@@ -114,6 +114,35 @@ __device__ __forceinline__ void dequant8(uint32_t w, const Bf16Lut& l, uint32_t 
     }
 }
 
+// Exact code values by bit placement, 8 codes of one 32-bit word at a time,
+// for a format with MANT mantissa bits (E1M2: 2, E2M1: 1, E3M0: 0) and bias
+// b = 2^(2-MANT) - 1.  The 3 magnitude bits of a code are placed so that the
+// format's exponent field lands on the lowest bf16 exponent bits: the bf16
+// value is then v * 2^(b-127) for every code, subnormal ones included (both
+// formats put a zero exponent field in the subnormal binade), and one bf16
+// multiply by 2^(127-b) gives v exactly.  A single integer multiply places
+// magnitude and sign of two codes 16 bits apart at once (the shifted copies
+// never overlap, so there are no carries); the result pairs are
+// p[i] = (code i, code i+4), low half first.  9 ALU + 8 FMA-pipe ops.
+template <int MANT>
+__device__ __forceinline__ void dequant8_exact(uint32_t w, uint32_t p[4]) {
+    constexpr int SHIFT = 7 - MANT;
+    constexpr uint32_t MUL0 = (1u << SHIFT) + (1u << 12);
+    constexpr uint32_t MUL1 = MUL0 >> 4;
+    constexpr uint32_t MASK = (0x8000u | (7u << SHIFT)) * 0x10001u;
+    constexpr int BIAS = (1 << (2 - MANT)) - 1;
+    constexpr uint32_t SC = (uint32_t)((254 - BIAS) << 7) * 0x10001u;  // bf16x2 of 2^(127-b)
+    const uint32_t w8 = w >> 8;
+    const uint32_t q0 = ((w & 0x000F000Fu) * MUL0) & MASK;
+    const uint32_t q1 = ((w & 0x00F000F0u) * MUL1) & MASK;
+    const uint32_t q2 = ((w8 & 0x000F000Fu) * MUL0) & MASK;
+    const uint32_t q3 = ((w8 & 0x00F000F0u) * MUL1) & MASK;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(p[0]) : "r"(q0), "r"(SC));
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(p[1]) : "r"(q1), "r"(SC));
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(p[2]) : "r"(q2), "r"(SC));
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(p[3]) : "r"(q3), "r"(SC));
+}
+
 __device__ __forceinline__ float load_scale(const void* scales, int sdt, size_t idx) {
     if (sdt == FP4_SCALE_F16) return __half2float(__ldg(reinterpret_cast<const __half*>(scales) + idx));
     return __ldg(reinterpret_cast<const float*>(scales) + idx);

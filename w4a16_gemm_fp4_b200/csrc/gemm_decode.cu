@@ -158,25 +158,149 @@ __global__ void __launch_bounds__(256) gemm_decode_kernel(DecodeParams p) {
     }
 }
 
+// ---------------------------------------------------------------------------
+// Group-128 path: exact code values (dequant8_exact, 9 ALU + 8 FMA-pipe ops
+// per 8 weights), one 128-wide chunk == one group, scaled once per chunk in
+// fp32.  The code pairs come out as (k, k+4) within every 8 consecutive k,
+// so the activation pairs are rebuilt the same way with two prmt per pair.
+// Chunks are double-buffered in registers (ping-pong, no copies) and every
+// address advances by a constant per chunk.
+template <int R, int MANT>
+__global__ void __launch_bounds__(256) gemm_decode_g128_kernel(DecodeParams p) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int n0 = blockIdx.x * 16 * R;
+    const int nchunks = (p.K + 127) >> 7;
+    const int c_begin = warp * nchunks / 8, c_end = (warp + 1) * nchunks / 8;
+    const int G = p.K >> 7;
+    const size_t rowbytes = (size_t)p.K >> 1;
+
+    // per-row base pointers (this lane's 16-byte segment of chunk 0)
+    const uint4* pa[R];
+    const uint4* pb[R];
+    bool va[R], vb[R];
+    const __half* sah[R];
+    const __half* sbh[R];
+    const float* saf[R];
+    const float* sbf[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int na = n0 + 16 * r + g, nb = na + 8;
+        va[r] = na < p.N;
+        vb[r] = nb < p.N;
+        pa[r] = reinterpret_cast<const uint4*>(p.packed + (size_t)(va[r] ? na : 0) * rowbytes) + t;
+        pb[r] = reinterpret_cast<const uint4*>(p.packed + (size_t)(vb[r] ? nb : 0) * rowbytes) + t;
+        sah[r] = reinterpret_cast<const __half*>(p.scales) + (size_t)(va[r] ? na : 0) * G;
+        sbh[r] = reinterpret_cast<const __half*>(p.scales) + (size_t)(vb[r] ? nb : 0) * G;
+        saf[r] = reinterpret_cast<const float*>(p.scales) + (size_t)(va[r] ? na : 0) * G;
+        sbf[r] = reinterpret_cast<const float*>(p.scales) + (size_t)(vb[r] ? nb : 0) * G;
+    }
+    const bool xv = g < p.M;
+    const uint4* px = reinterpret_cast<const uint4*>(p.X + (size_t)(xv ? g : 0) * p.K) + 4 * t;
+    const bool f16 = p.sdt == FP4_SCALE_F16;
+
+    float acc[R][4];
+#pragma unroll
+    for (int r = 0; r < R; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
+
+    auto load = [&](int c, ChunkRegs<R>& cr) {
+        const bool kv = c * 128 + 32 * t < p.K;  // K % 32 == 0: a lane's 32 codes are all in or all out
+#pragma unroll
+        for (int i = 0; i < 4; ++i) cr.x[i] = (kv && xv) ? __ldg(px + c * 16 + i) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            cr.wa[r] = (kv && va[r]) ? __ldg(pa[r] + c * 4) : make_uint4(0, 0, 0, 0);
+            cr.wb[r] = (kv && vb[r]) ? __ldg(pb[r] + c * 4) : make_uint4(0, 0, 0, 0);
+            cr.sa[r] = va[r] ? (f16 ? __half2float(__ldg(sah[r] + c)) : __ldg(saf[r] + c)) : 0.f;
+            cr.sb[r] = vb[r] ? (f16 ? __half2float(__ldg(sbh[r] + c)) : __ldg(sbf[r] + c)) : 0.f;
+        }
+    };
+    auto compute = [&](const ChunkRegs<R>& cr) {
+        // activation pairs (k, k+4) for every word of codes
+        uint32_t xb[16];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t x01 = cr.x[i].x, x23 = cr.x[i].y, x45 = cr.x[i].z, x67 = cr.x[i].w;
+            xb[4 * i + 0] = prmt(x01, x45, 0x5410u);  // (k0, k4)
+            xb[4 * i + 1] = prmt(x01, x45, 0x7632u);  // (k1, k5)
+            xb[4 * i + 2] = prmt(x23, x67, 0x5410u);  // (k2, k6)
+            xb[4 * i + 3] = prmt(x23, x67, 0x7632u);  // (k3, k7)
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            float part[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int wi = 0; wi < 4; ++wi) {
+                uint32_t qa[4], qb[4];
+                dequant8_exact<MANT>(word_of(cr.wa[r], wi), qa);
+                dequant8_exact<MANT>(word_of(cr.wb[r], wi), qb);
+                mma_bf16_16816(part, qa[0], qb[0], qa[1], qb[1], xb[4 * wi + 0], xb[4 * wi + 1]);
+                mma_bf16_16816(part, qa[2], qb[2], qa[3], qb[3], xb[4 * wi + 2], xb[4 * wi + 3]);
+            }
+            acc[r][0] = fmaf(cr.sa[r], part[0], acc[r][0]);
+            acc[r][1] = fmaf(cr.sa[r], part[1], acc[r][1]);
+            acc[r][2] = fmaf(cr.sb[r], part[2], acc[r][2]);
+            acc[r][3] = fmaf(cr.sb[r], part[3], acc[r][3]);
+        }
+    };
+
+    ChunkRegs<R> b0, b1;
+    if (c_begin < c_end) load(c_begin, b0);
+    for (int c = c_begin; c < c_end; c += 2) {
+        if (c + 1 < c_end) load(c + 1, b1);
+        compute(b0);
+        if (c + 2 < c_end) load(c + 2, b0);
+        if (c + 1 < c_end) compute(b1);
+    }
+
+    __shared__ float red[8][R][32][4];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) red[warp][r][lane][j] = acc[r][j];
+    __syncthreads();
+    const float rho = p.x_scale ? *p.x_scale : 1.f;
+    for (int e = threadIdx.x; e < R * 128; e += 256) {
+        const int r = e >> 7, l = (e >> 2) & 31, j = e & 3;
+        float sum = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) sum += red[w][r][l][j];
+        const int n = n0 + 16 * r + (l >> 2) + 8 * (j >> 1);
+        const int m = 2 * (l & 3) + (j & 1);
+        if (m < p.M && n < p.N) {
+            __nv_bfloat16 y = __float2bfloat16_rn(rho * sum);
+            p.Y[(size_t)m * p.N + n] = *reinterpret_cast<uint16_t*>(&y);
+        }
+    }
+}
+
+template <int R>
+static void launch_g128(const DecodeParams& p, int fmt, int blocks, cudaStream_t st) {
+    if (fmt == FP4_E1M2)
+        gemm_decode_g128_kernel<R, 2><<<blocks, 256, 0, st>>>(p);
+    else if (fmt == FP4_E2M1)
+        gemm_decode_g128_kernel<R, 1><<<blocks, 256, 0, st>>>(p);
+    else
+        gemm_decode_g128_kernel<R, 0><<<blocks, 256, 0, st>>>(p);
+}
+
 int decode_rows_per_cta(int N) { return N >= 16384 ? 2 : 1; }
 
 cudaError_t launch_gemm_decode(const uint16_t* X, const uint8_t* packed, const void* scales, int sdt,
-                               const FmtTable& t, int M, int N, int K, int group, const float* x_scale,
+                               const FmtTable& t, int fmt, int M, int N, int K, int group, const float* x_scale,
                                uint16_t* Y, cudaStream_t st) {
     DecodeParams p{X, packed, scales, sdt, t, M, N, K, group, x_scale, Y};
     const int R = decode_rows_per_cta(N);
     const int blocks = (N + 16 * R - 1) / (16 * R);
-    const bool lut_scale = group != 128;
-    if (R == 1) {
-        if (lut_scale)
-            gemm_decode_kernel<1, true><<<blocks, 256, 0, st>>>(p);
+    if (group == 128) {
+        if (R == 1)
+            launch_g128<1>(p, fmt, blocks, st);
         else
-            gemm_decode_kernel<1, false><<<blocks, 256, 0, st>>>(p);
+            launch_g128<2>(p, fmt, blocks, st);
+    } else if (R == 1) {
+        gemm_decode_kernel<1, true><<<blocks, 256, 0, st>>>(p);
     } else {
-        if (lut_scale)
-            gemm_decode_kernel<2, true><<<blocks, 256, 0, st>>>(p);
-        else
-            gemm_decode_kernel<2, false><<<blocks, 256, 0, st>>>(p);
+        gemm_decode_kernel<2, true><<<blocks, 256, 0, st>>>(p);
     }
     return cudaGetLastError();
 }

@@ -1,29 +1,37 @@
 // gemm_tc.cu -- W4A16 GEMM on the sm_100a tensor cores (tcgen05 + TMEM).
 //
-// Y[m,n] = bf16( rho * sum_k X[m,k] * v(code[n,k]) * s[n, k/g] )
+// Y[m,n] = bf16( rho * sum_g s[n,g] * sum_{k in g} X[m,k] * v(code[n,k]) )
 // (LLM-FP4 summary page "首个支持4-bit浮点量化的LLM来了", efficient matrix
-// multiplication; the group scale is applied while dequantizing, before the
-// bf16 product, so the tensor cores see plain bf16 operands.)
+// multiplication: the full-precision group scale stays outside the 4-bit
+// product.)  The tensor cores multiply the EXACT code values v (bf16 holds
+// every value of the three formats) by the bf16 activations with fp32
+// accumulation; each group's partial sum is scaled by s in fp32.  No
+// weight is ever rounded, so the only rounding besides fp32 accumulation
+// is the final bf16 store.
 //
-// CTA tile: 128 weight rows (MMA M) x BT activation rows (MMA N) x 64 k per
-// pipeline stage.  The product is computed transposed, D[n][m] = W . X^T,
-// so the 128 weight rows map onto the 128 TMEM lanes and the dequantizing
-// thread of row r is the thread that owns TMEM lane r.
+// CTA tile: 128 weight rows (MMA M) x BT activation rows (MMA N), 64 k per
+// pipeline stage.  The product is computed transposed, D[n][m] = W . X^T:
+// the 128 weight rows map onto the 128 TMEM lanes, so the per-row group
+// scale is a per-lane scalar.
 //
-// Warp roles (192 threads):
-//   warp 0      TMA producer: X tile (bf16, 128-byte swizzle) and the packed
-//               code tile (uint8 [128][32]) into a ring of smem stages;
-//   warp 1      TMEM allocator and MMA issuer: one thread issues 4
-//               tcgen05.mma (K = 16 each) per stage into an fp32 TMEM
-//               accumulator and commits the stage back to the producer;
-//   warps 2..5  dequantize the stage's codes into a bf16 K-major tile with
-//               the 128-byte swizzle (byte-plane LUT of bf16(v*s), 16-byte
-//               stores), then, after the last stage, run the epilogue:
-//               tcgen05.ld -> * rho -> bf16 -> global (or fp32 split-K
-//               partials, reduced in fixed order by the last CTA of a tile).
+// Warp roles (2 + DQW + NF warps):
+//   warp 0       TMA producer: X tile (bf16, 128-byte swizzle) and the
+//                packed code tile (uint8 [128][32], 32-byte swizzle) into a
+//                ring of shared-memory stages;
+//   warp 1       TMEM allocator and MMA issuer: one thread issues
+//                tcgen05.mma (K = 16) into one of two per-group TMEM
+//                accumulators, committing each finished group to the fold
+//                warps and each consumed stage back to the producer;
+//   DQW warps    dequantize codes into the exact bf16 values, K-major with
+//                the 128-byte swizzle (byte-plane LUT, 16-byte stores);
+//   NF warps     fold: for each group, tcgen05.ld the group accumulator and
+//                add s[n,g] * it to fp32 totals held in registers, then
+//                release the accumulator; finally the epilogue (* rho ->
+//                bf16 -> global, or fp32 split-K partials reduced in fixed
+//                order by the last CTA of the tile).
 // Every mbarrier wait is bounded; a wait that gives up sets
-// FP4_DEV_WAIT_TIMEOUT in the status word and the CTA winds down normally
-// (outstanding copies awaited, TMEM freed).  No multicast is used.
+// FP4_DEV_WAIT_TIMEOUT and the CTA winds down normally (its copies awaited,
+// TMEM freed).  No multicast is used.
 #include "common.cuh"
 
 namespace fp4 {
@@ -44,19 +52,43 @@ struct TcParams {
 
 template <int BT>
 struct TcCfg {
-    static constexpr int BW = 128;              // weight rows per tile (MMA M)
-    static constexpr int BK = 64;               // k per stage (one 128-byte swizzle row of bf16)
-    static constexpr int XBYTES = BT * 128;     // activation tile
-    static constexpr int WBYTES = BW * 128;     // dequantized weight tile
-    static constexpr int PBYTES = BW * 32;      // packed code tile
+    static constexpr int BW = 128;                 // weight rows per tile (MMA M)
+    static constexpr int BK = 64;                  // k per stage (one 128-byte swizzle row of bf16)
+    static constexpr int XBYTES = BT * 128;        // activation tile
+    static constexpr int WBYTES = BW * 128;        // dequantized weight tile
+    static constexpr int PBYTES = BW * 32;         // packed code tile
     static constexpr int STAGE = XBYTES + WBYTES + PBYTES;
-    static constexpr int STAGES = (220 * 1024) / STAGE > 8 ? 8 : (220 * 1024) / STAGE;
-    static constexpr int TMEM_COLS = BT < 32 ? 32 : BT;
+    // small token tiles (decode-sized problems) keep two CTAs per SM
+    static constexpr int BUDGET = BT <= 64 ? 110 * 1024 : 216 * 1024;
+    static constexpr int STAGES = BUDGET / STAGE > 8 ? 8 : BUDGET / STAGE;
+    static constexpr int CTAS_PER_SM = BT <= 64 ? 2 : 1;
+    static constexpr int FCOLS = BT < 64 ? BT : 64;  // accumulator columns per fold thread
+    static constexpr int FQ = BT / FCOLS;            // column blocks
+    static constexpr int NF = 4 * FQ;                // fold warps
+    static constexpr int DQW = BT >= 256 ? 2 : 4;    // dequant warps (each thread: 4 / DQW rows)
+    static constexpr int FW0 = 2 + DQW;              // first fold warp
+    static constexpr int THREADS = (FW0 + NF) * 32;
+    static constexpr int TMEM_COLS = 2 * BT;         // two group accumulators
     static constexpr int SMEM = STAGES * STAGE + 1024 + 256;
 };
 
+// The k-steps (16 wide) a CTA issues run from kbeg to kstop; groups split
+// them into fragments.  Fragment f covers group gfirst + f.
+struct KRange {
+    int kbeg, kstop, gfirst, nfrag;
+};
+
+__device__ __forceinline__ KRange k_range(const TcParams& p, int kb0, int kb1) {
+    KRange r;
+    r.kbeg = kb0 * 64;
+    r.kstop = min(kb1 * 64, p.K);
+    r.gfirst = r.kbeg / p.group;
+    r.nfrag = r.kstop > r.kbeg ? (r.kstop - 1) / p.group - r.gfirst + 1 : 0;
+    return r;
+}
+
 template <int BT>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, TcParams p) {
     using C = TcCfg<BT>;
     extern __shared__ uint8_t smem_raw[];
@@ -68,8 +100,9 @@ __global__ void __launch_bounds__(192, 1)
     uint64_t* full = bars;                                // TMA landed
     uint64_t* dq = bars + C::STAGES;                      // weight tile dequantized
     uint64_t* empty = bars + 2 * C::STAGES;               // MMA done with the stage
-    uint64_t* accf = bars + 3 * C::STAGES;                // accumulator complete
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * C::STAGES + 1);
+    uint64_t* gfull = bars + 3 * C::STAGES;               // [2] group accumulator complete
+    uint64_t* gempty = bars + 3 * C::STAGES + 2;          // [2] group accumulator folded
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * C::STAGES + 4);
     int* last_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -78,15 +111,19 @@ __global__ void __launch_bounds__(192, 1)
     const int kb0 = (int)((long long)split * kblocks / p.splits);
     const int kb1 = (int)((long long)(split + 1) * kblocks / p.splits);
     const int nkb = kb1 - kb0;
+    const KRange kr = k_range(p, kb0, kb1);
     const uint64_t to = p.timeout_ns;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&dq[s], 128);
+            mbar_init(&dq[s], C::DQW * 32);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(accf, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&gfull[b], 1);
+            mbar_init(&gempty[b], C::NF);
+        }
         fence_mbar_init();
         prefetch_tmap(&tmX);
         prefetch_tmap(&tmW);
@@ -129,119 +166,159 @@ __global__ void __launch_bounds__(192, 1)
         // ----------------------------------------------------- MMA issuer
         if (elect_one()) {
             const uint32_t idesc = idesc_bf16_f32(C::BW, BT);
-            for (int i = 0; i < nkb; ++i) {
+            int frag = -1;      // group fragment currently accumulating
+            int cur_group = -1;
+            bool ok = true;
+            for (int i = 0; i < nkb && ok; ++i) {
                 const int s = i % C::STAGES;
                 const uint32_t ph = (uint32_t)(i / C::STAGES) & 1u;
                 if (!mbar_wait(&dq[s], ph, to) || !mbar_wait(&full[s], ph, to)) {
                     raise_status(p.status, kStatusTimeout);
+                    ok = false;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t wa = smem_u32(ws + s * C::WBYTES);
                 const uint32_t xa = smem_u32(xs + s * C::XBYTES);
-#pragma unroll
-                for (int kk = 0; kk < C::BK / 16; ++kk)
-                    tc_mma_f16(tmem, sw128_desc(wa + kk * 32), sw128_desc(xa + kk * 32), idesc,
-                               (i > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll 1
+                for (int kk = 0; kk < C::BK / 16; ++kk) {
+                    const int k = (kb0 + i) * C::BK + kk * 16;
+                    if (k >= kr.kstop) break;
+                    const int g = k / p.group;
+                    if (g != cur_group) {
+                        // new group fragment: take the next accumulator once it is folded
+                        cur_group = g;
+                        ++frag;
+                        const int b = frag & 1;
+                        if (!mbar_wait(&gempty[b], ((uint32_t)(frag >> 1) & 1u) ^ 1u, to)) {
+                            raise_status(p.status, kStatusTimeout);
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                    }
+                    const int b = frag & 1;
+                    const bool first = (k == kr.kbeg) || (k % p.group == 0);
+                    tc_mma_f16(tmem + (uint32_t)(b * BT), sw128_desc(wa + kk * 32), sw128_desc(xa + kk * 32), idesc,
+                               first ? 0u : 1u);
+                    const bool last = (k + 16 >= kr.kstop) || ((k + 16) % p.group == 0);
+                    if (last) tc_commit(&gfull[b]);
+                }
                 tc_commit(&empty[s]);
             }
-            tc_commit(accf);  // arrives once every MMA issued above is complete
-            // TMEM is freed below: make sure no MMA is still writing it
-            if (!mbar_wait(accf, 0, to)) raise_status(p.status, kStatusTimeout);
+            // TMEM is freed below: the last group commit must have landed
+            if (frag >= 0 && !mbar_wait(&gfull[frag & 1], (uint32_t)(frag >> 1) & 1u, to))
+                raise_status(p.status, kStatusTimeout);
         }
         __syncwarp();
-    } else {
-        // ------------------------------------------- dequant + epilogue
-        const int q = warp & 3;        // TMEM lane quadrant of this warp
-        const int r = q * 32 + lane;   // weight row within the tile == TMEM lane
-        const int n = n0 + r;
-        const bool nvalid = n < p.N;
-        const int G = p.K / p.group;
-        int lut_group = -1;
-        Bf16Lut lut_a = make_lut(p.t.mag, 0.f), lut_b = lut_a;
-        bool ok = true;
+    } else if (warp < C::FW0) {
+        // ---------------------------------------------------- dequantize
+        const Bf16Lut lut = make_lut(p.t.mag, 1.f);
         for (int i = 0; i < nkb; ++i) {
             const int s = i % C::STAGES;
             const uint32_t ph = (uint32_t)(i / C::STAGES) & 1u;
-            const int k0 = (kb0 + i) * C::BK;
-            const int ga = k0 / p.group, gb = (k0 + 32) / p.group;
-            if (ga != lut_group) {
-                const float sa = (nvalid && k0 < p.K) ? load_scale(p.scales, p.sdt, (size_t)n * G + ga) : 0.f;
-                lut_a = make_lut(p.t.mag, sa);
-                lut_group = ga;
-            }
-            if (gb != ga) {
-                const float sb = (nvalid && k0 + 32 < p.K) ? load_scale(p.scales, p.sdt, (size_t)n * G + gb) : 0.f;
-                lut_b = make_lut(p.t.mag, sb);
-            } else {
-                lut_b = lut_a;
-            }
             if (!mbar_wait(&full[s], ph, to)) {
                 raise_status(p.status, kStatusTimeout);
-                ok = false;
                 break;
             }
-            const uint4* prow = reinterpret_cast<const uint4*>(ps + s * C::PBYTES + r * 32);
-            const uint4 w0 = prow[0], w1 = prow[1];
-            uint8_t* wrow = ws + s * C::WBYTES + r * 128;
-            const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint32_t v[4];
-                dequant8(words[c], c < 4 ? lut_a : lut_b, v);
-                *reinterpret_cast<uint4*>(wrow + ((c ^ (r & 7)) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
+            for (int rr = 0; rr < 4 / C::DQW; ++rr) {
+                const int r = (warp - 2 + rr * C::DQW) * 32 + lane;  // weight row within the tile
+                // packed tile has the 32-byte swizzle: 16-byte half h of row r
+                // sits at half h ^ ((r >> 2) & 1)
+                const uint8_t* prow = ps + s * C::PBYTES + r * 32;
+                const int sw = (r >> 2) & 1;
+                const uint4 w0 = *reinterpret_cast<const uint4*>(prow + ((0 ^ sw) << 4));
+                const uint4 w1 = *reinterpret_cast<const uint4*>(prow + ((1 ^ sw) << 4));
+                uint8_t* wrow = ws + s * C::WBYTES + r * 128;
+                const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t v[4];
+                    dequant8(words[c], lut, v);
+                    *reinterpret_cast<uint4*>(wrow + ((c ^ (r & 7)) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
+                }
             }
             fence_proxy_async_smem();
             mbar_arrive(&dq[s]);
         }
-        // epilogue
-        if (ok && !mbar_wait(accf, 0, to)) {
-            raise_status(p.status, kStatusTimeout);
-            ok = false;
-        }
-        tc_fence_after();
-        const float rho = p.x_scale ? *p.x_scale : 1.f;
-        const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
-        for (int c0 = 0; c0 < BT; c0 += 16) {
-            uint32_t v[16];
-            tmem_ld16(trow + c0, v);
-            tmem_ld_wait();
-            if (!ok || !nvalid) continue;
+    } else {
+        // ---------------------------------------------- fold + epilogue
+        const int fw = warp - C::FW0;
+        const int q = warp & 3;                  // TMEM lane quadrant of this warp
+        const int cb = (fw >> 2) * C::FCOLS;     // first accumulator column of this thread
+        const int r = q * 32 + lane;             // weight row within the tile == TMEM lane
+        const int n = n0 + r;
+        const bool nvalid = n < p.N;
+        const int G = p.K / p.group;
+        float tot[C::FCOLS];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const int m = m0 + c0 + j;
-                if (m >= p.M) break;
-                const float a = __uint_as_float(v[j]);
-                if (p.splits == 1) {
-                    __nv_bfloat16 y = __float2bfloat16_rn(rho * a);
-                    p.Y[(size_t)m * p.N + n] = *reinterpret_cast<uint16_t*>(&y);
-                } else {
-                    p.part[((size_t)split * p.M + m) * p.N + n] = a;
+        for (int j = 0; j < C::FCOLS; ++j) tot[j] = 0.f;
+        const uint32_t tlane = tmem + ((uint32_t)(q * 32) << 16);
+        bool ok = true;
+        float s_next = (nvalid && kr.nfrag > 0) ? load_scale(p.scales, p.sdt, (size_t)n * G + kr.gfirst) : 0.f;
+        for (int f = 0; f < kr.nfrag; ++f) {
+            const int b = f & 1;
+            const float s = s_next;
+            if (f + 1 < kr.nfrag)
+                s_next = nvalid ? load_scale(p.scales, p.sdt, (size_t)n * G + kr.gfirst + f + 1) : 0.f;
+            if (ok && !mbar_wait(&gfull[b], (uint32_t)(f >> 1) & 1u, to)) {
+                raise_status(p.status, kStatusTimeout);
+                ok = false;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < C::FCOLS; c += 16) {
+                uint32_t v[16];
+                tmem_ld16(tlane + (uint32_t)(b * BT + cb + c), v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) tot[c + j] = fmaf(s, __uint_as_float(v[j]), tot[c + j]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&gempty[b]);
+            if (!ok) break;
+        }
+        const float rho = p.x_scale ? *p.x_scale : 1.f;
+        if (ok && nvalid) {
+#pragma unroll
+            for (int j = 0; j < C::FCOLS; ++j) {
+                const int m = m0 + cb + j;
+                if (m < p.M) {
+                    if (p.splits == 1) {
+                        __nv_bfloat16 y = __float2bfloat16_rn(rho * tot[j]);
+                        p.Y[(size_t)m * p.N + n] = *reinterpret_cast<uint16_t*>(&y);
+                    } else {
+                        p.part[((size_t)split * p.M + m) * p.N + n] = tot[j];
+                    }
                 }
             }
         }
         if (p.splits > 1) {
             // the last CTA of this output tile sums the partials in split order
             __threadfence();
-            asm volatile("bar.sync 1, 128;" ::: "memory");
+            asm volatile("bar.sync 1, %0;" ::"r"(C::NF * 32) : "memory");
             const unsigned tile = blockIdx.y * gridDim.x + blockIdx.x;
-            if (threadIdx.x == 64) {
+            if (threadIdx.x == C::FW0 * 32) {
                 const unsigned old = atomicAdd(&p.counters[tile], 1u);
                 *last_flag = (old == (unsigned)p.splits - 1u) ? 1 : 0;
             }
-            asm volatile("bar.sync 1, 128;" ::: "memory");
+            asm volatile("bar.sync 1, %0;" ::"r"(C::NF * 32) : "memory");
             if (*last_flag) {
                 __threadfence();
                 if (nvalid) {
-                    const int mend = min(p.M, m0 + BT);
-                    for (int m = m0; m < mend; ++m) {
+#pragma unroll 4
+                    for (int j = 0; j < C::FCOLS; ++j) {
+                        const int m = m0 + cb + j;
+                        if (m >= p.M) break;
                         float a = 0.f;
                         for (int z = 0; z < p.splits; ++z) a += __ldcg(&p.part[((size_t)z * p.M + m) * p.N + n]);
                         __nv_bfloat16 y = __float2bfloat16_rn(rho * a);
                         p.Y[(size_t)m * p.N + n] = *reinterpret_cast<uint16_t*>(&y);
                     }
                 }
-                if (threadIdx.x == 64) p.counters[tile] = 0u;
+                if (threadIdx.x == C::FW0 * 32) p.counters[tile] = 0u;
             }
         }
     }
@@ -292,14 +369,16 @@ int tc_token_tile(int M) {
 }
 
 int tc_splits(int M, int N, int K) {
+    // split K only as far as one wave of CTAs covers the SMs
     const int BT = tc_token_tile(M);
     const long long tiles = (long long)((N + 127) / 128) * ((M + BT - 1) / BT);
     const int kblocks = (K + 63) / 64;
-    if (tiles >= 148 || tiles > 4096) return 1;
-    int s = (int)((2 * 148 + tiles - 1) / tiles);
-    s = s > kblocks / 4 ? kblocks / 4 : s;
+    const long long slots = 148LL * (BT <= 64 ? 2 : 1);
+    if (tiles >= slots / 2 || tiles > 4096) return 1;
+    long long s = slots / tiles;
+    if (s > kblocks / 4) s = kblocks / 4;
     if (s > 16) s = 16;
-    return s < 1 ? 1 : s;
+    return s < 1 ? 1 : (int)s;
 }
 
 size_t tc_ws_bytes(int M, int N, int K) {
@@ -320,7 +399,7 @@ static cudaError_t launch_tc_bt(const CUtensorMap& mx, const CUtensorMap& mw, co
         attr_set[dev] = true;
     }
     dim3 grid((p.N + C::BW - 1) / C::BW, (p.M + BT - 1) / BT, p.splits);
-    gemm_tc_kernel<BT><<<grid, 192, C::SMEM, st>>>(mx, mw, p);
+    gemm_tc_kernel<BT><<<grid, C::THREADS, C::SMEM, st>>>(mx, mw, p);
     return cudaGetLastError();
 }
 
@@ -342,7 +421,7 @@ cudaError_t launch_gemm_tc(const uint16_t* X, const uint8_t* packed, const void*
                    CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     if (!encode_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, packed, (uint64_t)K / 2, (uint64_t)N, 32, 128,
-                   CU_TENSOR_MAP_SWIZZLE_NONE))
+                   CU_TENSOR_MAP_SWIZZLE_32B))
         return cudaErrorInvalidValue;
     TcParams p;
     p.scales = scales;

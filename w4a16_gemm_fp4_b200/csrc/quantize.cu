@@ -24,6 +24,7 @@ namespace fp4 {
 
 constexpr int kQuantThreads = 256;
 constexpr int kSearchBlocksMax = 1184;  // fixed (shape-only) grid cap => deterministic SSE order
+constexpr int kUnroll = 4;             // units (128 weights) per warp iteration in the packing pass
 
 struct QuantParams {
     const float* W;
@@ -121,41 +122,48 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(QuantParams p, 
     }
     double sse = 0.0;
     bool bad = false, ovf = false;
-    for (long long u = wid; u < units; u += nw) {
-        const long long base = u * 128;
-        float w[4];
-        const bool valid = load4(p, base, w);
-        float a = 0.f;
+    // kUnroll consecutive units per warp iteration: their loads are all in
+    // flight before the first one is used
+    for (long long u0 = wid * kUnroll; u0 < units; u0 += nw * kUnroll) {
+        float w[kUnroll][4];
+        bool valid[kUnroll];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            bad |= valid && !isfinite(w[i]);
-            a = fmaxf(a, fabsf(w[i]));
-        }
-        const float A = group_absmax(a, lpg);
-        bool o;
-        uint32_t raw;
-        const float s = stored_scale(A, cj, t.qmax, p.sdt, &o, &raw);
-        if (!valid) continue;
-        ovf |= o;
-        uint32_t codes = 0;
+        for (int q = 0; q < kUnroll; ++q) valid[q] = load4(p, (u0 + q) * 128, w[q]);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            float v;
-            const int c = code_of(w[i], s, t, &v);
-            codes |= (uint32_t)c << (4 * i);
-            if (ws_sse) {
-                const double d = (double)w[i] - (double)v * (double)s;
-                sse = fma(d, d, sse);
+        for (int q = 0; q < kUnroll; ++q) {
+            const long long base = (u0 + q) * 128;
+            float a = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                bad |= valid[q] && !isfinite(w[q][i]);
+                a = fmaxf(a, fabsf(w[q][i]));
             }
-        }
-        const long long off = base + 4 * lane;
-        *reinterpret_cast<uint16_t*>(p.packed + off / 2) = (uint16_t)codes;
-        if ((lane & (lpg - 1)) == 0) {
-            const long long gi = off / p.group;
-            if (p.sdt == FP4_SCALE_F16)
-                reinterpret_cast<uint16_t*>(p.scales)[gi] = (uint16_t)raw;
-            else
-                reinterpret_cast<uint32_t*>(p.scales)[gi] = raw;
+            const float A = group_absmax(a, lpg);
+            bool o;
+            uint32_t raw;
+            const float s = stored_scale(A, cj, t.qmax, p.sdt, &o, &raw);
+            if (!valid[q]) continue;
+            ovf |= o;
+            uint32_t codes = 0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float v;
+                const int c = code_of(w[q][i], s, t, &v);
+                codes |= (uint32_t)c << (4 * i);
+                if (ws_sse) {
+                    const double d = (double)w[q][i] - (double)v * (double)s;
+                    sse = fma(d, d, sse);
+                }
+            }
+            const long long off = base + 4 * lane;
+            *reinterpret_cast<uint16_t*>(p.packed + off / 2) = (uint16_t)codes;
+            if ((lane & (lpg - 1)) == 0) {
+                const long long gi = off / p.group;
+                if (p.sdt == FP4_SCALE_F16)
+                    reinterpret_cast<uint16_t*>(p.scales)[gi] = (uint16_t)raw;
+                else
+                    reinterpret_cast<uint32_t*>(p.scales)[gi] = raw;
+            }
         }
     }
     if (bad) raise_status(p.status, kStatusNonfinite);
@@ -318,14 +326,18 @@ cudaError_t launch_quantize(const float* W, int N, int K, int group, int fmt, in
     const int jn = bias_search ? 8 : 1;
     const bool search = (f0 != f1) || jn > 1;
     const int blocks = quantize_grid_blocks(p.total);
+    // the packing pass takes kUnroll units per warp iteration
+    const long long pack_units = ((p.total + 127) / 128 + kUnroll - 1) / kUnroll;
+    int pblocks = (int)((pack_units + (kQuantThreads / 32) - 1) / (kQuantThreads / 32));
+    pblocks = pblocks < 1 ? 1 : (pblocks > kSearchBlocksMax ? kSearchBlocksMax : pblocks);
     double* wsd = reinterpret_cast<double*>(ws);
     if (search) {
         search_kernel<<<blocks, kQuantThreads, 0, st>>>(p, tabs, f0, f1, jn, wsd);
         search_finalize_kernel<<<1, 32, 0, st>>>(wsd, blocks, f0, f1, jn, choice, sse);
-        quantize_kernel<<<blocks, kQuantThreads, 0, st>>>(p, tabs, 0, 0, choice, nullptr, nullptr);
+        quantize_kernel<<<pblocks, kQuantThreads, 0, st>>>(p, tabs, 0, 0, choice, nullptr, nullptr);
     } else {
-        quantize_kernel<<<blocks, kQuantThreads, 0, st>>>(p, tabs, f0, 0, nullptr, choice, sse ? wsd : nullptr);
-        if (sse) sse_single_finalize_kernel<<<1, 32, 0, st>>>(wsd, blocks, f0, 0, sse);
+        quantize_kernel<<<pblocks, kQuantThreads, 0, st>>>(p, tabs, f0, 0, nullptr, choice, sse ? wsd : nullptr);
+        if (sse) sse_single_finalize_kernel<<<1, 32, 0, st>>>(wsd, pblocks, f0, 0, sse);
     }
     return cudaGetLastError();
 }
