@@ -162,14 +162,15 @@ FP4_API fp4_status fp4_preshift_apply(const uint16_t *X, int M, int K, const int
  *   fmt      the format the weights were quantized in (not AUTO).
  *   x_scale  device float (rho from fp4_preshift_calibrate) or NULL for 1.
  *   Y        [M][N] bf16 out; must not alias the inputs.
- *   workspace device scratch of fp4_gemm_workspace_size(M, N, K) bytes.  It
- *            must be ZERO-FILLED before its first use; every call leaves it
- *            ready for the next one.  Calls that may run concurrently need
- *            separate workspaces.  NULL (with ws_bytes 0) is accepted and
- *            disables split-K, which is slower for skinny problems.
- * Engines: M <= 8 uses the decode engine (streams the packed weights with
- * 128-bit loads, dequantizes in registers, warp-level MMAs); larger M uses
- * the tensor engine (TMA-staged tiles, tcgen05 MMAs into tensor memory).
+ *   workspace reserved: fp4_gemm_workspace_size() is 0 for every shape (the
+ *            split-K reduction of skinny problems runs between the CTAs of a
+ *            thread-block cluster in distributed shared memory); pass NULL, 0.
+ * Engines: M <= 8 uses the decode engine (per-warp TMA rings of packed
+ * codes, dequantization in registers, warp-level MMAs); larger M uses the
+ * tensor engine (TMA-staged tiles, tcgen05 MMAs into tensor memory).  Both
+ * multiply the exact code values and apply each group scale in fp32.
+ * The decode engine's E2M1 path runs its MMAs in f16: activations must lie
+ * within the fp16 range (|x| < 65504); smaller than 2^-14 they lose bits.
  * Device status: FP4_DEV_WAIT_TIMEOUT.
  * ---------------------------------------------------------------------- */
 FP4_API size_t fp4_gemm_workspace_size(int M, int N, int K);
@@ -178,8 +179,8 @@ FP4_API fp4_status fp4_gemm(const uint16_t *X, const uint8_t *packed, const void
                     const float *x_scale, uint16_t *Y, void *workspace, size_t ws_bytes,
                     cudaStream_t stream);
 
-/* fp4_gemm with an explicit engine and split-K count (0 = automatic);
- * meant for tests and tuning.  The decode engine accepts M <= 8 only. */
+/* fp4_gemm with an explicit engine and split-K count (0 = automatic, at
+ * most 8); meant for tests and tuning.  The decode engine accepts M <= 8. */
 FP4_API fp4_status fp4_gemm_ex(const uint16_t *X, const uint8_t *packed, const void *scales,
                        fp4_scale_dtype sdt, fp4_format fmt, int M, int N, int K, int group,
                        const float *x_scale, uint16_t *Y, void *workspace, size_t ws_bytes,

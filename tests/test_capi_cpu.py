@@ -107,7 +107,7 @@ def test_preshift_argument_errors(L):
 
 def test_workspace_sizes(L):
     assert L.fp4_gemm_workspace_size(1, 4096, 4096) == 0        # decode engine: none
-    assert L.fp4_gemm_workspace_size(64, 4096, 4096) > 0        # skinny tensor problem: split-K
+    assert L.fp4_gemm_workspace_size(64, 4096, 4096) == 0       # split-K reduces in a CTA cluster
     assert L.fp4_gemm_workspace_size(2048, 4096, 4096) == 0     # enough tiles: no split
     assert L.fp4_quantize_workspace_size(4096, 4096, 128, 1, 0) >= 8
     assert L.fp4_preshift_workspace_size(2048, 4096) >= 4096 * 4

@@ -237,7 +237,7 @@ def test_gemm_tensor_engine(fp4, oracle_mod, M, N, K, group):
     assert gemm_case(fp4, oracle_mod, 11 * M + N, N, K, M, group=group, engine=fp4.ENGINE_TENSOR) <= TOL
 
 
-@pytest.mark.parametrize("splits", [1, 2, 3, 5])
+@pytest.mark.parametrize("splits", [1, 2, 3, 5, 8])
 def test_gemm_tensor_split_k(fp4, oracle_mod, splits):
     assert gemm_case(fp4, oracle_mod, 5, 256, 1024, 40, engine=fp4.ENGINE_TENSOR, splits=splits, rho=2.5) <= TOL
 

@@ -22,7 +22,7 @@ cudaError_t launch_apply(const uint16_t* X, int M, int K, const int8_t* shift, c
                          cudaStream_t st);
 cudaError_t launch_gemm_decode(const uint16_t* X, const uint8_t* packed, const void* scales, int sdt,
                                const FmtTable& t, int fmt, int M, int N, int K, int group, const float* x_scale,
-                               uint16_t* Y, cudaStream_t st);
+                               uint16_t* Y, int* status, unsigned long long timeout_ns, cudaStream_t st);
 size_t tc_ws_bytes(int M, int N, int K);
 cudaError_t launch_gemm_tc(const uint16_t* X, const uint8_t* packed, const void* scales, int sdt, const FmtTable& t,
                            int M, int N, int K, int group, const float* x_scale, uint16_t* Y, void* ws,
@@ -249,16 +249,17 @@ fp4_status fp4_gemm_ex(const uint16_t* X, const uint8_t* packed, const void* sca
     if (!aligned(X, 16)) return FP4_ERR_MISALIGNED;
     if ((const void*)Y == (const void*)X || (const void*)Y == (const void*)packed) return FP4_ERR_INVALID_ARG;
     if (engine == FP4_ENGINE_AUTO) engine = M <= kDecodeMaxM ? FP4_ENGINE_DECODE : FP4_ENGINE_TENSOR;
+    if (engine == FP4_ENGINE_DECODE && M > kDecodeMaxM) return FP4_ERR_UNSUPPORTED_SHAPE;
     const FmtTable& t = tables().f[fmt];
-    if (engine == FP4_ENGINE_DECODE) {
-        if (M > kDecodeMaxM) return FP4_ERR_UNSUPPORTED_SHAPE;
-        return cuda_status(
-            launch_gemm_decode(X, packed, scales, (int)sdt, t, (int)fmt, M, N, K, group, x_scale, Y, stream));
-    }
     int* st = status_ptr();
     if (!st) return FP4_ERR_CUDA;
+    const unsigned long long to_ns = (unsigned long long)g_timeout_us * 1000ull;
+    if (engine == FP4_ENGINE_DECODE) {
+        return cuda_status(launch_gemm_decode(X, packed, scales, (int)sdt, t, (int)fmt, M, N, K, group, x_scale, Y,
+                                              st, to_ns, stream));
+    }
     return cuda_status(launch_gemm_tc(X, packed, scales, (int)sdt, t, M, N, K, group, x_scale, Y, workspace,
-                                      ws_bytes, splits, st, (unsigned long long)g_timeout_us * 1000ull, stream));
+                                      ws_bytes, splits, st, to_ns, stream));
 }
 
 fp4_status fp4_gemm(const uint16_t* X, const uint8_t* packed, const void* scales, fp4_scale_dtype sdt,

@@ -43,9 +43,7 @@ struct TcParams {
     int M, N, K, group;
     const float* x_scale;
     uint16_t* Y;
-    float* part;         // [splits][M][N] fp32 partials (splits > 1)
-    unsigned* counters;  // one per output tile (splits > 1)
-    int splits;
+    int splits;          // CTAs along K per output tile (one cluster)
     int* status;
     unsigned long long timeout_ns;
 };
@@ -65,9 +63,11 @@ struct TcCfg {
     static constexpr int FCOLS = BT < 64 ? BT : 64;  // accumulator columns per fold thread
     static constexpr int FQ = BT / FCOLS;            // column blocks
     static constexpr int NF = 4 * FQ;                // fold warps
-    static constexpr int DQW = BT >= 256 ? 2 : 4;    // dequant warps (each thread: 4 / DQW rows)
-    static constexpr int FW0 = 2 + DQW;              // first fold warp
+    static constexpr int DQW = 4;                    // dequant warps (one weight row per thread)
+    static constexpr int DQ0 = 2;                    // first dequant warp
+    static constexpr int FW0 = DQ0 + DQW;            // first fold warp
     static constexpr int THREADS = (FW0 + NF) * 32;
+    static_assert(BT <= 128, "fold totals of wider tiles do not fit in registers");
     static constexpr int TMEM_COLS = 2 * BT;         // two group accumulators
     static constexpr int SMEM = STAGES * STAGE + 1024 + 256;
 };
@@ -103,7 +103,6 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
     uint64_t* gfull = bars + 3 * C::STAGES;               // [2] group accumulator complete
     uint64_t* gempty = bars + 3 * C::STAGES + 2;          // [2] group accumulator folded
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * C::STAGES + 4);
-    int* last_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = blockIdx.x * C::BW, m0 = blockIdx.y * BT, split = blockIdx.z;
@@ -166,6 +165,7 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
         // ----------------------------------------------------- MMA issuer
         if (elect_one()) {
             const uint32_t idesc = idesc_bf16_f32(C::BW, BT);
+            const int gshift = __ffs(p.group) - 1, gmask = p.group - 1;  // group is a power of two
             int frag = -1;      // group fragment currently accumulating
             int cur_group = -1;
             bool ok = true;
@@ -184,7 +184,7 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
                 for (int kk = 0; kk < C::BK / 16; ++kk) {
                     const int k = (kb0 + i) * C::BK + kk * 16;
                     if (k >= kr.kstop) break;
-                    const int g = k / p.group;
+                    const int g = k >> gshift;
                     if (g != cur_group) {
                         // new group fragment: take the next accumulator once it is folded
                         cur_group = g;
@@ -198,10 +198,10 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
                         tc_fence_after();
                     }
                     const int b = frag & 1;
-                    const bool first = (k == kr.kbeg) || (k % p.group == 0);
+                    const bool first = (k == kr.kbeg) || ((k & gmask) == 0);
                     tc_mma_f16(tmem + (uint32_t)(b * BT), sw128_desc(wa + kk * 32), sw128_desc(xa + kk * 32), idesc,
                                first ? 0u : 1u);
-                    const bool last = (k + 16 >= kr.kstop) || ((k + 16) % p.group == 0);
+                    const bool last = (k + 16 >= kr.kstop) || (((k + 16) & gmask) == 0);
                     if (last) tc_commit(&gfull[b]);
                 }
                 tc_commit(&empty[s]);
@@ -211,9 +211,11 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
                 raise_status(p.status, kStatusTimeout);
         }
         __syncwarp();
-    } else if (warp < C::FW0) {
+    } else if (warp >= C::DQ0 && warp < C::FW0) {
         // ---------------------------------------------------- dequantize
         const Bf16Lut lut = make_lut(p.t.mag, 1.f);
+        const int r = (warp - C::DQ0) * 32 + lane;  // weight row within the tile
+        const int sw = (r >> 2) & 1;                // 32-byte swizzle of the packed tile
         for (int i = 0; i < nkb; ++i) {
             const int s = i % C::STAGES;
             const uint32_t ph = (uint32_t)(i / C::STAGES) & 1u;
@@ -221,28 +223,22 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
                 raise_status(p.status, kStatusTimeout);
                 break;
             }
+            // 16-byte half h of row r sits at half h ^ ((r >> 2) & 1)
+            const uint8_t* prow = ps + s * C::PBYTES + r * 32;
+            const uint4 w0 = *reinterpret_cast<const uint4*>(prow + ((0 ^ sw) << 4));
+            const uint4 w1 = *reinterpret_cast<const uint4*>(prow + ((1 ^ sw) << 4));
+            uint8_t* wrow = ws + s * C::WBYTES + r * 128;
+            const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-            for (int rr = 0; rr < 4 / C::DQW; ++rr) {
-                const int r = (warp - 2 + rr * C::DQW) * 32 + lane;  // weight row within the tile
-                // packed tile has the 32-byte swizzle: 16-byte half h of row r
-                // sits at half h ^ ((r >> 2) & 1)
-                const uint8_t* prow = ps + s * C::PBYTES + r * 32;
-                const int sw = (r >> 2) & 1;
-                const uint4 w0 = *reinterpret_cast<const uint4*>(prow + ((0 ^ sw) << 4));
-                const uint4 w1 = *reinterpret_cast<const uint4*>(prow + ((1 ^ sw) << 4));
-                uint8_t* wrow = ws + s * C::WBYTES + r * 128;
-                const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    uint32_t v[4];
-                    dequant8(words[c], lut, v);
-                    *reinterpret_cast<uint4*>(wrow + ((c ^ (r & 7)) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
-                }
+            for (int c = 0; c < 8; ++c) {
+                uint32_t v[4];
+                dequant8(words[c], lut, v);
+                *reinterpret_cast<uint4*>(wrow + ((c ^ (r & 7)) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
             }
             fence_proxy_async_smem();
             mbar_arrive(&dq[s]);
         }
-    } else {
+    } else if (warp >= C::FW0) {
         // ---------------------------------------------- fold + epilogue
         const int fw = warp - C::FW0;
         const int q = warp & 3;                  // TMEM lane quadrant of this warp
@@ -280,47 +276,57 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
             if (lane == 0) mbar_arrive(&gempty[b]);
             if (!ok) break;
         }
-        const float rho = p.x_scale ? *p.x_scale : 1.f;
-        if (ok && nvalid) {
+        if (p.splits == 1) {
+            const float rho = p.x_scale ? *p.x_scale : 1.f;
+            if (ok && nvalid) {
 #pragma unroll
-            for (int j = 0; j < C::FCOLS; ++j) {
-                const int m = m0 + cb + j;
-                if (m < p.M) {
-                    if (p.splits == 1) {
+                for (int j = 0; j < C::FCOLS; ++j) {
+                    const int m = m0 + cb + j;
+                    if (m < p.M) {
                         __nv_bfloat16 y = __float2bfloat16_rn(rho * tot[j]);
                         p.Y[(size_t)m * p.N + n] = *reinterpret_cast<uint16_t*>(&y);
-                    } else {
-                        p.part[((size_t)split * p.M + m) * p.N + n] = tot[j];
                     }
                 }
             }
+        } else {
+            // split-K: publish this CTA's fp32 partial tile [BT tokens][128 rows]
+            // in shared memory (the dequant stages are idle once the last group
+            // has been folded) for the cluster reduction below
+            float* part = reinterpret_cast<float*>(ws);
+#pragma unroll
+            for (int j = 0; j < C::FCOLS; ++j) part[(cb + j) * 128 + r] = tot[j];
         }
-        if (p.splits > 1) {
-            // the last CTA of this output tile sums the partials in split order
-            __threadfence();
-            asm volatile("bar.sync 1, %0;" ::"r"(C::NF * 32) : "memory");
-            const unsigned tile = blockIdx.y * gridDim.x + blockIdx.x;
-            if (threadIdx.x == C::FW0 * 32) {
-                const unsigned old = atomicAdd(&p.counters[tile], 1u);
-                *last_flag = (old == (unsigned)p.splits - 1u) ? 1 : 0;
-            }
-            asm volatile("bar.sync 1, %0;" ::"r"(C::NF * 32) : "memory");
-            if (*last_flag) {
-                __threadfence();
-                if (nvalid) {
-#pragma unroll 4
-                    for (int j = 0; j < C::FCOLS; ++j) {
-                        const int m = m0 + cb + j;
-                        if (m >= p.M) break;
-                        float a = 0.f;
-                        for (int z = 0; z < p.splits; ++z) a += __ldcg(&p.part[((size_t)z * p.M + m) * p.N + n]);
-                        __nv_bfloat16 y = __float2bfloat16_rn(rho * a);
-                        p.Y[(size_t)m * p.N + n] = *reinterpret_cast<uint16_t*>(&y);
-                    }
+    }
+
+    if (p.splits > 1) {
+        // The splits of one output tile form a thread-block cluster along z.
+        // Every CTA sums, in rank order, one slice of tokens over the partial
+        // tiles of all CTAs of the cluster (distributed shared memory).
+        cluster_sync();
+        if (warp >= C::FW0) {
+            const int f = threadIdx.x - C::FW0 * 32;
+            const int r = f & 127, h = f >> 7, hstep = (C::NF * 32) >> 7;
+            const int n = n0 + r;
+            const int rank = (int)cluster_ctarank();
+            const int j0 = rank * BT / p.splits, j1 = (rank + 1) * BT / p.splits;
+            const float rho = p.x_scale ? *p.x_scale : 1.f;
+            const uint32_t base = smem_u32(ws);
+            for (int j = j0 + h; j < j1; j += hstep) {
+                const int m = m0 + j;
+                const uint32_t off = base + (uint32_t)((j * 128 + r) * 4);
+                float v[8];
+#pragma unroll
+                for (int z = 0; z < 8; ++z) v[z] = z < p.splits ? ld_dsmem_f32(map_dsmem(off, (uint32_t)z)) : 0.f;
+                float a = 0.f;
+#pragma unroll
+                for (int z = 0; z < 8; ++z) a += v[z];
+                if (m < p.M && n < p.N) {
+                    __nv_bfloat16 y = __float2bfloat16_rn(rho * a);
+                    p.Y[(size_t)m * p.N + n] = *reinterpret_cast<uint16_t*>(&y);
                 }
-                if (threadIdx.x == C::FW0 * 32) p.counters[tile] = 0u;
             }
         }
+        cluster_sync();  // no CTA leaves while its partials are being read
     }
 
     tc_fence_before();
@@ -348,7 +354,7 @@ static EncodeTiledFn get_encode_fn() {
     return fn;
 }
 
-static bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, int elem_bytes, const void* base, uint64_t inner,
+bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, int elem_bytes, const void* base, uint64_t inner,
                       uint64_t outer, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
     EncodeTiledFn fn = get_encode_fn();
     if (!fn) return false;
@@ -364,27 +370,28 @@ static bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, int elem_bytes, 
 int tc_token_tile(int M) {
     if (M <= 32) return 32;
     if (M <= 64) return 64;
-    if (M <= 128) return 128;
-    return 256;
+    return 128;
 }
 
 int tc_splits(int M, int N, int K) {
-    // split K only as far as one wave of CTAs covers the SMs
+    // split K (a cluster of at most 8 CTAs per output tile) only as far as
+    // one wave of CTAs covers the SMs
     const int BT = tc_token_tile(M);
     const long long tiles = (long long)((N + 127) / 128) * ((M + BT - 1) / BT);
     const int kblocks = (K + 63) / 64;
     const long long slots = 148LL * (BT <= 64 ? 2 : 1);
-    if (tiles >= slots / 2 || tiles > 4096) return 1;
+    if (tiles >= slots / 2) return 1;
     long long s = slots / tiles;
     if (s > kblocks / 4) s = kblocks / 4;
-    if (s > 16) s = 16;
+    if (s > 8) s = 8;
     return s < 1 ? 1 : (int)s;
 }
 
 size_t tc_ws_bytes(int M, int N, int K) {
-    const int s = tc_splits(M, N, K);
-    if (s <= 1) return 0;
-    return 4096 * sizeof(unsigned) + (size_t)s * M * N * sizeof(float);
+    (void)M;
+    (void)N;
+    (void)K;
+    return 0;  // the split-K reduction runs in distributed shared memory
 }
 
 template <int BT>
@@ -399,7 +406,20 @@ static cudaError_t launch_tc_bt(const CUtensorMap& mx, const CUtensorMap& mw, co
         attr_set[dev] = true;
     }
     dim3 grid((p.N + C::BW - 1) / C::BW, (p.M + BT - 1) / BT, p.splits);
-    gemm_tc_kernel<BT><<<grid, C::THREADS, C::SMEM, st>>>(mx, mw, p);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(C::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = (unsigned)p.splits;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BT>, mx, mw, p);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
@@ -409,13 +429,11 @@ cudaError_t launch_gemm_tc(const uint16_t* X, const uint8_t* packed, const void*
                            cudaStream_t st) {
     const int BT = tc_token_tile(M);
     const int kblocks = (K + 63) / 64;
+    (void)ws;
+    (void)ws_bytes;
     if (splits <= 0) splits = tc_splits(M, N, K);
     if (splits > kblocks) splits = kblocks;
-    const long long tiles = (long long)((N + 127) / 128) * ((M + BT - 1) / BT);
-    if (splits > 1) {
-        const size_t need = 4096 * sizeof(unsigned) + (size_t)splits * M * N * sizeof(float);
-        if (!ws || ws_bytes < need || tiles > 4096) splits = 1;
-    }
+    if (splits > 8) splits = 8;
     CUtensorMap mx, mw;
     if (!encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, (uint64_t)K, (uint64_t)M, 64, (uint32_t)BT,
                    CU_TENSOR_MAP_SWIZZLE_128B))
@@ -433,16 +451,13 @@ cudaError_t launch_gemm_tc(const uint16_t* X, const uint8_t* packed, const void*
     p.group = group;
     p.x_scale = x_scale;
     p.Y = Y;
-    p.counters = splits > 1 ? reinterpret_cast<unsigned*>(ws) : nullptr;
-    p.part = splits > 1 ? reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + 4096 * sizeof(unsigned)) : nullptr;
     p.splits = splits;
     p.status = status;
     p.timeout_ns = timeout_ns;
     switch (BT) {
         case 32: return launch_tc_bt<32>(mx, mw, p, st);
         case 64: return launch_tc_bt<64>(mx, mw, p, st);
-        case 128: return launch_tc_bt<128>(mx, mw, p, st);
-        default: return launch_tc_bt<256>(mx, mw, p, st);
+        default: return launch_tc_bt<128>(mx, mw, p, st);
     }
 }
 
