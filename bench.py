@@ -204,16 +204,21 @@ def run_ours(args, world, rank):
         for s in range(args.warmup):          # eager warm-up (also loads modules, sets attributes)
             sweep(s % copies)
     torch.cuda.synchronize()
-    # one graph per weight copy; each holds the 12 launches and an event pair around each launch
-    graphs, gevents = [], []
+    # one graph per weight copy holding the 12 launches back to back; a
+    # second set with an event pair around every launch gives the per-kernel
+    # durations (event nodes serialise the launches, so they are kept out of
+    # the graphs that time the step)
+    graphs = [capture(torch, lambda c=c: sweep(c), stream) for c in range(copies)]
+    igraphs, gevents = [], []
     for c in range(copies):
         evs = {k: (torch.cuda.Event(enable_timing=True, external=True),
                    torch.cuda.Event(enable_timing=True, external=True)) for k in keys}
-        graphs.append(capture(torch, lambda c=c, evs=evs: sweep(c, evs), stream))
+        igraphs.append(capture(torch, lambda c=c, evs=evs: sweep(c, evs), stream))
         gevents.append(evs)
     with torch.cuda.stream(stream):
         for s in range(args.warmup):
             graphs[s % copies].replay()
+            igraphs[s % copies].replay()
     torch.cuda.synchronize()
     api.device_status(clear=True)
 
@@ -242,11 +247,21 @@ def run_ours(args, world, rank):
     barrier(world)
     clk = clocks.stop()
     ms = max_over_ranks(world, t0.elapsed_time(t1))
+    # per-launch durations over a second timed region of instrumented replays
+    per_sum = {k: 0.0 for k in keys}
+    reps = max(copies, min(args.steps, 200) // copies * copies)
+    with torch.cuda.stream(stream):
+        for s in range(reps):
+            igraphs[s % copies].replay()
+            if s % copies == copies - 1:
+                stream.synchronize()
+                for k in keys:
+                    per_sum[k] += sum(ev[k][0].elapsed_time(ev[k][1]) for ev in gevents)
+    torch.cuda.synchronize()
+    per = {k: v / reps for k, v in per_sum.items()}
     st = api.device_status(clear=True)
     if st:
         raise RuntimeError("device status %#x during the timed region" % st)
-    # per-launch durations: the last replay of every graph (the final `copies` steps of the timed region)
-    per = {k: statistics.mean(ev[k][0].elapsed_time(ev[k][1]) for ev in gevents) for k in keys}
 
     total_bytes = step_weight_bytes() * args.steps * world
     value = total_bytes / (ms * 1e-3) / 1e9

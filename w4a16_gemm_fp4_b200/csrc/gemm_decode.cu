@@ -248,6 +248,8 @@ __global__ void __launch_bounds__(256, 2)
     __syncwarp();
     fence_proxy_async_smem();
     __syncwarp();
+    pdl_wait();  // inputs may come from the previous kernel in the stream
+    pdl_launch_dependents();
 
     if (lane == 0) {
         for (int c = c_begin; c < c_end && c < c_begin + RG::STAGES; ++c) {
@@ -401,9 +403,17 @@ static cudaError_t launch_g128_t(const CUtensorMap& mw, const CUtensorMap& mx, c
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
-    gemm_decode_g128_kernel<R, MANT, SDT>
-        <<<(p.N + 16 * R - 1) / (16 * R), 256, DecodeRing<R>::SMEM, st>>>(mw, mx, p, status, to);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((p.N + 16 * R - 1) / (16 * R), 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.dynamicSmemBytes = DecodeRing<R>::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemm_decode_g128_kernel<R, MANT, SDT>, mw, mx, p, status, to);
 }
 
 template <int R>
