@@ -152,6 +152,24 @@ FP4_API fp4_status fp4_preshift_apply(const uint16_t *X, int M, int K, const int
                               uint16_t *Xt, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * fp4_preshift_calibrate_noalloc -- the method has no counterpart for this
+ * call: it is fp4_preshift_calibrate for callers that cannot obtain device
+ * memory when they calibrate (for instance a runtime that fixes its whole
+ * device-memory plan at start-up and forbids allocation afterwards, or a
+ * plug-in that receives tensors but no allocator).  It takes no workspace
+ * and allocates nothing; its scratch is a 256 KB buffer inside the library
+ * that every GPU loading the library keeps until the process exits.
+ *   Same arguments and results as fp4_preshift_calibrate (bit-identical
+ *   shift and rho).  K must be <= 65536: larger K returns FP4_ERR_WORKSPACE.
+ *   The first call on a device looks up the buffer's device address (with
+ *   that device current); make that first call before any stream capture.
+ *   All calls share the buffer: calls whose work overlaps on a GPU race and
+ *   must be ordered by the caller.  No part of it needs initialising.
+ * ---------------------------------------------------------------------- */
+FP4_API fp4_status fp4_preshift_calibrate_noalloc(const uint16_t *X, int M, int K, int8_t *shift, float *rho,
+                                                  cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * fp4_gemm -- Y = bf16( x_scale * X . dequant(W)^T ), fp32 accumulation.
  * (LLM-FP4 summary page, efficient matrix multiplication: the per-group
  * scales are applied outside the 4-bit products.)

@@ -27,7 +27,7 @@ STATUS = {0: "FP4_OK", 1: "FP4_ERR_INVALID_ARG", 2: "FP4_ERR_UNSUPPORTED_SHAPE",
 EXPORTS = ("fp4_abi_version", "fp4_status_string", "fp4_quantize_workspace_size", "fp4_quantize",
            "fp4_dequantize", "fp4_preshift_workspace_size", "fp4_preshift_calibrate", "fp4_preshift_apply",
            "fp4_gemm_workspace_size", "fp4_gemm", "fp4_gemm_ex", "fp4_get_device_status",
-           "fp4_set_wait_timeout_us", "fp4_selftest_bounded_wait")
+           "fp4_set_wait_timeout_us", "fp4_selftest_bounded_wait", "fp4_preshift_calibrate_noalloc")
 
 
 class Fp4Error(RuntimeError):
@@ -67,6 +67,7 @@ def lib():
                 "fp4_get_device_status": (i, [ctypes.POINTER(ctypes.c_int32), i, P]),
                 "fp4_set_wait_timeout_us": (None, [ll]),
                 "fp4_selftest_bounded_wait": (i, [ll, P]),
+                "fp4_preshift_calibrate_noalloc": (i, [P, i, i, P, P, P]),
             }
             for name, (res, args) in sigs.items():
                 fn = getattr(L, name)

@@ -29,6 +29,9 @@ cudaError_t launch_gemm_tc(const uint16_t* X, const uint8_t* packed, const void*
                            size_t ws_bytes, int splits, int* status, unsigned long long timeout_ns,
                            cudaStream_t st);
 cudaError_t launch_bounded_wait_probe(int* status, unsigned long long timeout_ns, cudaStream_t st);
+int noalloc_max_k();
+cudaError_t launch_calibrate_noalloc(const uint16_t* X, int M, int K, int8_t* shift, float* rho, int* status,
+                                     cudaStream_t st);
 }  // namespace fp4
 
 using namespace fp4;
@@ -212,6 +215,27 @@ fp4_status fp4_preshift_calibrate(const uint16_t* X, int M, int K, int8_t* shift
     int* st = status_ptr();
     if (!st) return FP4_ERR_CUDA;
     return cuda_status(launch_calibrate(X, M, K, shift, rho, workspace, st, stream));
+}
+
+fp4_status fp4_preshift_calibrate_noalloc(const uint16_t* X, int M, int K, int8_t* shift, float* rho,
+                                          cudaStream_t stream) {
+    if (M < 0 || K < 0) return FP4_ERR_INVALID_ARG;
+    if (K % 8 != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if (K > noalloc_max_k()) return FP4_ERR_WORKSPACE;  // the built-in buffer holds K <= 65536 columns
+    if (!rho || (K > 0 && !shift)) return FP4_ERR_INVALID_ARG;
+    if (!aligned(rho, 4) || (shift && !aligned(shift, 16))) return FP4_ERR_MISALIGNED;
+    if ((long long)M * K == 0) {
+        const float one = 1.0f;
+        cudaError_t e = cudaMemcpyAsync(rho, &one, sizeof(one), cudaMemcpyHostToDevice, stream);
+        if (e == cudaSuccess && K > 0) e = cudaMemsetAsync(shift, 0, (size_t)K, stream);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+        return cuda_status(e);
+    }
+    if (!X) return FP4_ERR_INVALID_ARG;
+    if (!aligned(X, 16)) return FP4_ERR_MISALIGNED;
+    int* st = status_ptr();
+    if (!st) return FP4_ERR_CUDA;
+    return cuda_status(launch_calibrate_noalloc(X, M, K, shift, rho, st, stream));
 }
 
 fp4_status fp4_preshift_apply(const uint16_t* X, int M, int K, const int8_t* shift, const float* rho, uint16_t* Xt,

@@ -138,3 +138,58 @@ cudaError_t launch_apply(const uint16_t* X, int M, int K, const int8_t* shift, c
 }
 
 }  // namespace fp4
+
+// ------------------------------------------------- allocation-free variant
+// fp4_preshift_calibrate_noalloc: the same two kernels, with the per-slab
+// column maxima kept in a buffer that is part of the library image instead
+// of a caller-provided workspace.  Some callers have no way to obtain device
+// memory at the point where they calibrate: an inference runtime that plans
+// all of its device memory at start-up and forbids allocation afterwards, or
+// a plug-in that is handed tensors but no allocator.  They use this entry.
+//
+// The buffer holds kNoAllocFloats fp32 values (256 KB), which bounds K at
+// kNoAllocFloats (one slab of column maxima per column at least).  Every
+// GPU that loads the library holds this buffer until the process exits.
+// Calls share it: two calls whose kernels overlap on a GPU (different
+// streams without ordering between them) race on it.  Nothing in it needs
+// to start at zero: the column-maximum kernel writes every entry the
+// finalize kernel reads, and each call overwrites what the previous left.
+namespace fp4 {
+
+constexpr int kNoAllocFloats = 65536;
+static __device__ __align__(256) float g_calib_scratch[kNoAllocFloats];
+
+// Host code must not use g_calib_scratch as a device address (on the host
+// the name stands for a host-side shadow); the device address is fetched
+// once per device, with that device current, and cached.
+static float* noalloc_scratch_ptr() {
+    static float* ptrs[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!ptrs[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_calib_scratch) != cudaSuccess) return nullptr;
+        ptrs[dev] = reinterpret_cast<float*>(p);
+    }
+    return ptrs[dev];
+}
+
+int noalloc_max_k() { return kNoAllocFloats; }
+
+cudaError_t launch_calibrate_noalloc(const uint16_t* X, int M, int K, int8_t* shift, float* rho, int* status,
+                                     cudaStream_t st) {
+    float* part = noalloc_scratch_ptr();
+    if (!part) return cudaErrorInvalidDevice;
+    // fewer row slabs than the workspace variant when K is large: the
+    // column maxima are exact in any grouping, so the results are the same
+    int slabs = calib_slabs(M, K);
+    if (slabs > kNoAllocFloats / K) slabs = kNoAllocFloats / K;
+    const int rows = (M + slabs - 1) / slabs;
+    slabs = (M + rows - 1) / rows;
+    dim3 grid((K + kColsPerBlock - 1) / kColsPerBlock, slabs);
+    colmax_kernel<<<grid, 256, 0, st>>>(X, M, K, rows, part, status);
+    calib_finalize_kernel<<<1, 1024, 0, st>>>(part, slabs, K, shift, rho);
+    return cudaGetLastError();
+}
+
+}  // namespace fp4
