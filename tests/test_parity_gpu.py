@@ -231,6 +231,36 @@ def test_gemm_decode_formats(fp4, oracle_mod, fmt, sdt):
     assert gemm_case(fp4, oracle_mod, 3, 96, 256, 4, fmt=fmt, sdt=sdt, engine=fp4.ENGINE_DECODE, rho=0.75) <= TOL
 
 
+@pytest.mark.parametrize("N,K,M", [
+    (10007, 256, 3),    # more blocks than two per resident CTA; ragged last block
+    (40, 6272, 2),      # one CTA of 16 warps per SM, two buffers, odd chunk count
+    (2400, 24576, 1),   # largest K of the contiguous-block path: one buffer, two blocks per CTA
+    (5000, 11008, 8),   # activations too large to stage: read from L2 per chunk, two buffers
+    (2500, 13824, 1),   # staged activations with one buffer
+    (64, 24704, 2),     # beyond it: the per-group kernel
+])
+def test_gemm_decode_block_schedule(fp4, oracle_mod, N, K, M):
+    """Decode engine, group 128: the persistent walk over 16-row blocks in
+    each of its shared-memory configurations."""
+    assert gemm_case(fp4, oracle_mod, N + K, N, K, M, engine=fp4.ENGINE_DECODE, rho=1.5) <= TOL
+
+
+def test_gemm_decode_unaligned_scales(fp4, oracle_mod):
+    """A scale pointer that is 4- but not 16-byte aligned: the scale rows are
+    then read from global memory instead of travelling with the codes."""
+    N, K, M = 700, 1024, 5
+    W, X = synth.random_case(31, N, K, M)
+    ref_q = oracle_mod.quantize(W, 128, 1, False, None, "f16")
+    res = fp4.quantize(dev_f32(W), 128, fp4.E2M1, False, None, "f16")
+    store = torch.empty(N * (K // 128) + 8, dtype=torch.float16, device="cuda")
+    sc = store[2:2 + N * (K // 128)].view(N, K // 128)
+    sc.copy_(res["scales"])
+    assert sc.data_ptr() % 16 != 0
+    Y = fp4.gemm(dev_bf16(X), res["packed"], sc, 1, 128, engine=fp4.ENGINE_DECODE)
+    Yref = oracle_mod.gemm(X, ref_q["packed"], ref_q["scales"], 1, 128)
+    assert rel_err(Y, Yref) <= TOL
+
+
 @pytest.mark.parametrize("M", [1, 9, 16, 33, 64, 65, 128, 200, 256, 300])
 @pytest.mark.parametrize("N,K,group", [(256, 512, 128), (200, 384, 64), (130, 96, 32)])
 def test_gemm_tensor_engine(fp4, oracle_mod, M, N, K, group):

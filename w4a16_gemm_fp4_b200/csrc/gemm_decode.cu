@@ -163,30 +163,27 @@ __global__ void __launch_bounds__(256) gemm_decode_kernel(DecodeParams p) {
 // the exact code values separately (the mma sums x * v in fp32) and is then
 // scaled once by s in fp32, so no weight is rounded.
 //
-// Memory: each warp owns a ring of kStages shared-memory stages filled by
-// TMA (its elected lane issues the copies): per chunk the R x 16 x 64-byte
-// packed-code tile and the activation tile (M rows x 128 k as two 128-byte
-// swizzled boxes).  A warp keeps kStages chunks in flight without holding
-// them in registers, which is what streaming HBM needs.
+// Memory.  A block is 16 adjacent weight rows x all of K: one contiguous
+// piece of the packed matrix, whose 16 rows of group scales are contiguous
+// too.  CTAs are persistent and walk the blocks blockIdx.x + i * gridDim.x
+// through nbuf shared-memory buffers (2 where they fit): one thread issues
+// the bulk copies of the next blocks (one per row and half of K, one for
+// the scale rows) while the warps compute the current one, so every DRAM
+// request is a long contiguous run.  The code rows sit at a pitch of
+// K/2 + 16 bytes so that the 8 rows a warp reads at once fall in different
+// banks.  The activations are staged once per CTA in shared memory, already
+// in the operand form of the mma and ordered so that the four lanes sharing
+// a token read 64 contiguous bytes; where M * K is too large for that they are
+// read from L2 per chunk instead.  The warps split K into chunks and reduce
+// their fp32 sums in shared memory in warp order (deterministic).
 //
-// Dequantization (the instruction count per weight decides decode speed):
+// Dequantization:
 //  - E2M1: the hardware e2m1x2 -> f16x2 convert, one instruction per two
-//    codes; the mma runs in f16 with fp32 accumulation, so the activations
-//    are converted bf16 -> f32 -> f16 in registers (exact for |x| in the fp16
-//    normal range, shared by the R row tiles of the warp);
+//    codes; the mma runs in f16 with fp32 accumulation and the activations
+//    are converted bf16 -> f32 -> f16 (exact for |x| in the fp16 normal
+//    range);
 //  - E1M2 / E3M0: exact bf16 by bit placement (dequant8_exact) with the
 //    activation pairs rebuilt as (k, k+4) pairs by prmt.
-constexpr int kWarpsPerCta = 8;
-
-template <int R>
-struct DecodeRing {
-    static constexpr int STAGES = R == 1 ? 4 : 3;
-    static constexpr int XBYTES = 2048;          // two 1 KB swizzled activation halves
-    static constexpr int WBYTES = R * 1024;      // R x 16 rows x 64 bytes of codes
-    static constexpr int STAGE = XBYTES + WBYTES;
-    static constexpr int SMEM = kWarpsPerCta * STAGES * STAGE + 1024 + kWarpsPerCta * STAGES * 8;
-};
-
 __device__ __forceinline__ void mma_f16_16816(float d[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                               uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -216,235 +213,302 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t x) {
     return d;
 }
 
-template <int R, int MANT, int SDT>
-__global__ void __launch_bounds__(256, 2)
-    gemm_decode_g128_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
-                            DecodeParams p, int* status, unsigned long long timeout_ns) {
-    using RG = DecodeRing<R>;
+// 8 bf16 activations (k0..k7 of one 16-byte vector) -> the four B-operand
+// registers of that vector: f16 natural pairs for the E2M1 path, bf16
+// (k, k+4) pairs matching dequant8_exact for the others.
+template <bool kCvt>
+__device__ __forceinline__ uint4 x_operand(const uint4 x) {
+    if (kCvt)
+        return make_uint4(bf16x2_to_f16x2(x.x), bf16x2_to_f16x2(x.y), bf16x2_to_f16x2(x.z), bf16x2_to_f16x2(x.w));
+    return make_uint4(prmt(x.x, x.z, 0x5410u), prmt(x.x, x.z, 0x7632u), prmt(x.y, x.w, 0x5410u),
+                      prmt(x.y, x.w, 0x7632u));
+}
+
+__device__ __forceinline__ uint4 lds128(const void* p) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(smem_u32(p)));
+    return v;
+}
+
+__device__ __forceinline__ void sts128(void* p, const uint4 v) {
+    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(smem_u32(p)), "r"(v.x), "r"(v.y), "r"(v.z),
+                 "r"(v.w));
+}
+
+constexpr int kDecMaxK = 24576;  // one buffer of 16 code rows and scale rows must fit shared memory
+constexpr int kDecSmemMax = 226 * 1024;
+
+// Row pitches are 64 modulo 128 bytes: the 8 lanes of a quarter-warp read
+// 16 bytes each from two rows and hit 8 different bank groups.
+__host__ __device__ constexpr int dec_pitch(int K) { return K / 2 + (((K / 2) & 127) == 0 ? 64 : 0); }
+// codes of 16 rows at the padded pitch + their scale rows (room for fp32)
+__host__ __device__ constexpr int dec_buf_bytes(int K) { return 16 * dec_pitch(K) + 16 * (K / 128) * 4; }
+__host__ __device__ constexpr int dec_xpitch(int K) { return 2 * K + 64; }
+__host__ __device__ constexpr int dec_smem_bytes(int K, int M, int nw, int nbuf, bool xs) {
+    return nbuf * dec_buf_bytes(K) + (xs ? M * dec_xpitch(K) : 0) + 2 * nw * 32 * 4 * 4 + 128;
+}
+
+template <int MANT, int SDT, int NW, bool XS>
+__global__ void __launch_bounds__(NW * 32, 16 / NW)
+    gemm_decode_g128_kernel(DecodeParams p, int nbuf, int sc_bulk, int* status, unsigned long long timeout_ns) {
     constexpr bool kCvt = MANT == 1;  // E2M1: hardware convert + f16 mma
+    constexpr int kEs = SDT == FP4_SCALE_F16 ? 2 : 4;
     extern __shared__ uint8_t dsmem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem_raw) + 127) & ~uintptr_t(127));
+    __shared__ __align__(8) uint64_t bar[2][3];  // [buffer][codes of half 0, codes of half 1, scale rows]
+    __shared__ volatile int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
-    uint8_t* ring = smem + warp * RG::STAGES * RG::STAGE;
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kWarpsPerCta * RG::STAGES * RG::STAGE) + warp * RG::STAGES;
+    const int K = p.K, G = K >> 7;
+    const int P = dec_pitch(K), SB = dec_buf_bytes(K), XP = dec_xpitch(K);
+    uint8_t* xs = base + nbuf * SB;
+    float* red = reinterpret_cast<float*>(xs + (XS ? p.M * XP : 0));  // [2][NW][32][4]
+    const int half_bytes = K / 4;       // K % 128 == 0: a multiple of 32 bytes
+    const int sc_bytes = 16 * G * kEs;  // scale rows of a full block: a multiple of 32 bytes
+    const int nblk = (p.N + 15) / 16;
+    const int iters = blockIdx.x < nblk ? (nblk - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
 
-    const int n0 = blockIdx.x * 16 * R;
-    const int nchunks = (p.K + 127) >> 7;
-    const int c_begin = warp * nchunks / kWarpsPerCta, c_end = (warp + 1) * nchunks / kWarpsPerCta;
-    const int mrows = p.M < 8 ? p.M : 8;
-    const uint32_t tx_bytes = (uint32_t)RG::WBYTES + 2u * 128u * (uint32_t)mrows;
-
-    // activation rows >= M are never loaded: zero them once so that the
-    // unused mma columns stay finite
-    for (int i = lane; i < RG::STAGES * (RG::XBYTES / 4); i += 32) {
-        const int st = i / (RG::XBYTES / 4), rem = i % (RG::XBYTES / 4);
-        reinterpret_cast<uint32_t*>(ring + st * RG::STAGE)[rem] = 0u;
-    }
-    if (lane == 0) {
-        for (int s = 0; s < RG::STAGES; ++s) mbar_init(&full[s], 1);
+    if (threadIdx.x == 0) {
+        for (int b = 0; b < 2; ++b)
+            for (int h = 0; h < 3; ++h) mbar_init(&bar[b][h], 1);
         fence_mbar_init();
+        abort_flag = 0;
     }
-    __syncwarp();
-    fence_proxy_async_smem();
-    __syncwarp();
+    __syncthreads();
     pdl_wait();  // inputs may come from the previous kernel in the stream
     pdl_launch_dependents();
 
-    if (lane == 0) {
-        for (int c = c_begin; c < c_end && c < c_begin + RG::STAGES; ++c) {
-            const int s = c - c_begin;
-            uint8_t* st = ring + s * RG::STAGE;
-            mbar_arrive_expect_tx(&full[s], tx_bytes);
-            tma_load_2d(st, &tmX, c * 128, 0, &full[s]);
-            tma_load_2d(st + 1024, &tmX, c * 128 + 64, 0, &full[s]);
-            tma_load_2d(st + RG::XBYTES, &tmW, c * 64, n0, &full[s]);
+    int issued = 0;  // blocks whose copies were issued (thread 0 only)
+    auto issue = [&](int it) {  // bulk copies of block `it` of this CTA into buffer it % nbuf
+        const int n0 = ((int)blockIdx.x + it * (int)gridDim.x) * 16;
+        const int nrows = p.N - n0 < 16 ? p.N - n0 : 16;
+        const int b = it % nbuf;
+        uint8_t* buf = base + b * SB;
+        for (int h = 0; h < 2; ++h) {
+            mbar_arrive_expect_tx(&bar[b][h], (uint32_t)(nrows * half_bytes));
+            for (int r = 0; r < nrows; ++r)
+                bulk_load(buf + r * P + h * half_bytes, p.packed + (size_t)(n0 + r) * (K / 2) + h * half_bytes,
+                          (uint32_t)half_bytes, &bar[b][h]);
         }
-    }
-
-    // scales of rows g and g+8 of each tile (rows past N read row 0; never stored)
-    const int G = p.K >> 7;
-    int rows[2 * R];
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-        const int na = n0 + 16 * r + g, nb = na + 8;
-        rows[2 * r] = na < p.N ? na : 0;
-        rows[2 * r + 1] = nb < p.N ? nb : 0;
-    }
-    auto scale_at = [&](int row, int c) -> float {
-        if (SDT == FP4_SCALE_F16)
-            return __half2float(__ldg(reinterpret_cast<const __half*>(p.scales) + (size_t)row * G + c));
-        return __ldg(reinterpret_cast<const float*>(p.scales) + (size_t)row * G + c);
+        if (sc_bulk && nrows == 16) {
+            mbar_arrive_expect_tx(&bar[b][2], (uint32_t)sc_bytes);
+            bulk_load(buf + 16 * P, static_cast<const uint8_t*>(p.scales) + (size_t)n0 * G * kEs,
+                      (uint32_t)sc_bytes, &bar[b][2]);
+        } else {
+            mbar_arrive(&bar[b][2]);  // a ragged last block reads its scales from global memory
+        }
+        issued = it + 1;
     };
-    float sc[2 * R];
-#pragma unroll
-    for (int i = 0; i < 2 * R; ++i) sc[i] = c_begin < c_end ? scale_at(rows[i], c_begin) : 0.f;
+    if (threadIdx.x == 0)
+        for (int it = 0; it < nbuf && it < iters; ++it) issue(it);
 
-    float acc[R][4];
-#pragma unroll
-    for (int r = 0; r < R; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
-    bool ok = true;
-    for (int c = c_begin; c < c_end; ++c) {
-        const int s = (c - c_begin) % RG::STAGES;
-        const uint32_t ph = (uint32_t)((c - c_begin) / RG::STAGES) & 1u;
-        float sn[2 * R];
-#pragma unroll
-        for (int i = 0; i < 2 * R; ++i) sn[i] = c + 1 < c_end ? scale_at(rows[i], c + 1) : 0.f;
-        if (!mbar_wait(&full[s], ph, timeout_ns)) {
-            ok = false;
-            break;
+    if (XS) {  // the activations, once per CTA, in operand form at row pitch XP
+        const int vpr = K >> 3;
+        const uint4* src = reinterpret_cast<const uint4*>(p.X);
+        for (int i = threadIdx.x; i < p.M * vpr; i += NW * 32) {
+            const int m = i / vpr, v = i - m * vpr;
+            // vector 4t + q of chunk c (lane t's q-th) sits at 16 * (4q + t)
+            const int pos = (v & ~15) * 16 + 16 * (4 * (v & 3) + ((v >> 2) & 3));
+            sts128(xs + m * XP + pos, x_operand<kCvt>(__ldg(src + i)));
         }
-        const uint8_t* st = ring + s * RG::STAGE;
-        // activations of token g, k = 32t .. 32t+31: half t/2, 16-byte chunks
-        // (t&1)*4 + i stored at chunk ^ (g & 7) (128-byte swizzle)
-        const uint8_t* xrow = st + (t >> 1) * 1024 + g * 128;
-        uint32_t xb[16];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint4 x = *reinterpret_cast<const uint4*>(xrow + ((((t & 1) * 4 + i) ^ (g & 7)) << 4));
-            if (kCvt) {
-                xb[4 * i + 0] = bf16x2_to_f16x2(x.x);
-                xb[4 * i + 1] = bf16x2_to_f16x2(x.y);
-                xb[4 * i + 2] = bf16x2_to_f16x2(x.z);
-                xb[4 * i + 3] = bf16x2_to_f16x2(x.w);
-            } else {
-                xb[4 * i + 0] = prmt(x.x, x.z, 0x5410u);  // (k0, k4)
-                xb[4 * i + 1] = prmt(x.x, x.z, 0x7632u);  // (k1, k5)
-                xb[4 * i + 2] = prmt(x.y, x.w, 0x5410u);  // (k2, k6)
-                xb[4 * i + 3] = prmt(x.y, x.w, 0x7632u);  // (k3, k7)
+        __syncthreads();
+    }
+
+    const int c_begin = warp * G / NW, c_end = (warp + 1) * G / NW;
+    const int hb = (c_begin * 64) / half_bytes;
+    const int he = c_end > c_begin ? ((c_end * 64) - 1) / half_bytes : hb - 1;
+    // token g of the mma's 8 columns (columns >= M use token 0 and are never stored)
+    const int gx = g < p.M ? g : 0;
+    const uint8_t* xrow = xs + gx * XP + 16 * t;
+    const uint4* px = reinterpret_cast<const uint4*>(p.X + (size_t)gx * K) + 4 * t;
+    const float rho = p.x_scale ? *p.x_scale : 1.f;
+
+    for (int it = 0; it < iters; ++it) {
+        const int n0 = ((int)blockIdx.x + it * (int)gridDim.x) * 16;
+        const int b = it % nbuf;
+        const uint8_t* wsm = base + b * SB;
+        const uint8_t* ssm = wsm + 16 * P;
+        const uint32_t ph = (uint32_t)(it / nbuf) & 1u;
+        const bool sc_smem = sc_bulk && p.N - n0 >= 16;
+        auto scale_at = [&](int rl, int c) -> float {  // block row rl, group c
+            if (sc_smem) {
+                if (SDT == FP4_SCALE_F16)
+                    return __half2float(*reinterpret_cast<const __half*>(ssm + 2 * (rl * G + c)));
+                return *reinterpret_cast<const float*>(ssm + 4 * (rl * G + c));
             }
-        }
+            const size_t row = n0 + rl < p.N ? n0 + rl : n0;
+            if (SDT == FP4_SCALE_F16)
+                return __half2float(__ldg(reinterpret_cast<const __half*>(p.scales) + row * G + c));
+            return __ldg(reinterpret_cast<const float*>(p.scales) + row * G + c);
+        };
+        uint4 xn[4];
+        if (!XS && c_begin < c_end) {
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-            const uint8_t* wt = st + RG::XBYTES + r * 1024;
-            const uint4 wa = *reinterpret_cast<const uint4*>(wt + g * 64 + 16 * t);
-            const uint4 wb = *reinterpret_cast<const uint4*>(wt + (g + 8) * 64 + 16 * t);
+            for (int q = 0; q < 4; ++q) xn[q] = __ldg(px + c_begin * 16 + q);
+        }
+        bool ok = abort_flag == 0;
+        if (c_begin < c_end) {
+            for (int h = hb; h <= he && h < 2 && ok; ++h)
+                if (!mbar_wait(&bar[b][h], ph, timeout_ns)) ok = false;
+            if (ok && !mbar_wait(&bar[b][2], ph, timeout_ns)) ok = false;
+        }
+        if (!ok) abort_flag = 1;
+
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int c = c_begin; c < c_end && ok; ++c) {
+            uint4 xv[4];
+            if (XS) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) xv[q] = lds128(xrow + 256 * c + 64 * q);
+            } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) xv[q] = x_operand<kCvt>(xn[q]);
+                if (c + 1 < c_end) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) xn[q] = __ldg(px + (c + 1) * 16 + q);
+                }
+            }
+            const float sa = scale_at(g, c), sb = scale_at(g + 8, c);
+            // this lane's 16 bytes of rows g and g+8 for chunk c: bytes 64c + 16t
+            const uint4 wa = lds128(wsm + g * P + 64 * c + 16 * t);
+            const uint4 wb = lds128(wsm + (g + 8) * P + 64 * c + 16 * t);
             float part[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int wi = 0; wi < 4; ++wi) {
+                const uint32_t xb0 = word_of(xv[wi], 0), xb1 = word_of(xv[wi], 1);
+                const uint32_t xb2 = word_of(xv[wi], 2), xb3 = word_of(xv[wi], 3);
                 uint32_t qa[4], qb[4];
                 if (kCvt) {
                     e2m1_to_f16x8(word_of(wa, wi), qa[0], qa[1], qa[2], qa[3]);
                     e2m1_to_f16x8(word_of(wb, wi), qb[0], qb[1], qb[2], qb[3]);
-                    mma_f16_16816(part, qa[0], qb[0], qa[1], qb[1], xb[4 * wi + 0], xb[4 * wi + 1]);
-                    mma_f16_16816(part, qa[2], qb[2], qa[3], qb[3], xb[4 * wi + 2], xb[4 * wi + 3]);
+                    mma_f16_16816(part, qa[0], qb[0], qa[1], qb[1], xb0, xb1);
+                    mma_f16_16816(part, qa[2], qb[2], qa[3], qb[3], xb2, xb3);
                 } else {
                     dequant8_exact<MANT>(word_of(wa, wi), qa);
                     dequant8_exact<MANT>(word_of(wb, wi), qb);
-                    mma_bf16_16816(part, qa[0], qb[0], qa[1], qb[1], xb[4 * wi + 0], xb[4 * wi + 1]);
-                    mma_bf16_16816(part, qa[2], qb[2], qa[3], qb[3], xb[4 * wi + 2], xb[4 * wi + 3]);
+                    mma_bf16_16816(part, qa[0], qb[0], qa[1], qb[1], xb0, xb1);
+                    mma_bf16_16816(part, qa[2], qb[2], qa[3], qb[3], xb2, xb3);
                 }
             }
-            acc[r][0] = fmaf(sc[2 * r], part[0], acc[r][0]);
-            acc[r][1] = fmaf(sc[2 * r], part[1], acc[r][1]);
-            acc[r][2] = fmaf(sc[2 * r + 1], part[2], acc[r][2]);
-            acc[r][3] = fmaf(sc[2 * r + 1], part[3], acc[r][3]);
+            acc[0] = fmaf(sa, part[0], acc[0]);
+            acc[1] = fmaf(sa, part[1], acc[1]);
+            acc[2] = fmaf(sb, part[2], acc[2]);
+            acc[3] = fmaf(sb, part[3], acc[3]);
         }
-#pragma unroll
-        for (int i = 0; i < 2 * R; ++i) sc[i] = sn[i];
-        __syncwarp();  // every lane has consumed the stage
-        if (lane == 0 && c + RG::STAGES < c_end) {
-            const int cn = c + RG::STAGES;
-            uint8_t* stn = ring + s * RG::STAGE;
-            mbar_arrive_expect_tx(&full[s], tx_bytes);
-            tma_load_2d(stn, &tmX, cn * 128, 0, &full[s]);
-            tma_load_2d(stn + 1024, &tmX, cn * 128 + 64, 0, &full[s]);
-            tma_load_2d(stn + RG::XBYTES, &tmW, cn * 64, n0, &full[s]);
-        }
-    }
-    if (!ok && lane == 0) {
-        raise_status(status, kStatusTimeout);
-        // copies still in flight must land before the CTA exits
-        for (int c = c_end - RG::STAGES > c_begin ? c_end - RG::STAGES : c_begin; c < c_end; ++c) {
-            const int s = (c - c_begin) % RG::STAGES;
-            mbar_wait(&full[s], (uint32_t)((c - c_begin) / RG::STAGES) & 1u, timeout_ns);
-        }
-    }
 
-    // cross-warp reduction in warp order (reusing the ring), then the epilogue
-    __syncthreads();
-    float* red = reinterpret_cast<float*>(smem);  // [8 warps][R][32][4]
+        // cross-warp reduction in warp order (double-buffered region)
+        float* rd = red + (it & 1) * (NW * 32 * 4);
 #pragma unroll
-    for (int r = 0; r < R; ++r)
+        for (int j = 0; j < 4; ++j) rd[(warp * 32 + lane) * 4 + j] = acc[j];
+        __syncthreads();  // every warp is done with this block's buffer and partials
+        if (threadIdx.x == 0 && it + nbuf < iters && abort_flag == 0) issue(it + nbuf);
+        if (threadIdx.x < 128) {
+            const int e = threadIdx.x, l = e >> 2, j = e & 3;
+            float sum = 0.f;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) red[((warp * R + r) * 32 + lane) * 4 + j] = acc[r][j];
-    __syncthreads();
-    const float rho = p.x_scale ? *p.x_scale : 1.f;
-    for (int e = threadIdx.x; e < R * 128; e += 256) {
-        const int r = e >> 7, l = (e >> 2) & 31, j = e & 3;
-        float sum = 0.f;
-#pragma unroll
-        for (int w = 0; w < kWarpsPerCta; ++w) sum += red[((w * R + r) * 32 + l) * 4 + j];
-        const int n = n0 + 16 * r + (l >> 2) + 8 * (j >> 1);
-        const int m = 2 * (l & 3) + (j & 1);
-        if (m < p.M && n < p.N) {
-            __nv_bfloat16 y = __float2bfloat16_rn(rho * sum);
-            p.Y[(size_t)m * p.N + n] = *reinterpret_cast<uint16_t*>(&y);
+            for (int w = 0; w < NW; ++w) sum += rd[(w * 32 + l) * 4 + j];
+            const int n = n0 + (l >> 2) + 8 * (j >> 1), m = 2 * (l & 3) + (j & 1);
+            if (m < p.M && n < p.N) {
+                __nv_bfloat16 y = __float2bfloat16_rn(rho * sum);
+                p.Y[(size_t)m * p.N + n] = *reinterpret_cast<uint16_t*>(&y);
+            }
         }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && abort_flag) {
+        raise_status(status, kStatusTimeout);
+        // copies still in flight (at most the last nbuf issued blocks: none
+        // is issued after an abort) must land before the CTA exits
+        for (int it = issued - nbuf < 0 ? 0 : issued - nbuf; it < issued; ++it)
+            for (int h = 0; h < 3; ++h) mbar_wait(&bar[it % nbuf][h], (uint32_t)(it / nbuf) & 1u, timeout_ns);
     }
 }
 
-// Rows per CTA = 16 * R; two row tiles share each activation conversion,
-// one keeps enough CTAs for narrow matrices.
+// Rows per CTA of the group-32/64 kernel (16 * R).
 int decode_rows_per_cta(int N) { return N >= 8192 ? 2 : 1; }
 
-bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, int elem_bytes, const void* base, uint64_t inner,
-               uint64_t outer, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw);
+// Shared-memory plan of the group-128 kernel: two CTAs of 8 warps per SM
+// where they fit, else one CTA of 16 warps; two buffers before one; staged
+// activations before per-chunk reads from L2.
+struct DecPlan {
+    int nw, nbuf;
+    bool xs;
+    int smem;
+};
 
-template <int R, int MANT, int SDT>
-static cudaError_t launch_g128_t(const CUtensorMap& mw, const CUtensorMap& mx, const DecodeParams& p, int* status,
-                                 unsigned long long to, cudaStream_t st) {
-    static bool attr_set[64] = {};
+static DecPlan dec_plan(int M, int K) {
+    for (int xs = 1; xs >= 0; --xs)
+        for (int nbuf = 2; nbuf >= 1; --nbuf) {
+            const int s8 = dec_smem_bytes(K, M, 8, nbuf, xs);
+            if (xs && 2 * (s8 + 1024 + 128) <= 228 * 1024) return {8, nbuf, true, s8};
+            const int s16 = dec_smem_bytes(K, M, 16, nbuf, xs);
+            if (s16 <= kDecSmemMax) return {16, nbuf, xs != 0, s16};
+        }
+    return {0, 0, false, 0};
+}
+
+template <int MANT, int SDT, int NW, bool XS>
+static cudaError_t launch_g128_t(const DecodeParams& p, const DecPlan& plan, int* status, unsigned long long to,
+                                 cudaStream_t st) {
     int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_decode_g128_kernel<R, MANT, SDT>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, DecodeRing<R>::SMEM);
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 64) return cudaErrorInvalidDevice;
+    auto kern = gemm_decode_g128_kernel<MANT, SDT, NW, XS>;
+    static bool attr_set[64] = {};
+    if (!attr_set[dev]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmemMax);
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
+    int per_sm = 0, sms = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NW * 32, plan.smem);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) per_sm = 1;
+    const int nblk = (p.N + 15) / 16;
+    int grid = per_sm * sms;
+    if (grid > nblk) grid = nblk;
+    // scale rows travel with the codes when the scale pointer allows bulk copies
+    const int sc_bulk = (reinterpret_cast<uintptr_t>(p.scales) & 15) == 0 ? 1 : 0;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((p.N + 16 * R - 1) / (16 * R), 1, 1);
-    cfg.blockDim = dim3(256, 1, 1);
-    cfg.dynamicSmemBytes = DecodeRing<R>::SMEM;
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(NW * 32, 1, 1);
+    cfg.dynamicSmemBytes = (size_t)plan.smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemm_decode_g128_kernel<R, MANT, SDT>, mw, mx, p, status, to);
+    return cudaLaunchKernelEx(&cfg, kern, p, plan.nbuf, sc_bulk, status, to);
 }
 
-template <int R>
-static cudaError_t launch_g128_r(const DecodeParams& p, int fmt, int* status, unsigned long long to,
-                                 cudaStream_t st) {
-    CUtensorMap mw, mx;
-    const int mrows = p.M < 8 ? p.M : 8;
-    if (!encode_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.packed, (uint64_t)p.K / 2, (uint64_t)p.N, 64,
-                   (uint32_t)(16 * R), CU_TENSOR_MAP_SWIZZLE_NONE))
-        return cudaErrorInvalidValue;
-    if (!encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.X, (uint64_t)p.K, (uint64_t)p.M, 64, (uint32_t)mrows,
-                   CU_TENSOR_MAP_SWIZZLE_128B))
-        return cudaErrorInvalidValue;
+template <int MANT, int SDT>
+static cudaError_t launch_g128_nw(const DecodeParams& p, int* status, unsigned long long to, cudaStream_t st) {
+    const DecPlan plan = dec_plan(p.M, p.K);
+    if (plan.nw == 0) return cudaErrorInvalidValue;
+    if (plan.xs && plan.nw == 8) return launch_g128_t<MANT, SDT, 8, true>(p, plan, status, to, st);
+    if (plan.xs) return launch_g128_t<MANT, SDT, 16, true>(p, plan, status, to, st);
+    return launch_g128_t<MANT, SDT, 16, false>(p, plan, status, to, st);
+}
+
+static cudaError_t launch_g128(const DecodeParams& p, int fmt, int* status, unsigned long long to, cudaStream_t st) {
     const bool f16 = p.sdt == FP4_SCALE_F16;
     if (fmt == FP4_E1M2)
-        return f16 ? launch_g128_t<R, 2, FP4_SCALE_F16>(mw, mx, p, status, to, st)
-                   : launch_g128_t<R, 2, FP4_SCALE_F32>(mw, mx, p, status, to, st);
+        return f16 ? launch_g128_nw<2, FP4_SCALE_F16>(p, status, to, st) : launch_g128_nw<2, FP4_SCALE_F32>(p, status, to, st);
     if (fmt == FP4_E2M1)
-        return f16 ? launch_g128_t<R, 1, FP4_SCALE_F16>(mw, mx, p, status, to, st)
-                   : launch_g128_t<R, 1, FP4_SCALE_F32>(mw, mx, p, status, to, st);
-    return f16 ? launch_g128_t<R, 0, FP4_SCALE_F16>(mw, mx, p, status, to, st)
-               : launch_g128_t<R, 0, FP4_SCALE_F32>(mw, mx, p, status, to, st);
+        return f16 ? launch_g128_nw<1, FP4_SCALE_F16>(p, status, to, st) : launch_g128_nw<1, FP4_SCALE_F32>(p, status, to, st);
+    return f16 ? launch_g128_nw<0, FP4_SCALE_F16>(p, status, to, st) : launch_g128_nw<0, FP4_SCALE_F32>(p, status, to, st);
 }
 
 cudaError_t launch_gemm_decode(const uint16_t* X, const uint8_t* packed, const void* scales, int sdt,
                                const FmtTable& t, int fmt, int M, int N, int K, int group, const float* x_scale,
                                uint16_t* Y, int* status, unsigned long long timeout_ns, cudaStream_t st) {
     DecodeParams p{X, packed, scales, sdt, t, M, N, K, group, x_scale, Y};
-    if (group == 128)
-        return decode_rows_per_cta(N) == 1 ? launch_g128_r<1>(p, fmt, status, timeout_ns, st)
-                                           : launch_g128_r<2>(p, fmt, status, timeout_ns, st);
+    if (group == 128 && K <= kDecMaxK) return launch_g128(p, fmt, status, timeout_ns, st);
     const int R = decode_rows_per_cta(N);
     const int blocks = (N + 16 * R - 1) / (16 * R);
     if (R == 1)

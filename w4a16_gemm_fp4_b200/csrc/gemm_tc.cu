@@ -50,16 +50,19 @@ struct TcParams {
 
 template <int BT>
 struct TcCfg {
-    static constexpr int BW = 128;                 // weight rows per tile (MMA M)
-    static constexpr int BK = 64;                  // k per stage (one 128-byte swizzle row of bf16)
-    static constexpr int XBYTES = BT * 128;        // activation tile
-    static constexpr int WBYTES = BW * 128;        // dequantized weight tile
-    static constexpr int PBYTES = BW * 32;         // packed code tile
-    static constexpr int STAGE = XBYTES + WBYTES + PBYTES;
+    static constexpr int BW = 128;           // weight rows per tile (MMA M)
+    static constexpr int BK = 64;            // k per k-block (one 128-byte swizzle row of bf16)
+    static constexpr int KSUP = 4;           // k-blocks per packed-code stage: 128 bytes per weight row
+    static constexpr int XBYTES = BT * 128;  // activation tile of one k-block
+    static constexpr int ABYTES = BW * 128;  // dequantized weight tile of one k-block
+    static constexpr int WBYTES = BW * 128;  // packed codes of KSUP k-blocks
     // small token tiles (decode-sized problems) keep two CTAs per SM
-    static constexpr int BUDGET = BT <= 64 ? 110 * 1024 : 216 * 1024;
-    static constexpr int STAGES = BUDGET / STAGE > 8 ? 8 : BUDGET / STAGE;
-    static constexpr int CTAS_PER_SM = BT <= 64 ? 2 : 1;
+    static constexpr bool kPair = BT <= 64;
+    static constexpr int CTAS_PER_SM = kPair ? 2 : 1;
+    static constexpr int AST = kPair ? 2 : 3;                      // dequantized tiles
+    static constexpr int XST = BT == 32 ? 6 : (BT == 64 ? 3 : 6);  // activation tiles
+    static constexpr int WST = BT == 128 ? 4 : 3;                  // packed-code stages
+    static constexpr int NACC = 4;                                 // group accumulators in TMEM
     static constexpr int FCOLS = BT < 64 ? BT : 64;  // accumulator columns per fold thread
     static constexpr int FQ = BT / FCOLS;            // column blocks
     static constexpr int NF = 4 * FQ;                // fold warps
@@ -68,8 +71,11 @@ struct TcCfg {
     static constexpr int FW0 = DQ0 + DQW;            // first fold warp
     static constexpr int THREADS = (FW0 + NF) * 32;
     static_assert(BT <= 128, "fold totals of wider tiles do not fit in registers");
-    static constexpr int TMEM_COLS = 2 * BT;         // two group accumulators
-    static constexpr int SMEM = STAGES * STAGE + 1024 + 256;
+    static constexpr int TMEM_COLS = NACC * BT;
+    static constexpr int RING = AST * ABYTES + XST * XBYTES + WST * WBYTES;
+    static constexpr int NBAR = 2 * (XST + WST + AST + NACC);
+    static constexpr int SMEM = RING + 1024 + NBAR * 8 + 16;
+    static_assert(BT * 128 * 4 <= AST * ABYTES + XST * XBYTES, "split-K partials overlay the A and X rings");
 };
 
 // The k-steps (16 wide) a CTA issues run from kbeg to kstop; groups split
@@ -87,22 +93,33 @@ __device__ __forceinline__ KRange k_range(const TcParams& p, int kb0, int kb1) {
     return r;
 }
 
+__device__ __forceinline__ uint4 lds128_tc(const void* p) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(smem_u32(p)));
+    return v;
+}
+
 template <int BT>
 __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, TcParams p) {
     using C = TcCfg<BT>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* xs = smem;                                   // STAGES x XBYTES
-    uint8_t* ws = smem + C::STAGES * C::XBYTES;           // STAGES x WBYTES
-    uint8_t* ps = ws + C::STAGES * C::WBYTES;             // STAGES x PBYTES
-    uint64_t* bars = reinterpret_cast<uint64_t*>(ps + C::STAGES * C::PBYTES);
-    uint64_t* full = bars;                                // TMA landed
-    uint64_t* dq = bars + C::STAGES;                      // weight tile dequantized
-    uint64_t* empty = bars + 2 * C::STAGES;               // MMA done with the stage
-    uint64_t* gfull = bars + 3 * C::STAGES;               // [2] group accumulator complete
-    uint64_t* gempty = bars + 3 * C::STAGES + 2;          // [2] group accumulator folded
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * C::STAGES + 4);
+    uint8_t* as = smem;                         // AST x ABYTES: dequantized weight tiles
+    uint8_t* xs = as + C::AST * C::ABYTES;      // XST x XBYTES: activation tiles
+    uint8_t* wsr = xs + C::XST * C::XBYTES;     // WST x WBYTES: packed-code stages
+    uint64_t* bars = reinterpret_cast<uint64_t*>(wsr + C::WST * C::WBYTES);
+    uint64_t* xfull = bars;                 // activation tile landed
+    uint64_t* xempty = xfull + C::XST;      // MMAs done with the activation tile
+    uint64_t* wfull = xempty + C::XST;      // packed codes landed
+    uint64_t* wempty = wfull + C::WST;      // packed codes read by the dequant warps
+    uint64_t* afull = wempty + C::WST;      // weight tile dequantized
+    uint64_t* aempty = afull + C::AST;      // MMAs done with the weight tile
+    uint64_t* gfull = aempty + C::AST;      // group accumulator complete
+    uint64_t* gempty = gfull + C::NACC;     // group accumulator folded
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gempty + C::NACC);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = blockIdx.x * C::BW, m0 = blockIdx.y * BT, split = blockIdx.z;
@@ -110,16 +127,24 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
     const int kb0 = (int)((long long)split * kblocks / p.splits);
     const int kb1 = (int)((long long)(split + 1) * kblocks / p.splits);
     const int nkb = kb1 - kb0;
+    const int nsup = (nkb + C::KSUP - 1) / C::KSUP;
     const KRange kr = k_range(p, kb0, kb1);
     const uint64_t to = p.timeout_ns;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&dq[s], C::DQW * 32);
-            mbar_init(&empty[s], 1);
+        for (int s = 0; s < C::XST; ++s) {
+            mbar_init(&xfull[s], 1);
+            mbar_init(&xempty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int s = 0; s < C::WST; ++s) {
+            mbar_init(&wfull[s], 1);
+            mbar_init(&wempty[s], C::DQW * 32);
+        }
+        for (int s = 0; s < C::AST; ++s) {
+            mbar_init(&afull[s], C::DQW * 32);
+            mbar_init(&aempty[s], 1);
+        }
+        for (int b = 0; b < C::NACC; ++b) {
             mbar_init(&gfull[b], 1);
             mbar_init(&gempty[b], C::NF);
         }
@@ -139,28 +164,51 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
     pdl_launch_dependents();
 
     if (warp == 0) {
-        // ------------------------------------------------------ producer
+        // -------------------------------------------------------- producer
+        // One thread feeds both rings without blocking on either: packed
+        // codes in stages of 128 weight rows x 128 contiguous bytes (KSUP
+        // k-blocks), activations per k-block.  It gives up once neither
+        // ring has moved for the timeout.
         if (elect_one()) {
-            int issued = 0;
-            for (int i = 0; i < nkb; ++i) {
-                const int s = i % C::STAGES;
-                const uint32_t ph = (uint32_t)(i / C::STAGES) & 1u;
-                if (!mbar_wait(&empty[s], ph ^ 1u, to)) {
-                    raise_status(p.status, kStatusTimeout);
-                    break;
+            int xi = 0, wj = 0;
+            bool ok = true;
+            uint64_t t_last = globaltimer_ns();
+            while (ok && (xi < nkb || wj < nsup)) {
+                bool moved = false;
+                if (wj < nsup && mbar_test_wait(&wempty[wj % C::WST], ((uint32_t)(wj / C::WST) & 1u) ^ 1u)) {
+                    const int s = wj % C::WST;
+                    mbar_arrive_expect_tx(&wfull[s], C::WBYTES);
+                    tma_load_2d(wsr + s * C::WBYTES, &tmW, (kb0 + wj * C::KSUP) * (C::BK / 2), n0, &wfull[s]);
+                    ++wj;
+                    moved = true;
                 }
-                mbar_arrive_expect_tx(&full[s], C::XBYTES + C::PBYTES);
-                tma_load_2d(xs + s * C::XBYTES, &tmX, (kb0 + i) * C::BK, m0, &full[s]);
-                tma_load_2d(ps + s * C::PBYTES, &tmW, (kb0 + i) * (C::BK / 2), n0, &full[s]);
-                issued = i + 1;
+                if (xi < nkb && mbar_test_wait(&xempty[xi % C::XST], ((uint32_t)(xi / C::XST) & 1u) ^ 1u)) {
+                    const int s = xi % C::XST;
+                    mbar_arrive_expect_tx(&xfull[s], C::XBYTES);
+                    tma_load_2d(xs + s * C::XBYTES, &tmX, (kb0 + xi) * C::BK, m0, &xfull[s]);
+                    ++xi;
+                    moved = true;
+                }
+                if (moved) {
+                    t_last = globaltimer_ns();
+                } else if (globaltimer_ns() - t_last > to) {
+                    raise_status(p.status, kStatusTimeout);
+                    ok = false;
+                } else {
+                    __nanosleep(32);
+                }
             }
             // wait until every copy this thread issued has landed
-            for (int i = issued - C::STAGES < 0 ? 0 : issued - C::STAGES; i < issued; ++i) {
-                if (!mbar_wait(&full[i % C::STAGES], (uint32_t)(i / C::STAGES) & 1u, to)) {
+            for (int i = xi - C::XST < 0 ? 0 : xi - C::XST; i < xi; ++i)
+                if (!mbar_wait(&xfull[i % C::XST], (uint32_t)(i / C::XST) & 1u, to)) {
                     raise_status(p.status, kStatusTimeout);
                     break;
                 }
-            }
+            for (int j = wj - C::WST < 0 ? 0 : wj - C::WST; j < wj; ++j)
+                if (!mbar_wait(&wfull[j % C::WST], (uint32_t)(j / C::WST) & 1u, to)) {
+                    raise_status(p.status, kStatusTimeout);
+                    break;
+                }
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -172,16 +220,16 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
             int cur_group = -1;
             bool ok = true;
             for (int i = 0; i < nkb && ok; ++i) {
-                const int s = i % C::STAGES;
-                const uint32_t ph = (uint32_t)(i / C::STAGES) & 1u;
-                if (!mbar_wait(&dq[s], ph, to) || !mbar_wait(&full[s], ph, to)) {
+                const int a = i % C::AST, x = i % C::XST;
+                if (!mbar_wait(&afull[a], (uint32_t)(i / C::AST) & 1u, to) ||
+                    !mbar_wait(&xfull[x], (uint32_t)(i / C::XST) & 1u, to)) {
                     raise_status(p.status, kStatusTimeout);
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t wa = smem_u32(ws + s * C::WBYTES);
-                const uint32_t xa = smem_u32(xs + s * C::XBYTES);
+                const uint32_t wa = smem_u32(as + a * C::ABYTES);
+                const uint32_t xa = smem_u32(xs + x * C::XBYTES);
 #pragma unroll 1
                 for (int kk = 0; kk < C::BK / 16; ++kk) {
                     const int k = (kb0 + i) * C::BK + kk * 16;
@@ -191,25 +239,26 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
                         // new group fragment: take the next accumulator once it is folded
                         cur_group = g;
                         ++frag;
-                        const int b = frag & 1;
-                        if (!mbar_wait(&gempty[b], ((uint32_t)(frag >> 1) & 1u) ^ 1u, to)) {
+                        const int b = frag % C::NACC;
+                        if (!mbar_wait(&gempty[b], ((uint32_t)(frag / C::NACC) & 1u) ^ 1u, to)) {
                             raise_status(p.status, kStatusTimeout);
                             ok = false;
                             break;
                         }
                         tc_fence_after();
                     }
-                    const int b = frag & 1;
+                    const int b = frag % C::NACC;
                     const bool first = (k == kr.kbeg) || ((k & gmask) == 0);
                     tc_mma_f16(tmem + (uint32_t)(b * BT), sw128_desc(wa + kk * 32), sw128_desc(xa + kk * 32), idesc,
                                first ? 0u : 1u);
                     const bool last = (k + 16 >= kr.kstop) || (((k + 16) & gmask) == 0);
                     if (last) tc_commit(&gfull[b]);
                 }
-                tc_commit(&empty[s]);
+                tc_commit(&aempty[a]);
+                tc_commit(&xempty[x]);
             }
             // TMEM is freed below: the last group commit must have landed
-            if (frag >= 0 && !mbar_wait(&gfull[frag & 1], (uint32_t)(frag >> 1) & 1u, to))
+            if (frag >= 0 && !mbar_wait(&gfull[frag % C::NACC], (uint32_t)(frag / C::NACC) & 1u, to))
                 raise_status(p.status, kStatusTimeout);
         }
         __syncwarp();
@@ -217,28 +266,33 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
         // ---------------------------------------------------- dequantize
         const Bf16Lut lut = make_lut(p.t.mag, 1.f);
         const int r = (warp - C::DQ0) * 32 + lane;  // weight row within the tile
-        const int sw = (r >> 2) & 1;                // 32-byte swizzle of the packed tile
+        const int sw = r & 7;                       // 128-byte swizzle (packed stage and weight tile)
         for (int i = 0; i < nkb; ++i) {
-            const int s = i % C::STAGES;
-            const uint32_t ph = (uint32_t)(i / C::STAGES) & 1u;
-            if (!mbar_wait(&full[s], ph, to)) {
+            const int j = i / C::KSUP, sub = i % C::KSUP, ws = j % C::WST, a = i % C::AST;
+            if (sub == 0 && !mbar_wait(&wfull[ws], (uint32_t)(j / C::WST) & 1u, to)) {
                 raise_status(p.status, kStatusTimeout);
                 break;
             }
-            // 16-byte half h of row r sits at half h ^ ((r >> 2) & 1)
-            const uint8_t* prow = ps + s * C::PBYTES + r * 32;
-            const uint4 w0 = *reinterpret_cast<const uint4*>(prow + ((0 ^ sw) << 4));
-            const uint4 w1 = *reinterpret_cast<const uint4*>(prow + ((1 ^ sw) << 4));
-            uint8_t* wrow = ws + s * C::WBYTES + r * 128;
+            if (!mbar_wait(&aempty[a], ((uint32_t)(i / C::AST) & 1u) ^ 1u, to)) {
+                raise_status(p.status, kStatusTimeout);
+                break;
+            }
+            // 16-byte chunk c of row r sits at chunk c ^ (r & 7); k-block sub
+            // of the stage is chunks 2 sub and 2 sub + 1
+            const uint8_t* prow = wsr + ws * C::WBYTES + r * 128;
+            const uint4 w0 = lds128_tc(prow + (((2 * sub) ^ sw) << 4));
+            const uint4 w1 = lds128_tc(prow + (((2 * sub + 1) ^ sw) << 4));
+            if (sub == C::KSUP - 1 || i == nkb - 1) mbar_arrive(&wempty[ws]);
+            uint8_t* arow = as + a * C::ABYTES + r * 128;
             const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
                 uint32_t v[4];
                 dequant8(words[c], lut, v);
-                *reinterpret_cast<uint4*>(wrow + ((c ^ (r & 7)) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
+                *reinterpret_cast<uint4*>(arow + ((c ^ sw) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
             }
             fence_proxy_async_smem();
-            mbar_arrive(&dq[s]);
+            mbar_arrive(&afull[a]);
         }
     } else if (warp >= C::FW0) {
         // ---------------------------------------------- fold + epilogue
@@ -256,11 +310,11 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
         bool ok = true;
         float s_next = (nvalid && kr.nfrag > 0) ? load_scale(p.scales, p.sdt, (size_t)n * G + kr.gfirst) : 0.f;
         for (int f = 0; f < kr.nfrag; ++f) {
-            const int b = f & 1;
+            const int b = f % C::NACC;
             const float s = s_next;
             if (f + 1 < kr.nfrag)
                 s_next = nvalid ? load_scale(p.scales, p.sdt, (size_t)n * G + kr.gfirst + f + 1) : 0.f;
-            if (ok && !mbar_wait(&gfull[b], (uint32_t)(f >> 1) & 1u, to)) {
+            if (ok && !mbar_wait(&gfull[b], (uint32_t)(f / C::NACC) & 1u, to)) {
                 raise_status(p.status, kStatusTimeout);
                 ok = false;
             }
@@ -292,9 +346,10 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
             }
         } else {
             // split-K: publish this CTA's fp32 partial tile [BT tokens][128 rows]
-            // in shared memory (the dequant stages are idle once the last group
-            // has been folded) for the cluster reduction below
-            float* part = reinterpret_cast<float*>(ws);
+            // in shared memory over the weight and activation tiles (every
+            // MMA, and so every copy and dequantization, has completed once
+            // the last group has been folded) for the cluster reduction below
+            float* part = reinterpret_cast<float*>(smem);
 #pragma unroll
             for (int j = 0; j < C::FCOLS; ++j) part[(cb + j) * 128 + r] = tot[j];
         }
@@ -312,7 +367,7 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
             const int rank = (int)cluster_ctarank();
             const int j0 = rank * BT / p.splits, j1 = (rank + 1) * BT / p.splits;
             const float rho = p.x_scale ? *p.x_scale : 1.f;
-            const uint32_t base = smem_u32(ws);
+            const uint32_t base = smem_u32(smem);
             for (int j = j0 + h; j < j1; j += hstep) {
                 const int m = m0 + j;
                 const uint32_t off = base + (uint32_t)((j * 128 + r) * 4);
@@ -442,8 +497,8 @@ cudaError_t launch_gemm_tc(const uint16_t* X, const uint8_t* packed, const void*
     if (!encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, (uint64_t)K, (uint64_t)M, 64, (uint32_t)BT,
                    CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    if (!encode_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, packed, (uint64_t)K / 2, (uint64_t)N, 32, 128,
-                   CU_TENSOR_MAP_SWIZZLE_32B))
+    if (!encode_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, packed, (uint64_t)K / 2, (uint64_t)N, 128, 128,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     TcParams p;
     p.scales = scales;
