@@ -167,11 +167,11 @@ __global__ void __launch_bounds__(256) gemm_decode_kernel(DecodeParams p) {
 // piece of the packed matrix, whose 16 rows of group scales are contiguous
 // too.  CTAs are persistent and walk the blocks blockIdx.x + i * gridDim.x
 // through nbuf shared-memory buffers (2 where they fit): one thread issues
-// the bulk copies of the next blocks (one per row and half of K, one for
-// the scale rows) while the warps compute the current one, so every DRAM
-// request is a long contiguous run.  The code rows sit at a pitch of
-// K/2 + 16 bytes so that the 8 rows a warp reads at once fall in different
-// banks.  The activations are staged once per CTA in shared memory, already
+// the next blocks' copies while the warps compute the current one.  Each
+// block takes exactly two bulk copies (its codes and its scale rows): a
+// bulk copy costs the issuing thread on the order of a hundred cycles, so
+// per-row copies would make issue, not HBM, the limit.  Every DRAM request
+// is one long contiguous run.  The activations are staged once per CTA in shared memory, already
 // in the operand form of the mma and ordered so that the four lanes sharing
 // a token read 64 contiguous bytes; where M * K is too large for that they are
 // read from L2 per chunk instead.  The warps split K into chunks and reduce
@@ -240,9 +240,10 @@ __device__ __forceinline__ void sts128(void* p, const uint4 v) {
 constexpr int kDecMaxK = 24576;  // one buffer of 16 code rows and scale rows must fit shared memory
 constexpr int kDecSmemMax = 226 * 1024;
 
-// Row pitches are 64 modulo 128 bytes: the 8 lanes of a quarter-warp read
-// 16 bytes each from two rows and hit 8 different bank groups.
-__host__ __device__ constexpr int dec_pitch(int K) { return K / 2 + (((K / 2) & 127) == 0 ? 64 : 0); }
+// Code rows are dense (one bulk copy per block); activation rows sit at a
+// pitch of 64 modulo 128 bytes so that the 8 lanes of a quarter-warp hit 8
+// different bank groups.
+__host__ __device__ constexpr int dec_pitch(int K) { return K / 2; }
 // codes of 16 rows at the padded pitch + their scale rows (room for fp32)
 __host__ __device__ constexpr int dec_buf_bytes(int K) { return 16 * dec_pitch(K) + 16 * (K / 128) * 4; }
 __host__ __device__ constexpr int dec_xpitch(int K) { return 2 * K + 64; }
@@ -257,7 +258,7 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
     constexpr int kEs = SDT == FP4_SCALE_F16 ? 2 : 4;
     extern __shared__ uint8_t dsmem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem_raw) + 127) & ~uintptr_t(127));
-    __shared__ __align__(8) uint64_t bar[2][3];  // [buffer][codes of half 0, codes of half 1, scale rows]
+    __shared__ __align__(8) uint64_t bar[2];  // per buffer: codes and scale rows landed
     __shared__ volatile int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
@@ -265,14 +266,12 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
     const int P = dec_pitch(K), SB = dec_buf_bytes(K), XP = dec_xpitch(K);
     uint8_t* xs = base + nbuf * SB;
     float* red = reinterpret_cast<float*>(xs + (XS ? p.M * XP : 0));  // [2][NW][32][4]
-    const int half_bytes = K / 4;       // K % 128 == 0: a multiple of 32 bytes
     const int sc_bytes = 16 * G * kEs;  // scale rows of a full block: a multiple of 32 bytes
     const int nblk = (p.N + 15) / 16;
     const int iters = blockIdx.x < nblk ? (nblk - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
 
     if (threadIdx.x == 0) {
-        for (int b = 0; b < 2; ++b)
-            for (int h = 0; h < 3; ++h) mbar_init(&bar[b][h], 1);
+        for (int b = 0; b < 2; ++b) mbar_init(&bar[b], 1);
         fence_mbar_init();
         abort_flag = 0;
     }
@@ -286,39 +285,45 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
         const int nrows = p.N - n0 < 16 ? p.N - n0 : 16;
         const int b = it % nbuf;
         uint8_t* buf = base + b * SB;
-        for (int h = 0; h < 2; ++h) {
-            mbar_arrive_expect_tx(&bar[b][h], (uint32_t)(nrows * half_bytes));
-            for (int r = 0; r < nrows; ++r)
-                bulk_load(buf + r * P + h * half_bytes, p.packed + (size_t)(n0 + r) * (K / 2) + h * half_bytes,
-                          (uint32_t)half_bytes, &bar[b][h]);
-        }
-        if (sc_bulk && nrows == 16) {
-            mbar_arrive_expect_tx(&bar[b][2], (uint32_t)sc_bytes);
+        // a ragged last block, or an unaligned scale pointer, reads its scales from global memory
+        const bool sc = sc_bulk && nrows == 16;
+        const uint32_t code_bytes = (uint32_t)nrows * (uint32_t)(K / 2);
+        mbar_arrive_expect_tx(&bar[b], code_bytes + (sc ? (uint32_t)sc_bytes : 0u));
+        bulk_load(buf, p.packed + (size_t)n0 * (K / 2), code_bytes, &bar[b]);
+        if (sc)
             bulk_load(buf + 16 * P, static_cast<const uint8_t*>(p.scales) + (size_t)n0 * G * kEs,
-                      (uint32_t)sc_bytes, &bar[b][2]);
-        } else {
-            mbar_arrive(&bar[b][2]);  // a ragged last block reads its scales from global memory
-        }
+                      (uint32_t)sc_bytes, &bar[b]);
         issued = it + 1;
     };
     if (threadIdx.x == 0)
         for (int it = 0; it < nbuf && it < iters; ++it) issue(it);
 
     if (XS) {  // the activations, once per CTA, in operand form at row pitch XP
-        const int vpr = K >> 3;
+        const int vpr = K >> 3, total = p.M * vpr;
         const uint4* src = reinterpret_cast<const uint4*>(p.X);
-        for (int i = threadIdx.x; i < p.M * vpr; i += NW * 32) {
-            const int m = i / vpr, v = i - m * vpr;
-            // vector 4t + q of chunk c (lane t's q-th) sits at 16 * (4q + t)
-            const int pos = (v & ~15) * 16 + 16 * (4 * (v & 3) + ((v >> 2) & 3));
-            sts128(xs + m * XP + pos, x_operand<kCvt>(__ldg(src + i)));
+        constexpr int kB = 8;  // loads in flight per thread
+        for (int i0 = threadIdx.x; i0 < total; i0 += kB * NW * 32) {
+            uint4 v[kB];
+#pragma unroll
+            for (int u = 0; u < kB; ++u) {
+                const int i = i0 + u * NW * 32;
+                if (i < total) v[u] = __ldg(src + i);
+            }
+#pragma unroll
+            for (int u = 0; u < kB; ++u) {
+                const int i = i0 + u * NW * 32;
+                if (i < total) {
+                    const int m = i / vpr, w = i - m * vpr;
+                    // vector 4t + q of chunk c (lane t's q-th) sits at 16 * (4q + t)
+                    const int pos = (w & ~15) * 16 + 16 * (4 * (w & 3) + ((w >> 2) & 3));
+                    sts128(xs + m * XP + pos, x_operand<kCvt>(v[u]));
+                }
+            }
         }
         __syncthreads();
     }
 
     const int c_begin = warp * G / NW, c_end = (warp + 1) * G / NW;
-    const int hb = (c_begin * 64) / half_bytes;
-    const int he = c_end > c_begin ? ((c_end * 64) - 1) / half_bytes : hb - 1;
     // token g of the mma's 8 columns (columns >= M use token 0 and are never stored)
     const int gx = g < p.M ? g : 0;
     const uint8_t* xrow = xs + gx * XP + 16 * t;
@@ -349,11 +354,7 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
             for (int q = 0; q < 4; ++q) xn[q] = __ldg(px + c_begin * 16 + q);
         }
         bool ok = abort_flag == 0;
-        if (c_begin < c_end) {
-            for (int h = hb; h <= he && h < 2 && ok; ++h)
-                if (!mbar_wait(&bar[b][h], ph, timeout_ns)) ok = false;
-            if (ok && !mbar_wait(&bar[b][2], ph, timeout_ns)) ok = false;
-        }
+        if (ok && c_begin < c_end && !mbar_wait(&bar[b], ph, timeout_ns)) ok = false;
         if (!ok) abort_flag = 1;
 
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -422,7 +423,7 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
         // copies still in flight (at most the last nbuf issued blocks: none
         // is issued after an abort) must land before the CTA exits
         for (int it = issued - nbuf < 0 ? 0 : issued - nbuf; it < issued; ++it)
-            for (int h = 0; h < 3; ++h) mbar_wait(&bar[it % nbuf][h], (uint32_t)(it / nbuf) & 1u, timeout_ns);
+            mbar_wait(&bar[it % nbuf], (uint32_t)(it / nbuf) & 1u, timeout_ns);
     }
 }
 
