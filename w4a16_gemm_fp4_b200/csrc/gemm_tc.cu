@@ -66,7 +66,7 @@ struct TcCfg {
     static constexpr int FCOLS = BT < 64 ? BT : 64;  // accumulator columns per fold thread
     static constexpr int FQ = BT / FCOLS;            // column blocks
     static constexpr int NF = 4 * FQ;                // fold warps
-    static constexpr int DQW = 4;                    // dequant warps (one weight row per thread)
+    static constexpr int DQW = kPair ? 4 : 8;        // dequant warps (one or two threads per weight row)
     static constexpr int DQ0 = 2;                    // first dequant warp
     static constexpr int FW0 = DQ0 + DQW;            // first fold warp
     static constexpr int THREADS = (FW0 + NF) * 32;
@@ -213,59 +213,79 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
         __syncwarp();
     } else if (warp == 1) {
         // ----------------------------------------------------- MMA issuer
+        // One thread issues every MMA, so its own instruction stream is the
+        // limit: stage descriptors are built once and advanced by adding
+        // the 16-byte-unit offset of each K = 16 step, ring slots and
+        // phases are counters, and group bookkeeping runs only at group
+        // boundaries.
         if (elect_one()) {
             const uint32_t idesc = idesc_bf16_f32(C::BW, BT);
-            const int gshift = __ffs(p.group) - 1, gmask = p.group - 1;  // group is a power of two
-            int frag = -1;      // group fragment currently accumulating
-            int cur_group = -1;
+            const uint64_t adesc0 = sw128_desc(smem_u32(as)), xdesc0 = sw128_desc(smem_u32(xs));
+            constexpr uint32_t kAStep = C::ABYTES >> 4, kXStep = C::XBYTES >> 4;
+            static_assert((C::NACC & (C::NACC - 1)) == 0, "accumulator count is a power of two");
+            constexpr int kNaccShift = C::NACC == 4 ? 2 : (C::NACC == 2 ? 1 : 0);
+            const int gmask = p.group - 1;  // group is a power of two
+            int a = 0, x = 0;
+            uint32_t aph = 0, xph = 0;
+            int frag = -1, b = 0;
+            int k = kr.kbeg;
             bool ok = true;
             for (int i = 0; i < nkb && ok; ++i) {
-                const int a = i % C::AST, x = i % C::XST;
-                if (!mbar_wait(&afull[a], (uint32_t)(i / C::AST) & 1u, to) ||
-                    !mbar_wait(&xfull[x], (uint32_t)(i / C::XST) & 1u, to)) {
+                if (!mbar_wait(&afull[a], aph, to) || !mbar_wait(&xfull[x], xph, to)) {
                     raise_status(p.status, kStatusTimeout);
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t wa = smem_u32(as + a * C::ABYTES);
-                const uint32_t xa = smem_u32(xs + x * C::XBYTES);
-#pragma unroll 1
+                const uint64_t ad = adesc0 + (uint64_t)(a * kAStep);
+                const uint64_t xd = xdesc0 + (uint64_t)(x * kXStep);
+#pragma unroll
                 for (int kk = 0; kk < C::BK / 16; ++kk) {
-                    const int k = (kb0 + i) * C::BK + kk * 16;
-                    if (k >= kr.kstop) break;
-                    const int g = k >> gshift;
-                    if (g != cur_group) {
-                        // new group fragment: take the next accumulator once it is folded
-                        cur_group = g;
-                        ++frag;
-                        const int b = frag % C::NACC;
-                        if (!mbar_wait(&gempty[b], ((uint32_t)(frag / C::NACC) & 1u) ^ 1u, to)) {
-                            raise_status(p.status, kStatusTimeout);
-                            ok = false;
-                            break;
+                    if (k < kr.kstop) {
+                        const bool first = (k == kr.kbeg) || ((k & gmask) == 0);
+                        if (first) {
+                            // new group fragment: take the next accumulator once it is folded
+                            ++frag;
+                            b = frag & (C::NACC - 1);
+                            if (!mbar_wait(&gempty[b], ((uint32_t)(frag >> kNaccShift) & 1u) ^ 1u, to)) {
+                                raise_status(p.status, kStatusTimeout);
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
                         }
-                        tc_fence_after();
+                        tc_mma_f16(tmem + (uint32_t)(b * BT), ad + (uint64_t)(2 * kk), xd + (uint64_t)(2 * kk), idesc,
+                                   first ? 0u : 1u);
+                        if ((k + 16 >= kr.kstop) || (((k + 16) & gmask) == 0)) tc_commit(&gfull[b]);
+                        k += 16;
                     }
-                    const int b = frag % C::NACC;
-                    const bool first = (k == kr.kbeg) || ((k & gmask) == 0);
-                    tc_mma_f16(tmem + (uint32_t)(b * BT), sw128_desc(wa + kk * 32), sw128_desc(xa + kk * 32), idesc,
-                               first ? 0u : 1u);
-                    const bool last = (k + 16 >= kr.kstop) || (((k + 16) & gmask) == 0);
-                    if (last) tc_commit(&gfull[b]);
                 }
                 tc_commit(&aempty[a]);
                 tc_commit(&xempty[x]);
+                if (++a == C::AST) {
+                    a = 0;
+                    aph ^= 1u;
+                }
+                if (++x == C::XST) {
+                    x = 0;
+                    xph ^= 1u;
+                }
             }
             // TMEM is freed below: the last group commit must have landed
-            if (frag >= 0 && !mbar_wait(&gfull[frag % C::NACC], (uint32_t)(frag / C::NACC) & 1u, to))
+            if (frag >= 0 && !mbar_wait(&gfull[frag & (C::NACC - 1)], (uint32_t)(frag >> kNaccShift) & 1u, to))
                 raise_status(p.status, kStatusTimeout);
         }
         __syncwarp();
     } else if (warp >= C::DQ0 && warp < C::FW0) {
         // ---------------------------------------------------- dequantize
+        // DQW = 4: one thread per weight row (8 words of codes per k-block);
+        // DQW = 8: two threads per row, each one 16-byte half (4 words).
+        constexpr int kHalves = C::DQW / 4;
+        constexpr int kWords = 8 / kHalves;
         const Bf16Lut lut = make_lut(p.t.mag, 1.f);
-        const int r = (warp - C::DQ0) * 32 + lane;  // weight row within the tile
+        const int tid = (warp - C::DQ0) * 32 + lane;
+        const int r = tid & 127;                    // weight row within the tile
+        const int hh = tid >> 7;                    // half of the row (DQW = 8)
         const int sw = r & 7;                       // 128-byte swizzle (packed stage and weight tile)
         for (int i = 0; i < nkb; ++i) {
             const int j = i / C::KSUP, sub = i % C::KSUP, ws = j % C::WST, a = i % C::AST;
@@ -280,16 +300,25 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
             // 16-byte chunk c of row r sits at chunk c ^ (r & 7); k-block sub
             // of the stage is chunks 2 sub and 2 sub + 1
             const uint8_t* prow = wsr + ws * C::WBYTES + r * 128;
-            const uint4 w0 = lds128_tc(prow + (((2 * sub) ^ sw) << 4));
-            const uint4 w1 = lds128_tc(prow + (((2 * sub + 1) ^ sw) << 4));
+            uint32_t words[kWords];
+            if (kHalves == 1) {
+                const uint4 w0 = lds128_tc(prow + (((2 * sub) ^ sw) << 4));
+                const uint4 w1 = lds128_tc(prow + (((2 * sub + 1) ^ sw) << 4));
+                words[0] = w0.x; words[1] = w0.y; words[2] = w0.z; words[3] = w0.w;
+                words[kWords > 4 ? 4 : 0] = w1.x; words[kWords > 5 ? 5 : 0] = w1.y;
+                words[kWords > 6 ? 6 : 0] = w1.z; words[kWords > 7 ? 7 : 0] = w1.w;
+            } else {
+                const uint4 w0 = lds128_tc(prow + (((2 * sub + hh) ^ sw) << 4));
+                words[0] = w0.x; words[1] = w0.y; words[2] = w0.z; words[3] = w0.w;
+            }
             if (sub == C::KSUP - 1 || i == nkb - 1) mbar_arrive(&wempty[ws]);
             uint8_t* arow = as + a * C::ABYTES + r * 128;
-            const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+            const int c0 = hh * kWords;  // first 16-byte unit (8 k) of this thread
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
+            for (int c = 0; c < kWords; ++c) {
                 uint32_t v[4];
                 dequant8(words[c], lut, v);
-                *reinterpret_cast<uint4*>(arow + ((c ^ sw) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
+                *reinterpret_cast<uint4*>(arow + (((c0 + c) ^ sw) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
             }
             fence_proxy_async_smem();
             mbar_arrive(&afull[a]);
