@@ -74,6 +74,7 @@ typedef enum fp4_engine { FP4_ENGINE_AUTO = 0, FP4_ENGINE_DECODE = 1, FP4_ENGINE
 #define FP4_DEV_NONFINITE_INPUT 0x1 /* NaN/Inf met in W or X                   */
 #define FP4_DEV_SCALE_OVERFLOW 0x2  /* a group scale does not fit in fp16       */
 #define FP4_DEV_WAIT_TIMEOUT 0x4    /* a pipeline wait gave up; output invalid  */
+#define FP4_DEV_LAYOUT 0x8          /* a kernel's shared-memory base lacked the alignment its layout needs; nothing written */
 
 /* Version of this interface (major * 100 + minor). */
 FP4_API int fp4_abi_version(void);
@@ -183,13 +184,15 @@ FP4_API fp4_status fp4_preshift_calibrate_noalloc(const uint16_t *X, int M, int 
  *   workspace reserved: fp4_gemm_workspace_size() is 0 for every shape (the
  *            split-K reduction of skinny problems runs between the CTAs of a
  *            thread-block cluster in distributed shared memory); pass NULL, 0.
- * Engines: M <= 8 uses the decode engine (per-warp TMA rings of packed
- * codes, dequantization in registers, warp-level MMAs); larger M uses the
- * tensor engine (TMA-staged tiles, tcgen05 MMAs into tensor memory).  Both
- * multiply the exact code values and apply each group scale in fp32.
+ * Engines: M <= 8 uses the decode engine (persistent CTAs stream 16-row
+ * blocks of packed codes by bulk copy, dequantize in registers, warp-level
+ * MMAs); larger M uses the tensor engine (TMA-staged tiles dequantized in
+ * shared memory, tcgen05 MMAs into tensor memory; at group 128 and M <= 64
+ * one 128-k group per pipeline stage).  Both multiply the exact code values
+ * and apply each group scale in fp32.
  * The decode engine's E2M1 path runs its MMAs in f16: activations must lie
  * within the fp16 range (|x| < 65504); smaller than 2^-14 they lose bits.
- * Device status: FP4_DEV_WAIT_TIMEOUT.
+ * Device status: FP4_DEV_WAIT_TIMEOUT, FP4_DEV_LAYOUT.
  * ---------------------------------------------------------------------- */
 FP4_API size_t fp4_gemm_workspace_size(int M, int N, int K);
 FP4_API fp4_status fp4_gemm(const uint16_t *X, const uint8_t *packed, const void *scales,

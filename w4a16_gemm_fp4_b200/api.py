@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(HERE, "libfp4w4a16.so")
 E1M2, E2M1, E3M0, AUTO = 0, 1, 2, -1
 SCALE_F32, SCALE_F16 = 0, 1
 ENGINE_AUTO, ENGINE_DECODE, ENGINE_TENSOR = 0, 1, 2
-DEV_NONFINITE_INPUT, DEV_SCALE_OVERFLOW, DEV_WAIT_TIMEOUT = 1, 2, 4
+DEV_NONFINITE_INPUT, DEV_SCALE_OVERFLOW, DEV_WAIT_TIMEOUT, DEV_LAYOUT = 1, 2, 4, 8
 
 STATUS = {0: "FP4_OK", 1: "FP4_ERR_INVALID_ARG", 2: "FP4_ERR_UNSUPPORTED_SHAPE", 3: "FP4_ERR_MISALIGNED",
           4: "FP4_ERR_WORKSPACE", 5: "FP4_ERR_CUDA", 6: "FP4_ERR_DEVICE_STATUS"}

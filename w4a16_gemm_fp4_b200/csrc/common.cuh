@@ -33,6 +33,7 @@ struct FmtTables {
 constexpr int kStatusNonfinite = FP4_DEV_NONFINITE_INPUT;
 constexpr int kStatusScaleOverflow = FP4_DEV_SCALE_OVERFLOW;
 constexpr int kStatusTimeout = FP4_DEV_WAIT_TIMEOUT;
+constexpr int kStatusLayout = FP4_DEV_LAYOUT;
 
 __device__ __forceinline__ void raise_status(int* status, int bits) {
     if (status) atomicOr(status, bits);

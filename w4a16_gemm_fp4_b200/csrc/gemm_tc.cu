@@ -101,11 +101,42 @@ __device__ __forceinline__ uint4 lds128_tc(const void* p) {
     return v;
 }
 
+// Split-K epilogue: the splits of one output tile form a thread-block
+// cluster along z, and each CTA has published its fp32 partial tile
+// [BT tokens][128 rows] at the start of its shared memory.  Every CTA sums,
+// in rank order, one slice of tokens over the partial tiles of all CTAs of
+// the cluster (distributed shared memory) and stores it.  All threads take
+// part, and each issues its loads from every rank before the first add.
+template <int BT>
+__device__ __forceinline__ void cluster_reduce_store(const TcParams& p, uint32_t part, int n0, int m0) {
+    cluster_sync();
+    const int rank = (int)cluster_ctarank();
+    const int j0 = rank * BT / p.splits, j1 = (rank + 1) * BT / p.splits;
+    const int cnt = (j1 - j0) * 128;
+    const float rho = p.x_scale ? *p.x_scale : 1.f;
+    for (int e = threadIdx.x; e < cnt; e += blockDim.x) {
+        const int j = j0 + (e >> 7), r = e & 127;
+        const uint32_t off = part + (uint32_t)((j * 128 + r) * 4);
+        float v[8];
+#pragma unroll
+        for (int z = 0; z < 8; ++z) v[z] = z < p.splits ? ld_dsmem_f32(map_dsmem(off, (uint32_t)z)) : 0.f;
+        float a = 0.f;
+#pragma unroll
+        for (int z = 0; z < 8; ++z) a += v[z];
+        const int m = m0 + j, n = n0 + r;
+        if (m < p.M && n < p.N) {
+            __nv_bfloat16 y = __float2bfloat16_rn(rho * a);
+            p.Y[(size_t)m * p.N + n] = *reinterpret_cast<uint16_t*>(&y);
+        }
+    }
+    cluster_sync();  // no CTA leaves while its partials are being read
+}
+
 template <int BT>
 __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, TcParams p) {
     using C = TcCfg<BT>;
-    extern __shared__ uint8_t smem_raw[];
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* as = smem;                         // AST x ABYTES: dequantized weight tiles
     uint8_t* xs = as + C::AST * C::ABYTES;      // XST x XBYTES: activation tiles
@@ -311,7 +342,6 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
                 const uint4 w0 = lds128_tc(prow + (((2 * sub + hh) ^ sw) << 4));
                 words[0] = w0.x; words[1] = w0.y; words[2] = w0.z; words[3] = w0.w;
             }
-            if (sub == C::KSUP - 1 || i == nkb - 1) mbar_arrive(&wempty[ws]);
             uint8_t* arow = as + a * C::ABYTES + r * 128;
             const int c0 = hh * kWords;  // first 16-byte unit (8 k) of this thread
 #pragma unroll
@@ -321,6 +351,9 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
                 *reinterpret_cast<uint4*>(arow + (((c0 + c) ^ sw) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
             }
             fence_proxy_async_smem();
+            // release the packed-code stage only after its words are consumed
+            // (see the group-128 variant below)
+            if (sub == C::KSUP - 1 || i == nkb - 1) mbar_arrive(&wempty[ws]);
             mbar_arrive(&afull[a]);
         }
     } else if (warp >= C::FW0) {
@@ -384,36 +417,293 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
         }
     }
 
-    if (p.splits > 1) {
-        // The splits of one output tile form a thread-block cluster along z.
-        // Every CTA sums, in rank order, one slice of tokens over the partial
-        // tiles of all CTAs of the cluster (distributed shared memory).
-        cluster_sync();
-        if (warp >= C::FW0) {
-            const int f = threadIdx.x - C::FW0 * 32;
-            const int r = f & 127, h = f >> 7, hstep = (C::NF * 32) >> 7;
-            const int n = n0 + r;
-            const int rank = (int)cluster_ctarank();
-            const int j0 = rank * BT / p.splits, j1 = (rank + 1) * BT / p.splits;
-            const float rho = p.x_scale ? *p.x_scale : 1.f;
-            const uint32_t base = smem_u32(smem);
-            for (int j = j0 + h; j < j1; j += hstep) {
-                const int m = m0 + j;
-                const uint32_t off = base + (uint32_t)((j * 128 + r) * 4);
-                float v[8];
-#pragma unroll
-                for (int z = 0; z < 8; ++z) v[z] = z < p.splits ? ld_dsmem_f32(map_dsmem(off, (uint32_t)z)) : 0.f;
-                float a = 0.f;
-#pragma unroll
-                for (int z = 0; z < 8; ++z) a += v[z];
-                if (m < p.M && n < p.N) {
-                    __nv_bfloat16 y = __float2bfloat16_rn(rho * a);
-                    p.Y[(size_t)m * p.N + n] = *reinterpret_cast<uint16_t*>(&y);
+    if (p.splits > 1) cluster_reduce_store<BT>(p, smem_u32(smem), n0, m0);
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+// ---------------------------------------------------------------------------
+// Group-128 variant for small token tiles (M <= 64, BT in {16, 32, 64}).
+// A k-block is one group (128 k): the MMA thread issues its 8 K=16 steps
+// into the stage's own TMEM accumulator and commits ONCE.  That commit both
+// frees the stage (dequantized codes, activations) for reuse and hands the
+// accumulator to the fold warps.  A commit costs the issuing thread about
+// one tensor-pipe round trip, and at these N an MMA issues in ~50 cycles;
+// with 64-k stages and separate commits for stage release and group
+// completion the commits, not the MMAs, set the pace.
+//
+// Stage s and accumulator s are the same index (STG == NACC): the next use
+// of a stage needs its accumulator folded first, so a stage barrier can
+// never run two phases ahead of the fold warps that wait on it.
+template <int BT>
+struct TgCfg {
+    static constexpr int BW = 128;              // weight rows per tile (MMA M)
+    static constexpr int KB = 128;              // k per stage = one group
+    static constexpr int XBOX = BT * 128;       // activation box: 64 k x BT rows, 128-byte swizzle
+    static constexpr int XBYTES = 2 * XBOX;     // activations of one stage (128 k)
+    static constexpr int ABYTES = 2 * 16384;    // dequantized codes: two 128-row x 64-k SW128 atoms
+    static constexpr int WBYTES = BW * 64;      // packed codes of one stage: 128 rows x 64 B, 64-byte swizzle
+    static constexpr int STG = 2;               // stages == TMEM accumulators
+    static constexpr int WST = 2;               // packed-code stages
+    static constexpr int FCOLS = BT;            // accumulator columns per fold thread
+    static constexpr int NF = 4;                // fold warps (one TMEM lane quadrant each)
+    static constexpr int DQW = 4;               // dequant warps (one weight row per thread)
+    static constexpr int DQ0 = 2;
+    static constexpr int FW0 = DQ0 + DQW;
+    static constexpr int THREADS = (FW0 + NF) * 32;
+    static constexpr int TMEM_COLS = STG * BT < 32 ? 32 : STG * BT;
+    static constexpr int RING = STG * (ABYTES + XBYTES) + WST * WBYTES;
+    static constexpr int NBAR = 4 * STG + 2 * WST;
+    // the 64-token layout only fits two CTAs per SM without alignment slack:
+    // it relies on the 1024-byte-aligned dynamic shared-memory base (checked)
+    static constexpr int SLACK = BT == 64 ? 0 : 1024;
+    static constexpr int SMEM = RING + SLACK + NBAR * 8 + 16;
+    static_assert(SMEM + 1024 <= 228 * 1024 / 2, "two CTAs per SM");
+    static_assert(BT * 128 * 4 <= STG * ABYTES, "split-K partials overlay the dequantized tiles");
+};
+
+template <int BT>
+__global__ void __launch_bounds__(TgCfg<BT>::THREADS, 2)
+    gemm_tcg_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, TcParams p) {
+    using C = TgCfg<BT>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    if (C::SLACK == 0 && smem != smem_raw) {
+        if (threadIdx.x == 0) raise_status(p.status, kStatusLayout);
+        return;  // before any barrier, copy or TMEM allocation
+    }
+    uint8_t* as = smem;                         // STG x ABYTES: dequantized codes
+    uint8_t* xs = as + C::STG * C::ABYTES;      // STG x XBYTES: activations
+    uint8_t* wsr = xs + C::STG * C::XBYTES;     // WST x WBYTES: packed codes
+    uint64_t* bars = reinterpret_cast<uint64_t*>(wsr + C::WST * C::WBYTES);
+    uint64_t* xfull = bars;                 // activations landed
+    uint64_t* afull = xfull + C::STG;       // codes dequantized
+    uint64_t* kdone = afull + C::STG;       // the stage's MMAs completed (stage free, accumulator ready)
+    uint64_t* wfull = kdone + C::STG;       // packed codes landed
+    uint64_t* wempty = wfull + C::WST;      // packed codes read
+    uint64_t* gempty = wempty + C::WST;     // accumulator folded (kdone's one arrival is the commit)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gempty + C::STG);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * C::BW, m0 = blockIdx.y * BT, split = blockIdx.z;
+    const int kblocks = p.K / C::KB;
+    const int kb0 = (int)((long long)split * kblocks / p.splits);
+    const int kb1 = (int)((long long)(split + 1) * kblocks / p.splits);
+    const int nkb = kb1 - kb0;
+    const uint64_t to = p.timeout_ns;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STG; ++s) {
+            mbar_init(&xfull[s], 1);
+            mbar_init(&afull[s], C::DQW * 32);
+            mbar_init(&kdone[s], 1);
+            mbar_init(&gempty[s], C::NF);
+        }
+        for (int s = 0; s < C::WST; ++s) {
+            mbar_init(&wfull[s], 1);
+            mbar_init(&wempty[s], C::DQW * 32);
+        }
+        fence_mbar_init();
+        prefetch_tmap(&tmX);
+        prefetch_tmap(&tmW);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    pdl_wait();  // inputs may come from the previous kernel in the stream
+    pdl_launch_dependents();
+
+    if (warp == 0) {
+        // -------------------------------------------------------- producer
+        if (elect_one()) {
+            int xi = 0, wj = 0;
+            bool ok = true;
+            uint64_t t_last = globaltimer_ns();
+            while (ok && (xi < nkb || wj < nkb)) {
+                bool moved = false;
+                if (wj < nkb && mbar_test_wait(&wempty[wj % C::WST], ((uint32_t)(wj / C::WST) & 1u) ^ 1u)) {
+                    const int s = wj % C::WST;
+                    mbar_arrive_expect_tx(&wfull[s], C::WBYTES);
+                    tma_load_2d(wsr + s * C::WBYTES, &tmW, (kb0 + wj) * (C::KB / 2), n0, &wfull[s]);
+                    ++wj;
+                    moved = true;
+                }
+                if (xi < nkb && mbar_test_wait(&kdone[xi % C::STG], ((uint32_t)(xi / C::STG) & 1u) ^ 1u)) {
+                    const int s = xi % C::STG;
+                    mbar_arrive_expect_tx(&xfull[s], C::XBYTES);
+                    tma_load_2d(xs + s * C::XBYTES, &tmX, (kb0 + xi) * C::KB, m0, &xfull[s]);
+                    tma_load_2d(xs + s * C::XBYTES + C::XBOX, &tmX, (kb0 + xi) * C::KB + 64, m0, &xfull[s]);
+                    ++xi;
+                    moved = true;
+                }
+                if (moved) {
+                    t_last = globaltimer_ns();
+                } else if (globaltimer_ns() - t_last > to) {
+                    raise_status(p.status, kStatusTimeout);
+                    ok = false;
+                } else {
+                    __nanosleep(32);
                 }
             }
+            for (int i = xi - C::STG < 0 ? 0 : xi - C::STG; i < xi; ++i)
+                if (!mbar_wait(&xfull[i % C::STG], (uint32_t)(i / C::STG) & 1u, to)) {
+                    raise_status(p.status, kStatusTimeout);
+                    break;
+                }
+            for (int j = wj - C::WST < 0 ? 0 : wj - C::WST; j < wj; ++j)
+                if (!mbar_wait(&wfull[j % C::WST], (uint32_t)(j / C::WST) & 1u, to)) {
+                    raise_status(p.status, kStatusTimeout);
+                    break;
+                }
         }
-        cluster_sync();  // no CTA leaves while its partials are being read
+        __syncwarp();
+    } else if (warp == 1) {
+        // ----------------------------------------------------- MMA issuer
+        if (elect_one()) {
+            const uint32_t idesc = idesc_bf16_f32(C::BW, BT);
+            const uint64_t adesc0 = sw128_desc(smem_u32(as)), xdesc0 = sw128_desc(smem_u32(xs));
+            constexpr uint32_t kAStep = C::ABYTES >> 4, kXStep = C::XBYTES >> 4;
+            constexpr uint32_t kAAtom = 16384 >> 4, kXAtom = C::XBOX >> 4;
+            int s = 0, committed = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int i = 0; i < nkb && ok; ++i) {
+                if (!mbar_wait(&afull[s], ph, to) || !mbar_wait(&xfull[s], ph, to) ||
+                    !mbar_wait(&gempty[s], ph ^ 1u, to)) {
+                    raise_status(p.status, kStatusTimeout);
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint64_t ad = adesc0 + (uint64_t)(s * kAStep);
+                const uint64_t xd = xdesc0 + (uint64_t)(s * kXStep);
+                const uint32_t d = tmem + (uint32_t)(s * BT);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    tc_mma_f16(d, ad + (uint64_t)((kk >> 2) * kAAtom + 2 * (kk & 3)),
+                               xd + (uint64_t)((kk >> 2) * kXAtom + 2 * (kk & 3)), idesc, kk ? 1u : 0u);
+                tc_commit(&kdone[s]);
+                ++committed;
+                if (++s == C::STG) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+            // TMEM is freed below: the last commit must have landed
+            if (committed > 0) {
+                const int last = committed - 1;
+                if (!mbar_wait(&kdone[last % C::STG], (uint32_t)(last / C::STG) & 1u, to))
+                    raise_status(p.status, kStatusTimeout);
+            }
+        }
+        __syncwarp();
+    } else if (warp >= C::DQ0 && warp < C::FW0) {
+        // ---------------------------------------------------- dequantize
+        const Bf16Lut lut = make_lut(p.t.mag, 1.f);
+        const int r = (warp - C::DQ0) * 32 + lane;  // weight row within the tile
+        const int sw = r & 7;                       // 128-byte swizzle of the dequantized atoms
+        const int swp = (r >> 1) & 3;               // 64-byte swizzle of the packed stage
+        for (int i = 0; i < nkb; ++i) {
+            const int ws = i % C::WST, s = i % C::STG;
+            if (!mbar_wait(&wfull[ws], (uint32_t)(i / C::WST) & 1u, to) ||
+                !mbar_wait(&kdone[s], ((uint32_t)(i / C::STG) & 1u) ^ 1u, to)) {
+                raise_status(p.status, kStatusTimeout);
+                break;
+            }
+            // 16-byte unit u of the row's 64 bytes sits at unit u ^ ((r >> 1) & 3)
+            const uint8_t* prow = wsr + ws * C::WBYTES + r * 64;
+            uint32_t words[16];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const uint4 w = lds128_tc(prow + ((u ^ swp) << 4));
+                words[4 * u + 0] = w.x;
+                words[4 * u + 1] = w.y;
+                words[4 * u + 2] = w.z;
+                words[4 * u + 3] = w.w;
+            }
+            // word c holds k = 8c..8c+7: atom c >> 3, 16-byte unit c & 7 of row r
+            uint8_t* arow = as + s * C::ABYTES + r * 128;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                uint32_t v[4];
+                dequant8(words[c], lut, v);
+                *reinterpret_cast<uint4*>(arow + (c >> 3) * 16384 + (((c & 7) ^ sw) << 4)) =
+                    make_uint4(v[0], v[1], v[2], v[3]);
+            }
+            fence_proxy_async_smem();
+            // The packed-code stage is released only once its words have been
+            // consumed: an arrive issued right after the shared-memory loads
+            // was seen to let the next TMA copy overwrite the stage before
+            // those loads had returned their data.
+            mbar_arrive(&wempty[ws]);
+            mbar_arrive(&afull[s]);
+        }
+    } else if (warp >= C::FW0) {
+        // ---------------------------------------------- fold + epilogue
+        const int q = warp & 3;                  // TMEM lane quadrant of this warp
+        const int r = q * 32 + lane;             // weight row within the tile == TMEM lane
+        const int n = n0 + r;
+        const bool nvalid = n < p.N;
+        const int G = p.K / 128;
+        float tot[C::FCOLS];
+#pragma unroll
+        for (int j = 0; j < C::FCOLS; ++j) tot[j] = 0.f;
+        const uint32_t tlane = tmem + ((uint32_t)(q * 32) << 16);
+        bool ok = true;
+        float s_next = (nvalid && nkb > 0) ? load_scale(p.scales, p.sdt, (size_t)n * G + kb0) : 0.f;
+        for (int i = 0; i < nkb; ++i) {
+            const int s = i % C::STG;
+            const float sc = s_next;
+            if (i + 1 < nkb) s_next = nvalid ? load_scale(p.scales, p.sdt, (size_t)n * G + kb0 + i + 1) : 0.f;
+            if (!mbar_wait(&kdone[s], (uint32_t)(i / C::STG) & 1u, to)) {
+                raise_status(p.status, kStatusTimeout);
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < C::FCOLS; c += 16) {
+                uint32_t v[16];
+                tmem_ld16(tlane + (uint32_t)(s * BT + c), v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) tot[c + j] = fmaf(sc, __uint_as_float(v[j]), tot[c + j]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&gempty[s]);
+        }
+        if (p.splits == 1) {
+            const float rho = p.x_scale ? *p.x_scale : 1.f;
+            if (ok && nvalid) {
+#pragma unroll
+                for (int j = 0; j < C::FCOLS; ++j) {
+                    const int m = m0 + j;
+                    if (m < p.M) {
+                        __nv_bfloat16 y = __float2bfloat16_rn(rho * tot[j]);
+                        p.Y[(size_t)m * p.N + n] = *reinterpret_cast<uint16_t*>(&y);
+                    }
+                }
+            }
+        } else {
+            // every MMA, and so every copy and dequantization, has completed
+            // once the last stage has been folded: the partial tile
+            // [BT tokens][128 rows] overlays the dequantized-code stages
+            float* part = reinterpret_cast<float*>(smem);
+#pragma unroll
+            for (int j = 0; j < C::FCOLS; ++j) part[j * 128 + r] = tot[j];
+        }
     }
+
+    if (p.splits > 1) cluster_reduce_store<BT>(p, smem_u32(smem), n0, m0);
 
     tc_fence_before();
     __syncthreads();
@@ -511,14 +801,95 @@ static cudaError_t launch_tc_bt(const CUtensorMap& mx, const CUtensorMap& mw, co
     return cudaGetLastError();
 }
 
+template <int BT>
+static cudaError_t launch_tcg_bt(const CUtensorMap& mx, const CUtensorMap& mw, const TcParams& p, cudaStream_t st) {
+    using C = TgCfg<BT>;
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(gemm_tcg_kernel<BT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((p.N + C::BW - 1) / C::BW, (p.M + BT - 1) / BT, p.splits);
+    cfg.blockDim = dim3(C::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = (unsigned)p.splits;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_tcg_kernel<BT>, mx, mw, p);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+// Token tile and split count of the group-128 small-M variant (0 when it
+// does not apply): one wave of two CTAs per SM, at least two 128-k stages
+// per split, at most 8 splits (one cluster).
+int tcg_token_tile(int M, int K, int group) {
+    if (group != 128 || K % 128 != 0 || M > 64) return 0;
+    return M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+}
+
+int tcg_splits(int M, int N, int K) {
+    const int BT = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+    const long long tiles = (long long)((N + 127) / 128) * ((M + BT - 1) / BT);
+    const int kblocks = K / 128;
+    const long long slots = 148LL * 2;
+    long long s = (slots + tiles - 1) / tiles;
+    if (tiles * s > slots + slots / 8) s = slots / tiles;
+    if (s > kblocks / 2) s = kblocks / 2;
+    if (s > 8) s = 8;
+    return s < 1 ? 1 : (int)s;
+}
+
 cudaError_t launch_gemm_tc(const uint16_t* X, const uint8_t* packed, const void* scales, int sdt, const FmtTable& t,
                            int M, int N, int K, int group, const float* x_scale, uint16_t* Y, void* ws,
                            size_t ws_bytes, int splits, int* status, unsigned long long timeout_ns,
                            cudaStream_t st) {
-    const int BT = tc_token_tile(M);
-    const int kblocks = (K + 63) / 64;
     (void)ws;
     (void)ws_bytes;
+    const int BTg = tcg_token_tile(M, K, group);
+    if (BTg > 0) {
+        if (splits <= 0) splits = tcg_splits(M, N, K);
+        if (splits > K / 128) splits = K / 128;
+        if (splits > 8) splits = 8;
+        CUtensorMap mx, mw;
+        if (!encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, (uint64_t)K, (uint64_t)M, 64, (uint32_t)BTg,
+                       CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+        if (!encode_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, packed, (uint64_t)K / 2, (uint64_t)N, 64, 128,
+                       CU_TENSOR_MAP_SWIZZLE_64B))
+            return cudaErrorInvalidValue;
+        TcParams p;
+        p.scales = scales;
+        p.sdt = sdt;
+        p.t = t;
+        p.M = M;
+        p.N = N;
+        p.K = K;
+        p.group = group;
+        p.x_scale = x_scale;
+        p.Y = Y;
+        p.splits = splits;
+        p.status = status;
+        p.timeout_ns = timeout_ns;
+        switch (BTg) {
+            case 16: return launch_tcg_bt<16>(mx, mw, p, st);
+            case 32: return launch_tcg_bt<32>(mx, mw, p, st);
+            default: return launch_tcg_bt<64>(mx, mw, p, st);
+        }
+    }
+    const int BT = tc_token_tile(M);
+    const int kblocks = (K + 63) / 64;
     if (splits <= 0) splits = tc_splits(M, N, K);
     if (splits > kblocks) splits = kblocks;
     if (splits > 8) splits = 8;
