@@ -185,6 +185,18 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
                  : "memory");
 }
 
+// Arrive after shared-memory loads have returned their data.  `dep` must be
+// computed from the loaded values and is stored to the calling thread's own
+// scratch word `slot` before the arrive: that store cannot issue before the
+// loads complete, and the arrive (release) is ordered after it, so the stage
+// cannot be released, and overwritten by the next copy, while its loads are
+// still in flight.  A plain arrive right after the loads was seen to let that
+// happen.
+__device__ __forceinline__ void mbar_arrive_after(uint64_t* bar, uint32_t dep, uint32_t* slot) {
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(smem_u32(slot)), "r"(dep) : "memory");
+    mbar_arrive(bar);
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
     asm volatile(
         "{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.release.cta.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(
@@ -284,6 +296,15 @@ __device__ __forceinline__ uint32_t map_dsmem(uint32_t smem_addr, uint32_t rank)
     uint32_t r;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr), "r"(rank));
     return r;
+}
+
+__device__ __forceinline__ float4 ld_dsmem_f32x4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
 }
 
 __device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {

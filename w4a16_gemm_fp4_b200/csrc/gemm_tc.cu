@@ -74,7 +74,8 @@ struct TcCfg {
     static constexpr int TMEM_COLS = NACC * BT;
     static constexpr int RING = AST * ABYTES + XST * XBYTES + WST * WBYTES;
     static constexpr int NBAR = 2 * (XST + WST + AST + NACC);
-    static constexpr int SMEM = RING + 1024 + NBAR * 8 + 16;
+    static constexpr int DEP = DQW * 32 * 4;  // per-dequant-thread scratch words (stage release)
+    static constexpr int SMEM = RING + 1024 + NBAR * 8 + 16 + DEP;
     static_assert(BT * 128 * 4 <= AST * ABYTES + XST * XBYTES, "split-K partials overlay the A and X rings");
 };
 
@@ -105,28 +106,59 @@ __device__ __forceinline__ uint4 lds128_tc(const void* p) {
 // cluster along z, and each CTA has published its fp32 partial tile
 // [BT tokens][128 rows] at the start of its shared memory.  Every CTA sums,
 // in rank order, one slice of tokens over the partial tiles of all CTAs of
-// the cluster (distributed shared memory) and stores it.  All threads take
-// part, and each issues its loads from every rank before the first add.
+// the cluster (distributed shared memory) and stores it.  Each thread owns
+// quads of 4 adjacent rows of one token (16-byte loads) and issues a quad's
+// loads from every rank before the first add, so a slice costs a few round
+// trips to the other CTAs rather than one per output.
 template <int BT>
 __device__ __forceinline__ void cluster_reduce_store(const TcParams& p, uint32_t part, int n0, int m0) {
+    constexpr int kQ = 1;
     cluster_sync();
     const int rank = (int)cluster_ctarank();
     const int j0 = rank * BT / p.splits, j1 = (rank + 1) * BT / p.splits;
-    const int cnt = (j1 - j0) * 128;
+    const int nq = (j1 - j0) * 32;  // quads of rows in this CTA's slice
     const float rho = p.x_scale ? *p.x_scale : 1.f;
-    for (int e = threadIdx.x; e < cnt; e += blockDim.x) {
-        const int j = j0 + (e >> 7), r = e & 127;
-        const uint32_t off = part + (uint32_t)((j * 128 + r) * 4);
-        float v[8];
+    const bool vec_store = (p.N & 3) == 0;
+    for (int q0 = threadIdx.x; q0 < nq; q0 += kQ * blockDim.x) {
+        float4 v[kQ][8];
 #pragma unroll
-        for (int z = 0; z < 8; ++z) v[z] = z < p.splits ? ld_dsmem_f32(map_dsmem(off, (uint32_t)z)) : 0.f;
-        float a = 0.f;
+        for (int u = 0; u < kQ; ++u) {
+            const int q = q0 + u * blockDim.x;
+            const int j = j0 + (q >> 5), r = (q & 31) * 4;
+            const uint32_t off = part + (uint32_t)((j * 128 + r) * 4);
 #pragma unroll
-        for (int z = 0; z < 8; ++z) a += v[z];
-        const int m = m0 + j, n = n0 + r;
-        if (m < p.M && n < p.N) {
-            __nv_bfloat16 y = __float2bfloat16_rn(rho * a);
-            p.Y[(size_t)m * p.N + n] = *reinterpret_cast<uint16_t*>(&y);
+            for (int z = 0; z < 8; ++z)
+                v[u][z] = (q < nq && z < p.splits) ? ld_dsmem_f32x4(map_dsmem(off, (uint32_t)z))
+                                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < kQ; ++u) {
+            const int q = q0 + u * blockDim.x;
+            if (q >= nq) break;
+            const int j = j0 + (q >> 5), r = (q & 31) * 4;
+            float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int z = 0; z < 8; ++z) {
+                a.x += v[u][z].x;
+                a.y += v[u][z].y;
+                a.z += v[u][z].z;
+                a.w += v[u][z].w;
+            }
+            const int m = m0 + j, n = n0 + r;
+            if (m >= p.M) continue;
+            __nv_bfloat16 y[4] = {__float2bfloat16_rn(rho * a.x), __float2bfloat16_rn(rho * a.y),
+                                  __float2bfloat16_rn(rho * a.z), __float2bfloat16_rn(rho * a.w)};
+            uint16_t* dst = p.Y + (size_t)m * p.N + n;
+            if (vec_store && n + 3 < p.N) {
+                uint2 w;
+                w.x = (uint32_t)(*reinterpret_cast<uint16_t*>(&y[0])) | ((uint32_t)(*reinterpret_cast<uint16_t*>(&y[1])) << 16);
+                w.y = (uint32_t)(*reinterpret_cast<uint16_t*>(&y[2])) | ((uint32_t)(*reinterpret_cast<uint16_t*>(&y[3])) << 16);
+                *reinterpret_cast<uint2*>(dst) = w;
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (n + e < p.N) dst[e] = *reinterpret_cast<uint16_t*>(&y[e]);
+            }
         }
     }
     cluster_sync();  // no CTA leaves while its partials are being read
@@ -151,6 +183,7 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
     uint64_t* gfull = aempty + C::AST;      // group accumulator complete
     uint64_t* gempty = gfull + C::NACC;     // group accumulator folded
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gempty + C::NACC);
+    uint32_t* dep_slots = tmem_slot + 4;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = blockIdx.x * C::BW, m0 = blockIdx.y * BT, split = blockIdx.z;
@@ -332,16 +365,21 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
             // of the stage is chunks 2 sub and 2 sub + 1
             const uint8_t* prow = wsr + ws * C::WBYTES + r * 128;
             uint32_t words[kWords];
+            uint32_t dep;
             if (kHalves == 1) {
                 const uint4 w0 = lds128_tc(prow + (((2 * sub) ^ sw) << 4));
                 const uint4 w1 = lds128_tc(prow + (((2 * sub + 1) ^ sw) << 4));
                 words[0] = w0.x; words[1] = w0.y; words[2] = w0.z; words[3] = w0.w;
                 words[kWords > 4 ? 4 : 0] = w1.x; words[kWords > 5 ? 5 : 0] = w1.y;
                 words[kWords > 6 ? 6 : 0] = w1.z; words[kWords > 7 ? 7 : 0] = w1.w;
+                dep = w0.x ^ w1.x;
             } else {
                 const uint4 w0 = lds128_tc(prow + (((2 * sub + hh) ^ sw) << 4));
                 words[0] = w0.x; words[1] = w0.y; words[2] = w0.z; words[3] = w0.w;
+                dep = w0.x;
             }
+            // release the packed-code stage as soon as its words are in registers
+            if (sub == C::KSUP - 1 || i == nkb - 1) mbar_arrive_after(&wempty[ws], dep, dep_slots + tid);
             uint8_t* arow = as + a * C::ABYTES + r * 128;
             const int c0 = hh * kWords;  // first 16-byte unit (8 k) of this thread
 #pragma unroll
@@ -351,9 +389,6 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
                 *reinterpret_cast<uint4*>(arow + (((c0 + c) ^ sw) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
             }
             fence_proxy_async_smem();
-            // release the packed-code stage only after its words are consumed
-            // (see the group-128 variant below)
-            if (sub == C::KSUP - 1 || i == nkb - 1) mbar_arrive(&wempty[ws]);
             mbar_arrive(&afull[a]);
         }
     } else if (warp >= C::FW0) {
@@ -447,7 +482,7 @@ struct TgCfg {
     static constexpr int ABYTES = 2 * 16384;    // dequantized codes: two 128-row x 64-k SW128 atoms
     static constexpr int WBYTES = BW * 64;      // packed codes of one stage: 128 rows x 64 B, 64-byte swizzle
     static constexpr int STG = 2;               // stages == TMEM accumulators
-    static constexpr int WST = 2;               // packed-code stages
+    static constexpr int WST = BT == 16 ? 4 : (BT == 32 ? 3 : 2);  // packed-code stages (as shared memory allows)
     static constexpr int FCOLS = BT;            // accumulator columns per fold thread
     static constexpr int NF = 4;                // fold warps (one TMEM lane quadrant each)
     static constexpr int DQW = 4;               // dequant warps (one weight row per thread)
@@ -457,10 +492,11 @@ struct TgCfg {
     static constexpr int TMEM_COLS = STG * BT < 32 ? 32 : STG * BT;
     static constexpr int RING = STG * (ABYTES + XBYTES) + WST * WBYTES;
     static constexpr int NBAR = 4 * STG + 2 * WST;
+    static constexpr int DEP = DQW * 32 * 4;  // per-dequant-thread scratch words (stage release)
     // the 64-token layout only fits two CTAs per SM without alignment slack:
     // it relies on the 1024-byte-aligned dynamic shared-memory base (checked)
     static constexpr int SLACK = BT == 64 ? 0 : 1024;
-    static constexpr int SMEM = RING + SLACK + NBAR * 8 + 16;
+    static constexpr int SMEM = RING + SLACK + NBAR * 8 + 16 + DEP;
     static_assert(SMEM + 1024 <= 228 * 1024 / 2, "two CTAs per SM");
     static_assert(BT * 128 * 4 <= STG * ABYTES, "split-K partials overlay the dequantized tiles");
 };
@@ -486,6 +522,7 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, 2)
     uint64_t* wempty = wfull + C::WST;      // packed codes read
     uint64_t* gempty = wempty + C::WST;     // accumulator folded (kdone's one arrival is the commit)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gempty + C::STG);
+    uint32_t* dep_slots = tmem_slot + 4;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = blockIdx.x * C::BW, m0 = blockIdx.y * BT, split = blockIdx.z;
@@ -629,6 +666,8 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, 2)
                 words[4 * u + 2] = w.z;
                 words[4 * u + 3] = w.w;
             }
+            // release the packed-code stage as soon as its words are in registers
+            mbar_arrive_after(&wempty[ws], words[0] ^ words[4] ^ words[8] ^ words[12], dep_slots + r);
             // word c holds k = 8c..8c+7: atom c >> 3, 16-byte unit c & 7 of row r
             uint8_t* arow = as + s * C::ABYTES + r * 128;
 #pragma unroll
@@ -639,11 +678,6 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, 2)
                     make_uint4(v[0], v[1], v[2], v[3]);
             }
             fence_proxy_async_smem();
-            // The packed-code stage is released only once its words have been
-            // consumed: an arrive issued right after the shared-memory loads
-            // was seen to let the next TMA copy overwrite the stage before
-            // those loads had returned their data.
-            mbar_arrive(&wempty[ws]);
             mbar_arrive(&afull[s]);
         }
     } else if (warp >= C::FW0) {
