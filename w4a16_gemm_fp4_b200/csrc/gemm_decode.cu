@@ -239,6 +239,7 @@ __device__ __forceinline__ void sts128(void* p, const uint4 v) {
 
 constexpr int kDecMaxK = 24576;  // one buffer of 16 code rows and scale rows must fit shared memory
 constexpr int kDecSmemMax = 226 * 1024;
+constexpr int kDecMaxBuf = 6;  // block buffers per CTA
 
 // Code rows are dense (one bulk copy per block); activation rows sit at a
 // pitch of 64 modulo 128 bytes so that the 8 lanes of a quarter-warp hit 8
@@ -258,7 +259,7 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
     constexpr int kEs = SDT == FP4_SCALE_F16 ? 2 : 4;
     extern __shared__ uint8_t dsmem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem_raw) + 127) & ~uintptr_t(127));
-    __shared__ __align__(8) uint64_t bar[2];  // per buffer: codes and scale rows landed
+    __shared__ __align__(8) uint64_t bar[kDecMaxBuf];  // per buffer: codes and scale rows landed
     __shared__ volatile int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
@@ -271,7 +272,7 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
     const int iters = blockIdx.x < nblk ? (nblk - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
 
     if (threadIdx.x == 0) {
-        for (int b = 0; b < 2; ++b) mbar_init(&bar[b], 1);
+        for (int b = 0; b < nbuf; ++b) mbar_init(&bar[b], 1);
         fence_mbar_init();
         abort_flag = 0;
     }
@@ -432,14 +433,18 @@ int decode_rows_per_cta(int N) { return N >= 8192 ? 2 : 1; }
 
 // Shared-memory plan of the group-128 kernel: two CTAs of 8 warps per SM
 // where they fit, else one CTA of 16 warps; two buffers before one; staged
-// activations before per-chunk reads from L2.
+// activations before per-chunk reads from L2.  (Measured: covering every
+// block of a CTA with a buffer, e.g. one 16-warp CTA per SM with 5 buffers
+// for 688 blocks, was slower than two 8-warp CTAs with two buffers each,
+// whose per-block barriers and reductions overlap.)
 struct DecPlan {
     int nw, nbuf;
     bool xs;
     int smem;
 };
 
-static DecPlan dec_plan(int M, int K) {
+static DecPlan dec_plan(int M, int N, int K) {
+    (void)N;
     for (int xs = 1; xs >= 0; --xs)
         for (int nbuf = 2; nbuf >= 1; --nbuf) {
             const int s8 = dec_smem_bytes(K, M, 8, nbuf, xs);
@@ -489,7 +494,7 @@ static cudaError_t launch_g128_t(const DecodeParams& p, const DecPlan& plan, int
 
 template <int MANT, int SDT>
 static cudaError_t launch_g128_nw(const DecodeParams& p, int* status, unsigned long long to, cudaStream_t st) {
-    const DecPlan plan = dec_plan(p.M, p.K);
+    const DecPlan plan = dec_plan(p.M, p.N, p.K);
     if (plan.nw == 0) return cudaErrorInvalidValue;
     if (plan.xs && plan.nw == 8) return launch_g128_t<MANT, SDT, 8, true>(p, plan, status, to, st);
     if (plan.xs) return launch_g128_t<MANT, SDT, 16, true>(p, plan, status, to, st);
