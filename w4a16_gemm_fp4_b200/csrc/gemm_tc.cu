@@ -481,11 +481,13 @@ struct TgCfg {
     static constexpr int XBYTES = 2 * XBOX;     // activations of one stage (128 k)
     static constexpr int ABYTES = 2 * 16384;    // dequantized codes: two 128-row x 64-k SW128 atoms
     static constexpr int WBYTES = BW * 64;      // packed codes of one stage: 128 rows x 64 B, 64-byte swizzle
+    static constexpr bool kPair = BT <= 64;     // two CTAs per SM for small token tiles
+    static constexpr int CTAS_PER_SM = kPair ? 2 : 1;
     static constexpr int STG = 2;               // stages == TMEM accumulators
-    static constexpr int WST = BT == 16 ? 4 : (BT == 32 ? 3 : 2);  // packed-code stages (as shared memory allows)
-    static constexpr int FCOLS = BT;            // accumulator columns per fold thread
-    static constexpr int NF = 4;                // fold warps (one TMEM lane quadrant each)
-    static constexpr int DQW = 4;               // dequant warps (one weight row per thread)
+    static constexpr int WST = BT == 16 ? 4 : (BT == 32 ? 3 : (BT == 64 ? 2 : 4));  // packed-code stages
+    static constexpr int FCOLS = BT < 64 ? BT : 64;  // accumulator columns per fold thread
+    static constexpr int NF = 4 * (BT / FCOLS);      // fold warps: 4 lane quadrants x column blocks
+    static constexpr int DQW = kPair ? 4 : 8;   // dequant warps: one thread per row, or two (halves of k)
     static constexpr int DQ0 = 2;
     static constexpr int FW0 = DQ0 + DQW;
     static constexpr int THREADS = (FW0 + NF) * 32;
@@ -497,12 +499,13 @@ struct TgCfg {
     // it relies on the 1024-byte-aligned dynamic shared-memory base (checked)
     static constexpr int SLACK = BT == 64 ? 0 : 1024;
     static constexpr int SMEM = RING + SLACK + NBAR * 8 + 16 + DEP;
-    static_assert(SMEM + 1024 <= 228 * 1024 / 2, "two CTAs per SM");
+    static_assert(!kPair || SMEM + 1024 <= 228 * 1024 / 2, "two CTAs per SM");
+    static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
     static_assert(BT * 128 * 4 <= STG * ABYTES, "split-K partials overlay the dequantized tiles");
 };
 
 template <int BT>
-__global__ void __launch_bounds__(TgCfg<BT>::THREADS, 2)
+__global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
     gemm_tcg_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, TcParams p) {
     using C = TgCfg<BT>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -644,8 +647,14 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, 2)
         __syncwarp();
     } else if (warp >= C::DQ0 && warp < C::FW0) {
         // ---------------------------------------------------- dequantize
+        // DQW = 4: one thread per weight row (16 words = 128 k per stage);
+        // DQW = 8: two threads per row, each one 64-k atom (8 words).
+        constexpr int kHalves = C::DQW / 4;
+        constexpr int kWords = 16 / kHalves;
         const Bf16Lut lut = make_lut(p.t.mag, 1.f);
-        const int r = (warp - C::DQ0) * 32 + lane;  // weight row within the tile
+        const int tid = (warp - C::DQ0) * 32 + lane;
+        const int r = tid & 127;                    // weight row within the tile
+        const int hh = kHalves == 1 ? 0 : tid >> 7; // atom (64-k half) of this thread
         const int sw = r & 7;                       // 128-byte swizzle of the dequantized atoms
         const int swp = (r >> 1) & 3;               // 64-byte swizzle of the packed stage
         for (int i = 0; i < nkb; ++i) {
@@ -655,26 +664,33 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, 2)
                 raise_status(p.status, kStatusTimeout);
                 break;
             }
-            // 16-byte unit u of the row's 64 bytes sits at unit u ^ ((r >> 1) & 3)
+            // 16-byte unit u of the row's 64 bytes sits at unit u ^ ((r >> 1) & 3);
+            // units 2 hh, 2 hh + 1 hold atom hh's 8 words
             const uint8_t* prow = wsr + ws * C::WBYTES + r * 64;
-            uint32_t words[16];
+            uint32_t words[kWords];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const uint4 w = lds128_tc(prow + ((u ^ swp) << 4));
+            for (int u = 0; u < kWords / 4; ++u) {
+                const uint4 w = lds128_tc(prow + (((u + 2 * hh) ^ swp) << 4));
                 words[4 * u + 0] = w.x;
                 words[4 * u + 1] = w.y;
                 words[4 * u + 2] = w.z;
                 words[4 * u + 3] = w.w;
             }
             // release the packed-code stage as soon as its words are in registers
-            mbar_arrive_after(&wempty[ws], words[0] ^ words[4] ^ words[8] ^ words[12], dep_slots + r);
-            // word c holds k = 8c..8c+7: atom c >> 3, 16-byte unit c & 7 of row r
+            // (the dependency takes one word of every load)
+            uint32_t dep = 0;
+#pragma unroll
+            for (int u = 0; u < kWords / 4; ++u) dep ^= words[4 * u];
+            mbar_arrive_after(&wempty[ws], dep, dep_slots + tid);
+            // word c of this thread holds k = 8 (c + kWords hh) .. + 7:
+            // atom (c + kWords hh) >> 3, 16-byte unit c & 7 of row r
             uint8_t* arow = as + s * C::ABYTES + r * 128;
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
+            for (int c = 0; c < kWords; ++c) {
+                const int cc = c + kWords * hh;
                 uint32_t v[4];
                 dequant8(words[c], lut, v);
-                *reinterpret_cast<uint4*>(arow + (c >> 3) * 16384 + (((c & 7) ^ sw) << 4)) =
+                *reinterpret_cast<uint4*>(arow + (cc >> 3) * 16384 + (((cc & 7) ^ sw) << 4)) =
                     make_uint4(v[0], v[1], v[2], v[3]);
             }
             fence_proxy_async_smem();
@@ -682,7 +698,9 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, 2)
         }
     } else if (warp >= C::FW0) {
         // ---------------------------------------------- fold + epilogue
+        const int fw = warp - C::FW0;
         const int q = warp & 3;                  // TMEM lane quadrant of this warp
+        const int cb = (fw >> 2) * C::FCOLS;     // first accumulator column of this thread
         const int r = q * 32 + lane;             // weight row within the tile == TMEM lane
         const int n = n0 + r;
         const bool nvalid = n < p.N;
@@ -706,7 +724,7 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, 2)
 #pragma unroll
             for (int c = 0; c < C::FCOLS; c += 16) {
                 uint32_t v[16];
-                tmem_ld16(tlane + (uint32_t)(s * BT + c), v);
+                tmem_ld16(tlane + (uint32_t)(s * BT + cb + c), v);
                 tmem_ld_wait();
 #pragma unroll
                 for (int j = 0; j < 16; ++j) tot[c + j] = fmaf(sc, __uint_as_float(v[j]), tot[c + j]);
@@ -720,7 +738,7 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, 2)
             if (ok && nvalid) {
 #pragma unroll
                 for (int j = 0; j < C::FCOLS; ++j) {
-                    const int m = m0 + j;
+                    const int m = m0 + cb + j;
                     if (m < p.M) {
                         __nv_bfloat16 y = __float2bfloat16_rn(rho * tot[j]);
                         p.Y[(size_t)m * p.N + n] = *reinterpret_cast<uint16_t*>(&y);
@@ -733,7 +751,7 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, 2)
             // [BT tokens][128 rows] overlays the dequantized-code stages
             float* part = reinterpret_cast<float*>(smem);
 #pragma unroll
-            for (int j = 0; j < C::FCOLS; ++j) part[j * 128 + r] = tot[j];
+            for (int j = 0; j < C::FCOLS; ++j) part[(cb + j) * 128 + r] = tot[j];
         }
     }
 
@@ -869,15 +887,15 @@ static cudaError_t launch_tcg_bt(const CUtensorMap& mx, const CUtensorMap& mw, c
 // does not apply): one wave of two CTAs per SM, at least two 128-k stages
 // per split, at most 8 splits (one cluster).
 int tcg_token_tile(int M, int K, int group) {
-    if (group != 128 || K % 128 != 0 || M > 64) return 0;
-    return M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+    if (group != 128 || K % 128 != 0) return 0;
+    return M <= 16 ? 16 : (M <= 32 ? 32 : (M <= 64 ? 64 : 128));
 }
 
 int tcg_splits(int M, int N, int K) {
-    const int BT = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+    const int BT = M <= 16 ? 16 : (M <= 32 ? 32 : (M <= 64 ? 64 : 128));
     const long long tiles = (long long)((N + 127) / 128) * ((M + BT - 1) / BT);
     const int kblocks = K / 128;
-    const long long slots = 148LL * 2;
+    const long long slots = 148LL * (BT <= 64 ? 2 : 1);
     long long s = (slots + tiles - 1) / tiles;
     if (tiles * s > slots + slots / 8) s = slots / tiles;
     if (s > kblocks / 2) s = kblocks / 2;
@@ -919,7 +937,8 @@ cudaError_t launch_gemm_tc(const uint16_t* X, const uint8_t* packed, const void*
         switch (BTg) {
             case 16: return launch_tcg_bt<16>(mx, mw, p, st);
             case 32: return launch_tcg_bt<32>(mx, mw, p, st);
-            default: return launch_tcg_bt<64>(mx, mw, p, st);
+            case 64: return launch_tcg_bt<64>(mx, mw, p, st);
+            default: return launch_tcg_bt<128>(mx, mw, p, st);
         }
     }
     const int BT = tc_token_tile(M);
