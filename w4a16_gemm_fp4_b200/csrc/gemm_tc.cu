@@ -483,15 +483,16 @@ struct TgCfg {
     static constexpr int WBYTES = BW * 64;      // packed codes of one stage: 128 rows x 64 B, 64-byte swizzle
     static constexpr bool kPair = BT <= 64;     // two CTAs per SM for small token tiles
     static constexpr int CTAS_PER_SM = kPair ? 2 : 1;
-    static constexpr int STG = 2;               // stages == TMEM accumulators
-    static constexpr int WST = BT == 16 ? 4 : (BT == 32 ? 3 : (BT == 64 ? 2 : 4));  // packed-code stages
+    static constexpr int STG = BT == 128 ? 3 : 2;  // stages == TMEM accumulators
+    static constexpr int WST = BT == 16 ? 4 : (BT == 32 ? 3 : 2);  // packed-code stages
     static constexpr int FCOLS = BT < 64 ? BT : 64;  // accumulator columns per fold thread
     static constexpr int NF = 4 * (BT / FCOLS);      // fold warps: 4 lane quadrants x column blocks
     static constexpr int DQW = kPair ? 4 : 8;   // dequant warps: one thread per row, or two (halves of k)
     static constexpr int DQ0 = 2;
     static constexpr int FW0 = DQ0 + DQW;
     static constexpr int THREADS = (FW0 + NF) * 32;
-    static constexpr int TMEM_COLS = STG * BT < 32 ? 32 : STG * BT;
+    static constexpr int TMEM_NEED = STG * BT < 32 ? 32 : STG * BT;
+    static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
     static constexpr int RING = STG * (ABYTES + XBYTES) + WST * WBYTES;
     static constexpr int NBAR = 4 * STG + 2 * WST;
     static constexpr int DEP = DQW * 32 * 4;  // per-dequant-thread scratch words (stage release)
