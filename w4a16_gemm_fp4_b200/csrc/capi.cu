@@ -7,6 +7,9 @@
 
 #include "common.cuh"
 
+#include <cmath>
+#include <cstring>
+
 namespace fp4 {
 // kernels (quantize.cu, preshift.cu, gemm_decode.cu, gemm_tc.cu)
 size_t quantize_ws_bytes(long long total, bool search, bool want_sse);
@@ -64,6 +67,29 @@ const FmtTables& tables() {
             for (int i = 0; i < 8; ++i) T.f[f].mag[i] = magnitude(em[f][0], em[f][1], i);
             for (int i = 0; i < 7; ++i) T.f[f].mid[i] = 0.5f * (T.f[f].mag[i] + T.f[f].mag[i + 1]);
             T.f[f].qmax = T.f[f].mag[7];
+            // Test i decides index >= i+1.  For even i it is fl32(y) > mid[i]
+            // (a tie at mid[i] stays on the even index i): fl32(y) exceeds m
+            // exactly when y lies above the rounding boundary between m and
+            // its successor m+, or on it when round-to-even picks m+.  For
+            // odd i it is fl32(y) >= mid[i] (a tie goes up to the even i+1):
+            // the boundary between m's predecessor m- and m, passed on the
+            // boundary when m is the even one.
+            T.tie_up[f] = 0;
+            for (int i = 0; i < 7; ++i) {
+                const float m = T.f[f].mid[i];
+                float lo, hi;
+                if ((i & 1) == 0) {
+                    lo = m;
+                    hi = std::nextafter(m, INFINITY);
+                } else {
+                    lo = std::nextafter(m, 0.f);
+                    hi = m;
+                }
+                T.hb[f][i] = 0.5 * ((double)lo + (double)hi);
+                uint32_t hbits;
+                std::memcpy(&hbits, &hi, 4);
+                if ((hbits & 1u) == 0) T.tie_up[f] |= 1u << i;
+            }
         }
         for (int j = 0; j < 8; ++j) T.cj[j] = (float)exp2(-(double)j / 8.0);
         init = true;

@@ -27,6 +27,11 @@ struct FmtTable {
 struct FmtTables {
     FmtTable f[3];
     float cj[8];  // fl32(2^(-j/8)): real-valued exponent-bias candidates
+    // Exact decision boundaries of the nearest-code tests (see code_threshold
+    // in quantize.cu): test i of format f passes when fl32(|x|/s) lies above
+    // hb[f][i], or exactly on it when bit i of tie_up[f] is set.
+    double hb[3][7];
+    uint32_t tie_up[3];
 };
 
 // Device status word bits (mirrors FP4_DEV_* of the public header).

@@ -98,11 +98,26 @@ __device__ __forceinline__ int code_of(float w, float s, const FmtTable& t, floa
     return (neg ? 8 : 0) | idx;
 }
 
+// Smallest magnitude |x| (fp32) whose quotient fl32(|x|/s) passes a
+// nearest-code test with rounding boundary hb (see FmtTables::hb): the test
+// is monotone in |x|, and it passes exactly when |x| > hb*s, or |x| == hb*s
+// and the tie rounds up.  hb*s is exact in fp64 (25 + 24 significant bits),
+// so the threshold equals what the IEEE division followed by the midpoint
+// compare decides, with no division per weight.  A zero or non-finite
+// scale maps every quotient to index 0 (NaN threshold: no |x| passes).
+__device__ __forceinline__ float code_threshold(double hb, bool tie_up, float s) {
+    if (!(s > 0.f) || isinf(s)) return __int_as_float(0x7fc00000);
+    const double H = hb * (double)s;
+    float T = __double2float_ru(H);  // smallest float >= H
+    if ((double)T == H && !tie_up) T = __int_as_float(__float_as_int(T) + 1);
+    return T;
+}
+
 // Fused pass: group absmax -> scale -> codes -> pack, for a fixed
 // candidate (format, j) taken from kernel arguments or, when `choice` is
 // non-null, from device memory (written by the search).  Optionally
 // accumulates SSE per block into ws_sse[block] (fp64).
-__global__ void __launch_bounds__(kQuantThreads) quantize_kernel(QuantParams p, FmtTables tabs, int fmt, int j,
+__global__ void __launch_bounds__(kQuantThreads, 4) quantize_kernel(QuantParams p, FmtTables tabs, int fmt, int j,
                                                                  const int32_t* choice, int32_t* choice_out,
                                                                  double* ws_sse) {
     if (choice) {
@@ -142,15 +157,30 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(QuantParams p, 
             bool o;
             uint32_t raw;
             const float s = stored_scale(A, cj, t.qmax, p.sdt, &o, &raw);
+            // the unit's 7 x (128 / group) thresholds: lane L < 7 * groups
+            // computes test L % 7 of group L / 7, then every lane gathers
+            // the 7 of its own group
+            const int gl = lane / 7, ti = lane - 7 * gl;
+            const bool tl = gl < (128 / p.group);
+            const float sg = __shfl_sync(0xffffffffu, s, (tl ? gl : 0) * lpg);
+            const float myT = tl ? code_threshold(tabs.hb[fmt][ti], (tabs.tie_up[fmt] >> ti) & 1u, sg) : 0.f;
+            const int g0 = (lane / lpg) * 7;
+            float T[7];
+#pragma unroll
+            for (int i = 0; i < 7; ++i) T[i] = __shfl_sync(0xffffffffu, myT, g0 + i);
             if (!valid[q]) continue;
             ovf |= o;
             uint32_t codes = 0;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                float v;
-                const int c = code_of(w[q][i], s, t, &v);
-                codes |= (uint32_t)c << (4 * i);
+                const float ax = fabsf(w[q][i]);
+                int idx = 0;
+#pragma unroll
+                for (int k = 0; k < 7; ++k) idx += ax >= T[k] ? 1 : 0;
+                const bool neg = signbit(w[q][i]);
+                codes |= (uint32_t)((neg ? 8 : 0) | idx) << (4 * i);
                 if (ws_sse) {
+                    const float v = neg ? -t.mag[idx] : t.mag[idx];
                     const double d = (double)w[q][i] - (double)v * (double)s;
                     sse = fma(d, d, sse);
                 }
