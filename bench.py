@@ -80,8 +80,11 @@ def recorded_traffic(key):
     return e["dram_bytes"]
 
 
-def tc_token_tile(M):
-    return 32 if M <= 32 else (64 if M <= 64 else 128)
+def gemm_kernel_name(M):
+    """Kernel that serves an E2M1 group-128 GEMM with M activation rows."""
+    if M <= 8:
+        return "gemm_decode_g128_kernel"
+    return "gemm_tcg_kernel<%d>" % (16 if M <= 16 else 32 if M <= 32 else 64 if M <= 64 else 128)
 
 
 def host_cores():
@@ -308,7 +311,7 @@ def run_ours(args, world, rank):
     Nd, Kd = mats[idom]["N"], mats[idom]["K"]
     alg = weight_bytes(Nd, Kd) + Mdom * Kd * 2 + Mdom * Nd * 2
     achieved = alg / (per[(idom, Mdom)] * 1e-3) / 1e9
-    kname = "gemm_decode_g128_kernel" if Mdom <= 8 else "gemm_tc_kernel<%d>" % tc_token_tile(Mdom)
+    kname = gemm_kernel_name(Mdom)
     key = "%s %dx%d M=%d" % (kname, Nd, Kd, Mdom)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": recorded_traffic(key),
@@ -505,6 +508,37 @@ def run_reference(args, world, rank):
             "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def profile_case(case):
+    """One configuration, three eager calls (the first loads modules and sets
+    attributes; captures skip it)."""
+    import torch
+    from w4a16_gemm_fp4_b200 import api, build, synth
+    build.build()
+    kind, *dims = case.split(":")
+    dims = [int(d) for d in dims]
+    rng = np.random.default_rng(1)
+    if kind == "gemm":
+        N, K, M = dims
+        W = torch.from_numpy(synth.lognormal_row_weights(rng, N, K)).cuda()
+        q = api.quantize(W, GROUP, api.E2M1)
+        del W
+        X = torch.from_numpy(synth.activations(rng, M, K).view(np.int16)).cuda().view(torch.bfloat16)
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        for _ in range(3):
+            api.gemm(X, q["packed"], q["scales"], api.E2M1, GROUP, out=Y)
+    elif kind == "quantize":
+        N, K = dims
+        W = torch.from_numpy(synth.lognormal_row_weights(rng, N, K)).cuda()
+        o = api.quantize(W, GROUP, api.E2M1)
+        for _ in range(3):
+            api.quantize_into(W, o["packed"], o["scales"], o["choice"], GROUP, api.E2M1)
+    else:
+        raise SystemExit("unknown profile case " + case)
+    torch.cuda.synchronize()
+    st = api.device_status(clear=True)
+    print("profile case %s done, device status %d" % (case, st))
+
+
 TRAFFIC_CMD = ("ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none -k regex:gemm_ "
                "-c 12 --csv --log-file traffic.csv python bench.py --steps 1 --warmup 3 --soak-s 0 --no-parts "
                "--no-e2e --no-cpu-baseline")
@@ -534,7 +568,7 @@ def record_traffic(csv_path):
     out = {}
     for (i, M), lid in zip(keys, order):
         N, K = SHAPES[i]
-        kname = "gemm_decode_g128_kernel" if M <= 8 else "gemm_tc_kernel<%d>" % tc_token_tile(M)
+        kname = gemm_kernel_name(M)
         assert kname.split("<")[0] in vals[lid]["name"], (kname, vals[lid]["name"])
         d = vals[lid]
         out["%s %dx%d M=%d" % (kname, N, K, M)] = {
@@ -558,12 +592,18 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg")
     ap.add_argument("--soak-s", type=float, default=1.5,
                     help="seconds of untimed replays before the timed region (clock sampling)")
+    ap.add_argument("--profile-case", metavar="CASE",
+                    help="run one case a few times and exit, for ncu captures: gemm:N:K:M (E2M1 g128 fp16 "
+                         "scales, synthetic weights and activations) or quantize:N:K")
     ap.add_argument("--record-traffic", metavar="CSV",
                     help="write profiles/traffic.json from an ncu CSV of the first 12 GEMM launches "
                          "(dram__bytes_read.sum, dram__bytes_write.sum) of this script, then exit")
     args = ap.parse_args()
     if args.record_traffic:
         record_traffic(args.record_traffic)
+        return
+    if args.profile_case:
+        profile_case(args.profile_case)
         return
     if args.warmup < 3:
         args.warmup = 3
