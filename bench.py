@@ -80,9 +80,9 @@ def recorded_traffic(key):
     return e["dram_bytes"]
 
 
-def gemm_kernel_name(M):
-    """Kernel that serves an E2M1 group-128 GEMM with M activation rows."""
-    if M <= 8:
+def gemm_kernel_name(api, M, N, K):
+    """Kernel that serves an E2M1 group-128 GEMM of this shape."""
+    if api.gemm_engine_for(M, N, K, GROUP) == api.ENGINE_DECODE:
         return "gemm_decode_g128_kernel"
     return "gemm_tcg_kernel<%d>" % (16 if M <= 16 else 32 if M <= 32 else 64 if M <= 64 else 128)
 
@@ -311,7 +311,7 @@ def run_ours(args, world, rank):
     Nd, Kd = mats[idom]["N"], mats[idom]["K"]
     alg = weight_bytes(Nd, Kd) + Mdom * Kd * 2 + Mdom * Nd * 2
     achieved = alg / (per[(idom, Mdom)] * 1e-3) / 1e9
-    kname = gemm_kernel_name(Mdom)
+    kname = gemm_kernel_name(api, Mdom, Nd, Kd)
     key = "%s %dx%d M=%d" % (kname, Nd, Kd, Mdom)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": recorded_traffic(key),
@@ -549,6 +549,7 @@ def record_traffic(csv_path):
     sweep, in key order (for M in MS, for each matrix); ncu flushes the
     caches before each profiled launch, so the bytes are cold-cache."""
     import csv
+    from w4a16_gemm_fp4_b200 import api
     vals = {}
     order = []
     with open(csv_path) as f:
@@ -568,7 +569,7 @@ def record_traffic(csv_path):
     out = {}
     for (i, M), lid in zip(keys, order):
         N, K = SHAPES[i]
-        kname = gemm_kernel_name(M)
+        kname = gemm_kernel_name(api, M, N, K)
         assert kname.split("<")[0] in vals[lid]["name"], (kname, vals[lid]["name"])
         d = vals[lid]
         out["%s %dx%d M=%d" % (kname, N, K, M)] = {

@@ -181,15 +181,24 @@ FP4_API fp4_status fp4_preshift_calibrate_noalloc(const uint16_t *X, int M, int 
  *   fmt      the format the weights were quantized in (not AUTO).
  *   x_scale  device float (rho from fp4_preshift_calibrate) or NULL for 1.
  *   Y        [M][N] bf16 out; must not alias the inputs.
- *   workspace reserved: fp4_gemm_workspace_size() is 0 for every shape (the
- *            split-K reduction of skinny problems runs between the CTAs of a
- *            thread-block cluster in distributed shared memory); pass NULL, 0.
- * Engines: M <= 8 uses the decode engine (persistent CTAs stream 16-row
- * blocks of packed codes by bulk copy, dequantize in registers, warp-level
- * MMAs); larger M uses the tensor engine (TMA-staged tiles dequantized in
- * shared memory, tcgen05 MMAs into tensor memory; at group 128 and M <= 64
- * one 128-k group per pipeline stage).  Both multiply the exact code values
- * and apply each group scale in fp32.
+ *   workspace optional, 16-byte aligned, not overlapping the other buffers;
+ *            fp4_gemm_workspace_size() bytes (0 for M <= 64; the split-K
+ *            reduction of skinny problems runs between the CTAs of a
+ *            thread-block cluster in distributed shared memory).  For
+ *            M > 64 with E2M1 weights at group 128 it holds the activations
+ *            in f16: each row is scaled by a power of two that brings its
+ *            largest magnitude into [2^14, 2^15) (exact; elements more than
+ *            2^31 below the row maximum round to the f16 subnormal grid)
+ *            and the factor is undone in fp32 in the epilogue, so the codes
+ *            convert to f16 in hardware.  Smaller or NULL: the bf16 path.
+ * Engines (fp4_gemm_engine_for reports the choice): M <= 8, and M <= 16 at
+ * group 128 where the decode engine can hold the activations and two weight
+ * blocks in shared memory, use the decode engine (persistent CTAs stream
+ * 16-row blocks of packed codes by bulk copy, dequantize in registers,
+ * warp-level MMAs); larger M uses the tensor engine (TMA-staged tiles
+ * dequantized in shared memory, tcgen05 MMAs into tensor memory; at group
+ * 128 one 128-k group per pipeline stage).  Both multiply the exact code
+ * values and apply each group scale in fp32.
  * The decode engine's E2M1 path runs its MMAs in f16: activations must lie
  * within the fp16 range (|x| < 65504); smaller than 2^-14 they lose bits.
  * Device status: FP4_DEV_WAIT_TIMEOUT, FP4_DEV_LAYOUT.
@@ -201,11 +210,18 @@ FP4_API fp4_status fp4_gemm(const uint16_t *X, const uint8_t *packed, const void
                     cudaStream_t stream);
 
 /* fp4_gemm with an explicit engine and split-K count (0 = automatic, at
- * most 8); meant for tests and tuning.  The decode engine accepts M <= 8. */
+ * most 8); meant for tests and tuning.  The decode engine accepts M <= 16
+ * at group 128 with K <= 24576 (two 8-token MMA tiles), otherwise M <= 8;
+ * larger M returns FP4_ERR_UNSUPPORTED_SHAPE. */
 FP4_API fp4_status fp4_gemm_ex(const uint16_t *X, const uint8_t *packed, const void *scales,
                        fp4_scale_dtype sdt, fp4_format fmt, int M, int N, int K, int group,
                        const float *x_scale, uint16_t *Y, void *workspace, size_t ws_bytes,
                        fp4_engine engine, int splits, cudaStream_t stream);
+
+/* Engine fp4_gemm runs for this shape (FP4_ENGINE_DECODE or
+ * FP4_ENGINE_TENSOR); host-only, no device call.  Non-positive sizes or an
+ * unsupported group return FP4_ENGINE_AUTO. */
+FP4_API fp4_engine fp4_gemm_engine_for(int M, int N, int K, int group);
 
 /* ------------------------------------------------------------------------
  * fp4_get_device_status -- synchronises `stream`, copies the current

@@ -245,6 +245,15 @@ def test_gemm_decode_block_schedule(fp4, oracle_mod, N, K, M):
     assert gemm_case(fp4, oracle_mod, N + K, N, K, M, engine=fp4.ENGINE_DECODE, rho=1.5) <= TOL
 
 
+@pytest.mark.parametrize("N,K,M", [(256, 512, 9), (200, 1024, 16), (1000, 4096, 16), (600, 11008, 12),
+                                    (4101, 2048, 13)])
+def test_gemm_decode_two_token_tiles(fp4, oracle_mod, N, K, M):
+    """Decode engine with 9..16 activation rows: two 8-token MMA tiles that
+    share each dequantized weight fragment (staged activations, and L2
+    reads where M*K is too large to stage)."""
+    assert gemm_case(fp4, oracle_mod, 3 * N + M, N, K, M, engine=fp4.ENGINE_DECODE, rho=0.5) <= TOL
+
+
 def test_gemm_decode_unaligned_scales(fp4, oracle_mod):
     """A scale pointer that is 4- but not 16-byte aligned: the scale rows are
     then read from global memory instead of travelling with the codes."""
@@ -309,6 +318,54 @@ def test_gemm_engines_agree(fp4, oracle_mod):
     Yref = oracle_mod.gemm(X, res["packed"].cpu().numpy(), res["scales"].cpu().numpy(), 1, 128)
     assert rel_err(a, Yref) <= TOL and rel_err(b, Yref) <= TOL
     assert (a - b).abs().max().item() <= 2 * TOL * float(np.max(np.abs(Yref)))
+
+
+def wide_range_rows(seed, M, K):
+    """Activation rows at magnitudes 2^-60 .. 2^60 (far outside the f16
+    range on both sides), a row of zeros, and a row alternating 2^20 and
+    2^-20 entries."""
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((M, K), dtype=np.float32)
+    x *= np.exp2(rng.integers(-60, 61, M).astype(np.float32))[:, None]
+    x[0] = 0.0
+    x[1, 0::2] *= np.float32(2.0 ** 20)
+    x[1, 1::2] *= np.float32(2.0 ** -20)
+    return synth.to_bf16_bits(x)
+
+
+def row_rel_err(Y, Yref):
+    """Largest per-row error relative to that row's max|Y_ref| (a zero row
+    must come out zero)."""
+    Y = Y.float().cpu().numpy().astype(np.float64)
+    worst = 0.0
+    for m in range(Yref.shape[0]):
+        d = np.max(np.abs(Yref[m]))
+        e = np.max(np.abs(Y[m] - Yref[m]))
+        worst = max(worst, e / d if d > 0 else (0.0 if e == 0 else np.inf))
+    return worst
+
+
+@pytest.mark.parametrize("M,splits", [(65, 0), (200, 0), (300, 0), (300, 1), (130, 3)])
+def test_gemm_f16_activation_rows(fp4, oracle_mod, M, splits):
+    """The 128-token tile runs E2M1 weights in f16 when given the workspace:
+    each activation row is rescaled by a power of two into the f16 range and
+    the factor is undone in the epilogue.  Rows 2^120 apart in magnitude
+    must each meet the bound against their own magnitude, with and without
+    the workspace (bf16 path)."""
+    N, K = 256, 1024
+    W, _ = synth.random_case(40 + M, N, K, 1)
+    X = wide_range_rows(41 + M, M, K)
+    res = fp4.quantize(dev_f32(W), 128, 1)
+    Yref = oracle_mod.gemm(X, res["packed"].cpu().numpy(), res["scales"].cpu().numpy(), 1, 128, 0.5)
+    xs = torch.tensor([0.5], dtype=torch.float32, device="cuda")
+    need = fp4.gemm_workspace_size(M, N, K)
+    assert need >= M * K * 2 + M * 4
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    small = torch.empty(16, dtype=torch.uint8, device="cuda")
+    a = fp4.gemm(dev_bf16(X), res["packed"], res["scales"], 1, 128, x_scale=xs, splits=splits, workspace=ws)
+    b = fp4.gemm(dev_bf16(X), res["packed"], res["scales"], 1, 128, x_scale=xs, splits=splits, workspace=small)
+    assert row_rel_err(a, Yref) <= TOL
+    assert row_rel_err(b, Yref) <= TOL
 
 
 def test_gemm_empty_and_k0(fp4):

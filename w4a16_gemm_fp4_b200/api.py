@@ -27,7 +27,8 @@ STATUS = {0: "FP4_OK", 1: "FP4_ERR_INVALID_ARG", 2: "FP4_ERR_UNSUPPORTED_SHAPE",
 EXPORTS = ("fp4_abi_version", "fp4_status_string", "fp4_quantize_workspace_size", "fp4_quantize",
            "fp4_dequantize", "fp4_preshift_workspace_size", "fp4_preshift_calibrate", "fp4_preshift_apply",
            "fp4_gemm_workspace_size", "fp4_gemm", "fp4_gemm_ex", "fp4_get_device_status",
-           "fp4_set_wait_timeout_us", "fp4_selftest_bounded_wait", "fp4_preshift_calibrate_noalloc")
+           "fp4_set_wait_timeout_us", "fp4_selftest_bounded_wait", "fp4_preshift_calibrate_noalloc",
+           "fp4_gemm_engine_for")
 
 
 class Fp4Error(RuntimeError):
@@ -68,6 +69,7 @@ def lib():
                 "fp4_set_wait_timeout_us": (None, [ll]),
                 "fp4_selftest_bounded_wait": (i, [ll, P]),
                 "fp4_preshift_calibrate_noalloc": (i, [P, i, i, P, P, P]),
+                "fp4_gemm_engine_for": (i, [i, i, i, i]),
             }
             for name, (res, args) in sigs.items():
                 fn = getattr(L, name)
@@ -125,9 +127,10 @@ _ws = {}
 
 
 def _workspace(device, kind="scratch"):
-    """Per-device buffers.  "gemm" is reserved for fp4_gemm, whose split-K
-    tile counters must stay zero between calls; "scratch" serves the calls
-    whose workspace needs no initialisation (quantize, calibrate)."""
+    """Per-device grow-only buffers, one per kind: "gemm" holds fp4_gemm's
+    f16 activations, "scratch" serves quantize and calibrate.  Calls on one
+    stream reuse them in order; calls on concurrent streams need their own
+    (pass ``workspace=``)."""
     key = (device.type, device.index, kind)
     if key not in _ws:
         _ws[key] = Workspace(device)
@@ -215,6 +218,11 @@ def gemm_workspace_size(M, N, K):
     return lib().fp4_gemm_workspace_size(M, N, K)
 
 
+def gemm_engine_for(M, N, K, group=128):
+    """Engine the automatic choice runs for this shape (ENGINE_DECODE or ENGINE_TENSOR)."""
+    return lib().fp4_gemm_engine_for(M, N, K, group)
+
+
 def gemm(X, packed, scales, fmt=E2M1, group=128, x_scale=None, out=None, engine=ENGINE_AUTO, splits=0,
          workspace=None, stream=None):
     """Y = bf16(x_scale * X . dequant(W)^T).  X: [M][K] bf16 CUDA tensor."""
@@ -227,8 +235,6 @@ def gemm(X, packed, scales, fmt=E2M1, group=128, x_scale=None, out=None, engine=
     L = lib()
     if workspace is None:
         need = L.fp4_gemm_workspace_size(M, N, K)
-        if splits > 0:
-            need = max(need, 16384 + splits * M * N * 4)
         ws, wsb = _workspace(X.device, "gemm").get(need)
     else:
         ws, wsb = workspace, workspace.numel() * workspace.element_size()

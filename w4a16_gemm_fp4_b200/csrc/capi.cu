@@ -27,8 +27,10 @@ cudaError_t launch_gemm_decode(const uint16_t* X, const uint8_t* packed, const v
                                const FmtTable& t, int fmt, int M, int N, int K, int group, const float* x_scale,
                                uint16_t* Y, int* status, unsigned long long timeout_ns, cudaStream_t st);
 size_t tc_ws_bytes(int M, int N, int K);
+int decode_max_m(int K, int group);
+bool decode_preferred(int M, int N, int K, int group);
 cudaError_t launch_gemm_tc(const uint16_t* X, const uint8_t* packed, const void* scales, int sdt, const FmtTable& t,
-                           int M, int N, int K, int group, const float* x_scale, uint16_t* Y, void* ws,
+                           bool e2m1, int M, int N, int K, int group, const float* x_scale, uint16_t* Y, void* ws,
                            size_t ws_bytes, int splits, int* status, unsigned long long timeout_ns,
                            cudaStream_t st);
 cudaError_t launch_bounded_wait_probe(int* status, unsigned long long timeout_ns, cudaStream_t st);
@@ -298,8 +300,8 @@ fp4_status fp4_gemm_ex(const uint16_t* X, const uint8_t* packed, const void* sca
     if (!X) return FP4_ERR_INVALID_ARG;
     if (!aligned(X, 16)) return FP4_ERR_MISALIGNED;
     if ((const void*)Y == (const void*)X || (const void*)Y == (const void*)packed) return FP4_ERR_INVALID_ARG;
-    if (engine == FP4_ENGINE_AUTO) engine = M <= kDecodeMaxM ? FP4_ENGINE_DECODE : FP4_ENGINE_TENSOR;
-    if (engine == FP4_ENGINE_DECODE && M > kDecodeMaxM) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if (engine == FP4_ENGINE_AUTO) engine = fp4_gemm_engine_for(M, N, K, group);
+    if (engine == FP4_ENGINE_DECODE && M > decode_max_m(K, group)) return FP4_ERR_UNSUPPORTED_SHAPE;
     const FmtTable& t = tables().f[fmt];
     int* st = status_ptr();
     if (!st) return FP4_ERR_CUDA;
@@ -308,8 +310,14 @@ fp4_status fp4_gemm_ex(const uint16_t* X, const uint8_t* packed, const void* sca
         return cuda_status(launch_gemm_decode(X, packed, scales, (int)sdt, t, (int)fmt, M, N, K, group, x_scale, Y,
                                               st, to_ns, stream));
     }
-    return cuda_status(launch_gemm_tc(X, packed, scales, (int)sdt, t, M, N, K, group, x_scale, Y, workspace,
-                                      ws_bytes, splits, st, to_ns, stream));
+    return cuda_status(launch_gemm_tc(X, packed, scales, (int)sdt, t, fmt == FP4_E2M1, M, N, K, group, x_scale, Y,
+                                      workspace, ws_bytes, splits, st, to_ns, stream));
+}
+
+fp4_engine fp4_gemm_engine_for(int M, int N, int K, int group) {
+    if (M <= 0 || N <= 0 || K <= 0) return FP4_ENGINE_AUTO;
+    if (group != 32 && group != 64 && group != 128) return FP4_ENGINE_AUTO;
+    return decode_preferred(M, N, K, group) ? FP4_ENGINE_DECODE : FP4_ENGINE_TENSOR;
 }
 
 fp4_status fp4_gemm(const uint16_t* X, const uint8_t* packed, const void* scales, fp4_scale_dtype sdt,

@@ -268,6 +268,29 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                  : "memory");
 }
 
+// Eight E2M1 codes (one 32-bit word, code 2j in the low nibble of byte j)
+// -> four f16x2 words by the hardware convert, one instruction per byte:
+// q_j = (v(code 2j) low half, v(code 2j+1) high half), exact values.
+__device__ __forceinline__ void e2m1_to_f16x8(uint32_t w, uint32_t& q0, uint32_t& q1, uint32_t& q2, uint32_t& q3) {
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(q0), "=r"(q1), "=r"(q2), "=r"(q3)
+        : "r"(w));
+}
+
+// Bulk prefetch of a global range into L2 (16-byte aligned address and size).
+// L2 is the point of coherence, so a line fetched early still reflects any
+// later write: the consumer's real reads, issued after the dependency wait,
+// see the producer's data.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
+                 : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -389,6 +412,12 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr) {
 
 // Instruction descriptor: kind::f16, A = B = bf16 (K-major), D = fp32,
 // shape M x N.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
+    return (1u << 4)                       // D format fp32; A and B format f16 (0)
+           | ((uint32_t)(N >> 3) << 17)    // N / 8
+           | ((uint32_t)(M >> 4) << 24);   // M / 16
+}
+
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
     return (1u << 4)                       // D format fp32
            | (1u << 7)                     // A format bf16

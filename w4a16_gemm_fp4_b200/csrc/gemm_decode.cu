@@ -193,18 +193,6 @@ __device__ __forceinline__ void mma_f16_16816(float d[4], uint32_t a0, uint32_t 
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// 8 E2M1 codes (one word, low nibble first) -> 4 f16x2 natural pairs
-__device__ __forceinline__ void e2m1_to_f16x8(uint32_t w, uint32_t& q0, uint32_t& q1, uint32_t& q2, uint32_t& q3) {
-    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
-        : "=r"(q0), "=r"(q1), "=r"(q2), "=r"(q3)
-        : "r"(w));
-}
-
 // bf16x2 -> f16x2 (exact inside the fp16 normal range)
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t x) {
     const float lo = __uint_as_float(x << 16), hi = __uint_as_float(x & 0xffff0000u);
@@ -248,11 +236,13 @@ __host__ __device__ constexpr int dec_pitch(int K) { return K / 2; }
 // codes of 16 rows at the padded pitch + their scale rows (room for fp32)
 __host__ __device__ constexpr int dec_buf_bytes(int K) { return 16 * dec_pitch(K) + 16 * (K / 128) * 4; }
 __host__ __device__ constexpr int dec_xpitch(int K) { return 2 * K + 64; }
+// NT = token tiles of 8 (1 for M <= 8, 2 for M <= 16): the reduction buffer
+// holds NT partial tiles per warp, double-buffered
 __host__ __device__ constexpr int dec_smem_bytes(int K, int M, int nw, int nbuf, bool xs) {
-    return nbuf * dec_buf_bytes(K) + (xs ? M * dec_xpitch(K) : 0) + 2 * nw * 32 * 4 * 4 + 128;
+    return nbuf * dec_buf_bytes(K) + (xs ? M * dec_xpitch(K) : 0) + 2 * nw * 32 * 4 * 4 * (M > 8 ? 2 : 1) + 128;
 }
 
-template <int MANT, int SDT, int NW, bool XS>
+template <int MANT, int SDT, int NW, bool XS, int NT>
 __global__ void __launch_bounds__(NW * 32, 16 / NW)
     gemm_decode_g128_kernel(DecodeParams p, int nbuf, int sc_bulk, int* status, unsigned long long timeout_ns) {
     constexpr bool kCvt = MANT == 1;  // E2M1: hardware convert + f16 mma
@@ -266,7 +256,7 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
     const int K = p.K, G = K >> 7;
     const int P = dec_pitch(K), SB = dec_buf_bytes(K), XP = dec_xpitch(K);
     uint8_t* xs = base + nbuf * SB;
-    float* red = reinterpret_cast<float*>(xs + (XS ? p.M * XP : 0));  // [2][NW][32][4]
+    float* red = reinterpret_cast<float*>(xs + (XS ? p.M * XP : 0));  // [2][NT][NW][32][4]
     const int sc_bytes = 16 * G * kEs;  // scale rows of a full block: a multiple of 32 bytes
     const int nblk = (p.N + 15) / 16;
     const int iters = blockIdx.x < nblk ? (nblk - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
@@ -275,6 +265,17 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
         for (int b = 0; b < nbuf; ++b) mbar_init(&bar[b], 1);
         fence_mbar_init();
         abort_flag = 0;
+    }
+    if (threadIdx.x == 0) {
+        // start every block of this CTA towards L2 before the dependency wait:
+        // the weight stream overlaps the tail of the previous kernel
+        for (int it = 0; it < iters; ++it) {
+            const int n0 = ((int)blockIdx.x + it * (int)gridDim.x) * 16;
+            const int nrows = p.N - n0 < 16 ? p.N - n0 : 16;
+            bulk_prefetch_l2(p.packed + (size_t)n0 * (K / 2), (uint32_t)nrows * (uint32_t)(K / 2));
+            if (sc_bulk && nrows == 16)
+                bulk_prefetch_l2(static_cast<const uint8_t*>(p.scales) + (size_t)n0 * G * kEs, (uint32_t)sc_bytes);
+        }
     }
     __syncthreads();
     pdl_wait();  // inputs may come from the previous kernel in the stream
@@ -325,10 +326,16 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
     }
 
     const int c_begin = warp * G / NW, c_end = (warp + 1) * G / NW;
-    // token g of the mma's 8 columns (columns >= M use token 0 and are never stored)
-    const int gx = g < p.M ? g : 0;
-    const uint8_t* xrow = xs + gx * XP + 16 * t;
-    const uint4* px = reinterpret_cast<const uint4*>(p.X + (size_t)gx * K) + 4 * t;
+    // token 8 tt + g of tile tt's 8 mma columns (columns >= M use token 0 and
+    // are never stored)
+    const uint8_t* xrow[NT];
+    const uint4* px[NT];
+#pragma unroll
+    for (int tt = 0; tt < NT; ++tt) {
+        const int gx = 8 * tt + g < p.M ? 8 * tt + g : 0;
+        xrow[tt] = xs + gx * XP + 16 * t;
+        px[tt] = reinterpret_cast<const uint4*>(p.X + (size_t)gx * K) + 4 * t;
+    }
     const float rho = p.x_scale ? *p.x_scale : 1.f;
 
     for (int it = 0; it < iters; ++it) {
@@ -349,69 +356,90 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
                 return __half2float(__ldg(reinterpret_cast<const __half*>(p.scales) + row * G + c));
             return __ldg(reinterpret_cast<const float*>(p.scales) + row * G + c);
         };
-        uint4 xn[4];
+        uint4 xn[NT][4];
         if (!XS && c_begin < c_end) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) xn[q] = __ldg(px + c_begin * 16 + q);
+            for (int tt = 0; tt < NT; ++tt)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) xn[tt][q] = __ldg(px[tt] + c_begin * 16 + q);
         }
         bool ok = abort_flag == 0;
         if (ok && c_begin < c_end && !mbar_wait(&bar[b], ph, timeout_ns)) ok = false;
         if (!ok) abort_flag = 1;
 
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        float acc[NT][4];
+#pragma unroll
+        for (int tt = 0; tt < NT; ++tt) acc[tt][0] = acc[tt][1] = acc[tt][2] = acc[tt][3] = 0.f;
         for (int c = c_begin; c < c_end && ok; ++c) {
-            uint4 xv[4];
-            if (XS) {
+            uint4 xv[NT][4];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) xv[q] = lds128(xrow + 256 * c + 64 * q);
-            } else {
+            for (int tt = 0; tt < NT; ++tt) {
+                if (XS) {
 #pragma unroll
-                for (int q = 0; q < 4; ++q) xv[q] = x_operand<kCvt>(xn[q]);
-                if (c + 1 < c_end) {
+                    for (int q = 0; q < 4; ++q) xv[tt][q] = lds128(xrow[tt] + 256 * c + 64 * q);
+                } else {
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) xn[q] = __ldg(px + (c + 1) * 16 + q);
+                    for (int q = 0; q < 4; ++q) xv[tt][q] = x_operand<kCvt>(xn[tt][q]);
+                    if (c + 1 < c_end) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) xn[tt][q] = __ldg(px[tt] + (c + 1) * 16 + q);
+                    }
                 }
             }
             const float sa = scale_at(g, c), sb = scale_at(g + 8, c);
             // this lane's 16 bytes of rows g and g+8 for chunk c: bytes 64c + 16t
             const uint4 wa = lds128(wsm + g * P + 64 * c + 16 * t);
             const uint4 wb = lds128(wsm + (g + 8) * P + 64 * c + 16 * t);
-            float part[4] = {0.f, 0.f, 0.f, 0.f};
+            float part[NT][4];
+#pragma unroll
+            for (int tt = 0; tt < NT; ++tt) part[tt][0] = part[tt][1] = part[tt][2] = part[tt][3] = 0.f;
 #pragma unroll
             for (int wi = 0; wi < 4; ++wi) {
-                const uint32_t xb0 = word_of(xv[wi], 0), xb1 = word_of(xv[wi], 1);
-                const uint32_t xb2 = word_of(xv[wi], 2), xb3 = word_of(xv[wi], 3);
                 uint32_t qa[4], qb[4];
                 if (kCvt) {
                     e2m1_to_f16x8(word_of(wa, wi), qa[0], qa[1], qa[2], qa[3]);
                     e2m1_to_f16x8(word_of(wb, wi), qb[0], qb[1], qb[2], qb[3]);
-                    mma_f16_16816(part, qa[0], qb[0], qa[1], qb[1], xb0, xb1);
-                    mma_f16_16816(part, qa[2], qb[2], qa[3], qb[3], xb2, xb3);
                 } else {
                     dequant8_exact<MANT>(word_of(wa, wi), qa);
                     dequant8_exact<MANT>(word_of(wb, wi), qb);
-                    mma_bf16_16816(part, qa[0], qb[0], qa[1], qb[1], xb0, xb1);
-                    mma_bf16_16816(part, qa[2], qb[2], qa[3], qb[3], xb2, xb3);
+                }
+                // the dequantized A fragment serves every token tile
+#pragma unroll
+                for (int tt = 0; tt < NT; ++tt) {
+                    const uint32_t xb0 = word_of(xv[tt][wi], 0), xb1 = word_of(xv[tt][wi], 1);
+                    const uint32_t xb2 = word_of(xv[tt][wi], 2), xb3 = word_of(xv[tt][wi], 3);
+                    if (kCvt) {
+                        mma_f16_16816(part[tt], qa[0], qb[0], qa[1], qb[1], xb0, xb1);
+                        mma_f16_16816(part[tt], qa[2], qb[2], qa[3], qb[3], xb2, xb3);
+                    } else {
+                        mma_bf16_16816(part[tt], qa[0], qb[0], qa[1], qb[1], xb0, xb1);
+                        mma_bf16_16816(part[tt], qa[2], qb[2], qa[3], qb[3], xb2, xb3);
+                    }
                 }
             }
-            acc[0] = fmaf(sa, part[0], acc[0]);
-            acc[1] = fmaf(sa, part[1], acc[1]);
-            acc[2] = fmaf(sb, part[2], acc[2]);
-            acc[3] = fmaf(sb, part[3], acc[3]);
+#pragma unroll
+            for (int tt = 0; tt < NT; ++tt) {
+                acc[tt][0] = fmaf(sa, part[tt][0], acc[tt][0]);
+                acc[tt][1] = fmaf(sa, part[tt][1], acc[tt][1]);
+                acc[tt][2] = fmaf(sb, part[tt][2], acc[tt][2]);
+                acc[tt][3] = fmaf(sb, part[tt][3], acc[tt][3]);
+            }
         }
 
         // cross-warp reduction in warp order (double-buffered region)
-        float* rd = red + (it & 1) * (NW * 32 * 4);
+        float* rd = red + (it & 1) * (NT * NW * 32 * 4);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) rd[(warp * 32 + lane) * 4 + j] = acc[j];
+        for (int tt = 0; tt < NT; ++tt)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) rd[((tt * NW + warp) * 32 + lane) * 4 + j] = acc[tt][j];
         __syncthreads();  // every warp is done with this block's buffer and partials
         if (threadIdx.x == 0 && it + nbuf < iters && abort_flag == 0) issue(it + nbuf);
-        if (threadIdx.x < 128) {
-            const int e = threadIdx.x, l = e >> 2, j = e & 3;
+        if (threadIdx.x < 128 * NT) {
+            const int tt = threadIdx.x >> 7, e = threadIdx.x & 127, l = e >> 2, j = e & 3;
             float sum = 0.f;
 #pragma unroll
-            for (int w = 0; w < NW; ++w) sum += rd[(w * 32 + l) * 4 + j];
-            const int n = n0 + (l >> 2) + 8 * (j >> 1), m = 2 * (l & 3) + (j & 1);
+            for (int w = 0; w < NW; ++w) sum += rd[((tt * NW + w) * 32 + l) * 4 + j];
+            const int n = n0 + (l >> 2) + 8 * (j >> 1), m = 8 * tt + 2 * (l & 3) + (j & 1);
             if (m < p.M && n < p.N) {
                 __nv_bfloat16 y = __float2bfloat16_rn(rho * sum);
                 p.Y[(size_t)m * p.N + n] = *reinterpret_cast<uint16_t*>(&y);
@@ -455,14 +483,14 @@ static DecPlan dec_plan(int M, int N, int K) {
     return {0, 0, false, 0};
 }
 
-template <int MANT, int SDT, int NW, bool XS>
+template <int MANT, int SDT, int NW, bool XS, int NT>
 static cudaError_t launch_g128_t(const DecodeParams& p, const DecPlan& plan, int* status, unsigned long long to,
                                  cudaStream_t st) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= 64) return cudaErrorInvalidDevice;
-    auto kern = gemm_decode_g128_kernel<MANT, SDT, NW, XS>;
+    auto kern = gemm_decode_g128_kernel<MANT, SDT, NW, XS, NT>;
     static bool attr_set[64] = {};
     if (!attr_set[dev]) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmemMax);
@@ -492,13 +520,20 @@ static cudaError_t launch_g128_t(const DecodeParams& p, const DecPlan& plan, int
     return cudaLaunchKernelEx(&cfg, kern, p, plan.nbuf, sc_bulk, status, to);
 }
 
+template <int MANT, int SDT, int NT>
+static cudaError_t launch_g128_plan(const DecodeParams& p, const DecPlan& plan, int* status, unsigned long long to,
+                                    cudaStream_t st) {
+    if (plan.xs && plan.nw == 8) return launch_g128_t<MANT, SDT, 8, true, NT>(p, plan, status, to, st);
+    if (plan.xs) return launch_g128_t<MANT, SDT, 16, true, NT>(p, plan, status, to, st);
+    return launch_g128_t<MANT, SDT, 16, false, NT>(p, plan, status, to, st);
+}
+
 template <int MANT, int SDT>
 static cudaError_t launch_g128_nw(const DecodeParams& p, int* status, unsigned long long to, cudaStream_t st) {
     const DecPlan plan = dec_plan(p.M, p.N, p.K);
     if (plan.nw == 0) return cudaErrorInvalidValue;
-    if (plan.xs && plan.nw == 8) return launch_g128_t<MANT, SDT, 8, true>(p, plan, status, to, st);
-    if (plan.xs) return launch_g128_t<MANT, SDT, 16, true>(p, plan, status, to, st);
-    return launch_g128_t<MANT, SDT, 16, false>(p, plan, status, to, st);
+    if (p.M > 8) return launch_g128_plan<MANT, SDT, 2>(p, plan, status, to, st);
+    return launch_g128_plan<MANT, SDT, 1>(p, plan, status, to, st);
 }
 
 static cudaError_t launch_g128(const DecodeParams& p, int fmt, int* status, unsigned long long to, cudaStream_t st) {
@@ -510,10 +545,25 @@ static cudaError_t launch_g128(const DecodeParams& p, int fmt, int* status, unsi
     return f16 ? launch_g128_nw<0, FP4_SCALE_F16>(p, status, to, st) : launch_g128_nw<0, FP4_SCALE_F32>(p, status, to, st);
 }
 
+// Largest M the decode engine takes: two 8-token MMA tiles on the group-128
+// path, one on the per-group-LUT kernel.
+int decode_max_m(int K, int group) { return (group == 128 && K <= kDecMaxK) ? 16 : 8; }
+
+// Automatic engine choice for M <= decode_max_m: the decode engine for
+// M <= 8; for 9..16 rows only when its plan stages the activations with two
+// block buffers (measured: otherwise the tensor engine is faster).
+bool decode_preferred(int M, int N, int K, int group) {
+    if (M <= 8) return true;
+    if (M > decode_max_m(K, group)) return false;
+    const DecPlan plan = dec_plan(M, N, K);
+    return plan.nw != 0 && plan.xs && plan.nbuf == 2;
+}
+
 cudaError_t launch_gemm_decode(const uint16_t* X, const uint8_t* packed, const void* scales, int sdt,
                                const FmtTable& t, int fmt, int M, int N, int K, int group, const float* x_scale,
                                uint16_t* Y, int* status, unsigned long long timeout_ns, cudaStream_t st) {
     DecodeParams p{X, packed, scales, sdt, t, M, N, K, group, x_scale, Y};
+    if (M > decode_max_m(K, group)) return cudaErrorInvalidValue;
     if (group == 128 && K <= kDecMaxK) return launch_g128(p, fmt, status, timeout_ns, st);
     const int R = decode_rows_per_cta(N);
     const int blocks = (N + 16 * R - 1) / (16 * R);

@@ -42,6 +42,7 @@ struct TcParams {
     FmtTable t;
     int M, N, K, group;
     const float* x_scale;
+    const float* xrow;   // f16 activations: per-row factor 2^e undoing their scaling (else nullptr)
     uint16_t* Y;
     int splits;          // CTAs along K per output tile (one cluster)
     int* status;
@@ -146,6 +147,13 @@ __device__ __forceinline__ void cluster_reduce_store(const TcParams& p, uint32_t
             }
             const int m = m0 + j, n = n0 + r;
             if (m >= p.M) continue;
+            if (p.xrow) {
+                const float f = p.xrow[m];
+                a.x *= f;
+                a.y *= f;
+                a.z *= f;
+                a.w *= f;
+            }
             __nv_bfloat16 y[4] = {__float2bfloat16_rn(rho * a.x), __float2bfloat16_rn(rho * a.y),
                                   __float2bfloat16_rn(rho * a.z), __float2bfloat16_rn(rho * a.w)};
             uint16_t* dst = p.Y + (size_t)m * p.N + n;
@@ -505,7 +513,7 @@ struct TgCfg {
     static_assert(BT * 128 * 4 <= STG * ABYTES, "split-K partials overlay the dequantized tiles");
 };
 
-template <int BT>
+template <int BT, bool F16>
 __global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
     gemm_tcg_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, TcParams p) {
     using C = TgCfg<BT>;
@@ -609,7 +617,7 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
     } else if (warp == 1) {
         // ----------------------------------------------------- MMA issuer
         if (elect_one()) {
-            const uint32_t idesc = idesc_bf16_f32(C::BW, BT);
+            const uint32_t idesc = F16 ? idesc_f16_f32(C::BW, BT) : idesc_bf16_f32(C::BW, BT);
             const uint64_t adesc0 = sw128_desc(smem_u32(as)), xdesc0 = sw128_desc(smem_u32(xs));
             constexpr uint32_t kAStep = C::ABYTES >> 4, kXStep = C::XBYTES >> 4;
             constexpr uint32_t kAAtom = 16384 >> 4, kXAtom = C::XBOX >> 4;
@@ -690,7 +698,10 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
             for (int c = 0; c < kWords; ++c) {
                 const int cc = c + kWords * hh;
                 uint32_t v[4];
-                dequant8(words[c], lut, v);
+                if constexpr (F16)
+                    e2m1_to_f16x8(words[c], v[0], v[1], v[2], v[3]);
+                else
+                    dequant8(words[c], lut, v);
                 *reinterpret_cast<uint4*>(arow + (cc >> 3) * 16384 + (((cc & 7) ^ sw) << 4)) =
                     make_uint4(v[0], v[1], v[2], v[3]);
             }
@@ -741,7 +752,8 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
                 for (int j = 0; j < C::FCOLS; ++j) {
                     const int m = m0 + cb + j;
                     if (m < p.M) {
-                        __nv_bfloat16 y = __float2bfloat16_rn(rho * tot[j]);
+                        const float t = F16 ? tot[j] * p.xrow[m] : tot[j];
+                        __nv_bfloat16 y = __float2bfloat16_rn(rho * t);
                         p.Y[(size_t)m * p.N + n] = *reinterpret_cast<uint16_t*>(&y);
                     }
                 }
@@ -816,11 +828,12 @@ int tc_splits(int M, int N, int K) {
     return s < 1 ? 1 : (int)s;
 }
 
+// The split-K reduction runs in distributed shared memory and needs no
+// workspace; the f16 activations of the 128-token tile do (M > 64).
+size_t tc_f16_ws_bytes(int M, int K);
 size_t tc_ws_bytes(int M, int N, int K) {
-    (void)M;
     (void)N;
-    (void)K;
-    return 0;  // the split-K reduction runs in distributed shared memory
+    return M > 64 && K > 0 ? tc_f16_ws_bytes(M, K) : 0;
 }
 
 template <int BT>
@@ -854,14 +867,86 @@ static cudaError_t launch_tc_bt(const CUtensorMap& mx, const CUtensorMap& mw, co
     return cudaGetLastError();
 }
 
-template <int BT>
+// Activations of the f16 tensor path.  Row m of X (bf16) is multiplied by
+// 2^sh, the power of two that brings its largest finite magnitude into
+// [2^14, 2^15) (sh clamped to [-113, 126]), and rounded to f16; xrow[m] =
+// 2^-sh undoes it in the epilogue.  The scaling is exact, and a bf16 value
+// (8 significant bits) converts to f16 exactly when its scaled magnitude is
+// at least 2^-17: every element within 2^31 of the row's maximum.  Smaller
+// ones round to the f16 subnormal grid (error below 2^-25 after scaling,
+// i.e. under 2^-39 of the row maximum); infinities and NaNs pass through.
+__global__ void __launch_bounds__(256) x_rows_to_f16_kernel(const uint16_t* __restrict__ X, int K,
+                                                            uint16_t* __restrict__ Xh, float* __restrict__ xrow) {
+    __shared__ uint32_t wmax[8];
+    const int m = blockIdx.x, nv = K >> 3;
+    const uint4* src = reinterpret_cast<const uint4*>(X + (size_t)m * K);
+    uint4* dst = reinterpret_cast<uint4*>(Xh + (size_t)m * K);
+    pdl_wait();  // X may come from the previous kernel in the stream
+    pdl_launch_dependents();
+    uint32_t mx2 = 0;  // per-half maxima of the finite magnitudes (bf16 bits order like the values)
+    for (int i = threadIdx.x; i < nv; i += 256) {
+        const uint4 v = src[i];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t a = w[j] & 0x7fff7fffu;
+            mx2 = __vmaxu2(mx2, a & __vcmpltu2(a, 0x7f807f80u));
+        }
+    }
+    uint32_t mx = max(mx2 & 0xffffu, mx2 >> 16);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    mx = wmax[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) mx = max(mx, wmax[w]);
+    const int E = (int)(mx >> 7);  // biased exponent of the row maximum
+    int sh = mx == 0 ? 0 : 141 - (E < 1 ? 1 : E);
+    if (sh > 126) sh = 126;
+    const float sc = __int_as_float((127 + sh) << 23);
+    if (threadIdx.x == 0) xrow[m] = __int_as_float((127 - sh) << 23);
+    for (int i = threadIdx.x; i < nv; i += 256) {
+        const uint4 v = src[i];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t h[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float lo = __uint_as_float(w[j] << 16) * sc, hi = __uint_as_float(w[j] & 0xffff0000u) * sc;
+            asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h[j]) : "f"(hi), "f"(lo));
+        }
+        dst[i] = make_uint4(h[0], h[1], h[2], h[3]);
+    }
+}
+
+// Bytes of the f16 activations (16-byte aligned rows) and their row factors.
+static size_t xh_bytes(int M, int K) { return ((size_t)M * K * 2 + 255) & ~(size_t)255; }
+
+size_t tc_f16_ws_bytes(int M, int K) { return xh_bytes(M, K) + (size_t)M * 4; }
+
+static cudaError_t launch_x_rows_to_f16(const uint16_t* X, int M, int K, uint16_t* Xh, float* xrow, cudaStream_t st) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)M, 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel, X, K, Xh, xrow);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+template <int BT, bool F16>
 static cudaError_t launch_tcg_bt(const CUtensorMap& mx, const CUtensorMap& mw, const TcParams& p, cudaStream_t st) {
     using C = TgCfg<BT>;
     static bool attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_tcg_kernel<BT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        cudaError_t e = cudaFuncSetAttribute(gemm_tcg_kernel<BT, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
@@ -879,7 +964,7 @@ static cudaError_t launch_tcg_bt(const CUtensorMap& mx, const CUtensorMap& mw, c
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_tcg_kernel<BT>, mx, mw, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_tcg_kernel<BT, F16>, mx, mw, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -905,19 +990,22 @@ int tcg_splits(int M, int N, int K) {
 }
 
 cudaError_t launch_gemm_tc(const uint16_t* X, const uint8_t* packed, const void* scales, int sdt, const FmtTable& t,
-                           int M, int N, int K, int group, const float* x_scale, uint16_t* Y, void* ws,
+                           bool e2m1, int M, int N, int K, int group, const float* x_scale, uint16_t* Y, void* ws,
                            size_t ws_bytes, int splits, int* status, unsigned long long timeout_ns,
                            cudaStream_t st) {
-    (void)ws;
-    (void)ws_bytes;
     const int BTg = tcg_token_tile(M, K, group);
     if (BTg > 0) {
         if (splits <= 0) splits = tcg_splits(M, N, K);
         if (splits > K / 128) splits = K / 128;
         if (splits > 8) splits = 8;
+        // E2M1 codes on the 128-token tile: hardware convert to f16 and f16
+        // activations (needs the workspace; without it the bf16 path runs)
+        const bool f16 = BTg == 128 && e2m1 && ws != nullptr && ws_bytes >= tc_f16_ws_bytes(M, K);
+        uint16_t* Xh = f16 ? static_cast<uint16_t*>(ws) : nullptr;
+        float* xrow = f16 ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + xh_bytes(M, K)) : nullptr;
         CUtensorMap mx, mw;
-        if (!encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, (uint64_t)K, (uint64_t)M, 64, (uint32_t)BTg,
-                       CU_TENSOR_MAP_SWIZZLE_128B))
+        if (!encode_2d(&mx, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                       f16 ? Xh : X, (uint64_t)K, (uint64_t)M, 64, (uint32_t)BTg, CU_TENSOR_MAP_SWIZZLE_128B))
             return cudaErrorInvalidValue;
         if (!encode_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, packed, (uint64_t)K / 2, (uint64_t)N, 64, 128,
                        CU_TENSOR_MAP_SWIZZLE_64B))
@@ -931,15 +1019,21 @@ cudaError_t launch_gemm_tc(const uint16_t* X, const uint8_t* packed, const void*
         p.K = K;
         p.group = group;
         p.x_scale = x_scale;
+        p.xrow = xrow;
         p.Y = Y;
         p.splits = splits;
         p.status = status;
         p.timeout_ns = timeout_ns;
+        if (f16) {
+            cudaError_t e = launch_x_rows_to_f16(X, M, K, Xh, xrow, st);
+            if (e != cudaSuccess) return e;
+            return launch_tcg_bt<128, true>(mx, mw, p, st);
+        }
         switch (BTg) {
-            case 16: return launch_tcg_bt<16>(mx, mw, p, st);
-            case 32: return launch_tcg_bt<32>(mx, mw, p, st);
-            case 64: return launch_tcg_bt<64>(mx, mw, p, st);
-            default: return launch_tcg_bt<128>(mx, mw, p, st);
+            case 16: return launch_tcg_bt<16, false>(mx, mw, p, st);
+            case 32: return launch_tcg_bt<32, false>(mx, mw, p, st);
+            case 64: return launch_tcg_bt<64, false>(mx, mw, p, st);
+            default: return launch_tcg_bt<128, false>(mx, mw, p, st);
         }
     }
     const int BT = tc_token_tile(M);
@@ -963,6 +1057,7 @@ cudaError_t launch_gemm_tc(const uint16_t* X, const uint8_t* packed, const void*
     p.K = K;
     p.group = group;
     p.x_scale = x_scale;
+    p.xrow = nullptr;
     p.Y = Y;
     p.splits = splits;
     p.status = status;
