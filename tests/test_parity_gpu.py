@@ -368,6 +368,19 @@ def test_gemm_f16_activation_rows(fp4, oracle_mod, M, splits):
     assert row_rel_err(b, Yref) <= TOL
 
 
+@pytest.mark.parametrize("K", [2176, 4224, 8320, 16512])
+def test_gemm_f16_row_lengths(fp4, oracle_mod, K):
+    """Row lengths that take each form of the f16 activation pre-pass (the
+    row held in 2, 4 or 8 registers per thread, or read twice)."""
+    M, N = 70, 128
+    W, _ = synth.random_case(K, N, K, 1)
+    X = wide_range_rows(K + 1, M, K)
+    res = fp4.quantize(dev_f32(W), 128, 1)
+    Yref = oracle_mod.gemm(X, res["packed"].cpu().numpy(), res["scales"].cpu().numpy(), 1, 128)
+    Y = fp4.gemm(dev_bf16(X), res["packed"], res["scales"], 1, 128)
+    assert row_rel_err(Y, Yref) <= TOL
+
+
 def test_gemm_empty_and_k0(fp4):
     packed = torch.zeros((16, 0), dtype=torch.uint8, device="cuda")
     scales = torch.zeros((16, 0), dtype=torch.float16, device="cuda")

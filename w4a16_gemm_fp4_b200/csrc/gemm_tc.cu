@@ -492,7 +492,7 @@ struct TgCfg {
     static constexpr bool kPair = BT <= 64;     // two CTAs per SM for small token tiles
     static constexpr int CTAS_PER_SM = kPair ? 2 : 1;
     static constexpr int STG = BT == 128 ? 3 : 2;  // stages == TMEM accumulators
-    static constexpr int WST = BT == 16 ? 4 : (BT == 32 ? 3 : 2);  // packed-code stages
+    static constexpr int WST = BT == 16 ? 4 : (BT == 32 || BT == 128 ? 3 : 2);  // packed-code stages
     static constexpr int FCOLS = BT < 64 ? BT : 64;  // accumulator columns per fold thread
     static constexpr int NF = 4 * (BT / FCOLS);      // fold warps: 4 lane quadrants x column blocks
     static constexpr int DQW = kPair ? 4 : 8;   // dequant warps: one thread per row, or two (halves of k)
@@ -875,6 +875,26 @@ static cudaError_t launch_tc_bt(const CUtensorMap& mx, const CUtensorMap& mw, co
 // at least 2^-17: every element within 2^31 of the row's maximum.  Smaller
 // ones round to the f16 subnormal grid (error below 2^-25 after scaling,
 // i.e. under 2^-39 of the row maximum); infinities and NaNs pass through.
+//
+// R = 16-byte vectors of the row each thread keeps in registers (one read
+// of X); R = 0 reads the row twice (any K).
+__device__ __forceinline__ uint32_t finite_mag_max2(uint32_t mx2, uint32_t w) {
+    const uint32_t a = w & 0x7fff7fffu;  // magnitudes; >= 0x7f80 is inf or NaN
+    return __vmaxu2(mx2, a & __vcmpltu2(a, 0x7f807f80u));
+}
+
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4 v, float sc) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t h[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float lo = __uint_as_float(w[j] << 16) * sc, hi = __uint_as_float(w[j] & 0xffff0000u) * sc;
+        asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h[j]) : "f"(hi), "f"(lo));
+    }
+    return make_uint4(h[0], h[1], h[2], h[3]);
+}
+
+template <int R>
 __global__ void __launch_bounds__(256) x_rows_to_f16_kernel(const uint16_t* __restrict__ X, int K,
                                                             uint16_t* __restrict__ Xh, float* __restrict__ xrow) {
     __shared__ uint32_t wmax[8];
@@ -884,13 +904,21 @@ __global__ void __launch_bounds__(256) x_rows_to_f16_kernel(const uint16_t* __re
     pdl_wait();  // X may come from the previous kernel in the stream
     pdl_launch_dependents();
     uint32_t mx2 = 0;  // per-half maxima of the finite magnitudes (bf16 bits order like the values)
-    for (int i = threadIdx.x; i < nv; i += 256) {
-        const uint4 v = src[i];
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint4 v[R > 0 ? R : 1];
+    if constexpr (R > 0) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const uint32_t a = w[j] & 0x7fff7fffu;
-            mx2 = __vmaxu2(mx2, a & __vcmpltu2(a, 0x7f807f80u));
+        for (int r = 0; r < R; ++r) {
+            const int i = threadIdx.x + r * 256;
+            v[r] = i < nv ? src[i] : make_uint4(0u, 0u, 0u, 0u);
+            mx2 = finite_mag_max2(mx2, v[r].x);
+            mx2 = finite_mag_max2(mx2, v[r].y);
+            mx2 = finite_mag_max2(mx2, v[r].z);
+            mx2 = finite_mag_max2(mx2, v[r].w);
+        }
+    } else {
+        for (int i = threadIdx.x; i < nv; i += 256) {
+            const uint4 u = src[i];
+            mx2 = finite_mag_max2(finite_mag_max2(finite_mag_max2(finite_mag_max2(mx2, u.x), u.y), u.z), u.w);
         }
     }
     uint32_t mx = max(mx2 & 0xffffu, mx2 >> 16);
@@ -906,16 +934,14 @@ __global__ void __launch_bounds__(256) x_rows_to_f16_kernel(const uint16_t* __re
     if (sh > 126) sh = 126;
     const float sc = __int_as_float((127 + sh) << 23);
     if (threadIdx.x == 0) xrow[m] = __int_as_float((127 - sh) << 23);
-    for (int i = threadIdx.x; i < nv; i += 256) {
-        const uint4 v = src[i];
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        uint32_t h[4];
+    if constexpr (R > 0) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float lo = __uint_as_float(w[j] << 16) * sc, hi = __uint_as_float(w[j] & 0xffff0000u) * sc;
-            asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h[j]) : "f"(hi), "f"(lo));
+        for (int r = 0; r < R; ++r) {
+            const int i = threadIdx.x + r * 256;
+            if (i < nv) dst[i] = bf16x8_to_f16x8(v[r], sc);
         }
-        dst[i] = make_uint4(h[0], h[1], h[2], h[3]);
+    } else {
+        for (int i = threadIdx.x; i < nv; i += 256) dst[i] = bf16x8_to_f16x8(src[i], sc);
     }
 }
 
@@ -934,7 +960,13 @@ static cudaError_t launch_x_rows_to_f16(const uint16_t* X, int M, int K, uint16_
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel, X, K, Xh, xrow);
+    const int nv = K / 8;
+    cudaError_t e;
+    if (nv <= 256) e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<1>, X, K, Xh, xrow);
+    else if (nv <= 512) e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<2>, X, K, Xh, xrow);
+    else if (nv <= 1024) e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<4>, X, K, Xh, xrow);
+    else if (nv <= 2048) e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<8>, X, K, Xh, xrow);
+    else e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<0>, X, K, Xh, xrow);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
