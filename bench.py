@@ -436,7 +436,8 @@ def run_parts(api, torch, peaks, dev, stream):
     flops = sum(2.0 * X.shape[0] * N * K for (N, K) in ((4096, 4096), (11008, 4096)))
     tf = flops / (ms * 1e-3) / 1e12
     out["prefill"] = {"workload": "LLaMA-7B prefill X 2048x4096 (1% outlier channels x50), pre-shift on, "
-                                  "W 4096x4096 + 11008x4096", "ms": round(ms, 4), "tflops": round(tf, 1),
+                                  "W 4096x4096 + 11008x4096; each call includes its f16 activation pre-pass",
+                      "ms": round(ms, 4), "tflops": round(tf, 1),
                       "peak_tflops": peaks["bf16_tflops"], "frac": round(tf / peaks["bf16_tflops"], 4)}
     ws_cal = torch.zeros(api.lib().fp4_preshift_workspace_size(*X.shape), dtype=torch.uint8, device=dev)
     ms_pro = time_graph(torch, lambda: api.preshift_apply(X, shift, rho, out=Xt), stream, 20)
