@@ -281,6 +281,15 @@ def test_gemm_tensor_split_k(fp4, oracle_mod, splits):
     assert gemm_case(fp4, oracle_mod, 5, 256, 1024, 40, engine=fp4.ENGINE_TENSOR, splits=splits, rho=2.5) <= TOL
 
 
+@pytest.mark.parametrize("M,N,fmt", [(65, 256, 1), (129, 200, 1), (300, 136, 1), (300, 130, 1), (200, 264, 0)])
+def test_gemm_tensor_tile_store(fp4, oracle_mod, M, N, fmt):
+    """Without split K the 128-token tile stores its output through shared
+    memory in 16-byte chunks, bounded by M and N (N % 8 == 0); other N store
+    element by element."""
+    assert gemm_case(fp4, oracle_mod, M + 3 * N, N, 512, M, fmt=fmt, engine=fp4.ENGINE_TENSOR, splits=1,
+                     rho=0.25) <= TOL
+
+
 @pytest.mark.parametrize("fmt,sdt", [(0, "f16"), (2, "f32")])
 def test_gemm_tensor_formats(fp4, oracle_mod, fmt, sdt):
     assert gemm_case(fp4, oracle_mod, 9, 128, 256, 100, fmt=fmt, sdt=sdt, engine=fp4.ENGINE_TENSOR) <= TOL

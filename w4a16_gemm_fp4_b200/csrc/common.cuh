@@ -259,6 +259,11 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
         : "memory");
 }
 
+// barrier among `count` threads (a multiple of 32) of the CTA, id 1..15
+__device__ __forceinline__ void named_barrier_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // 1D bulk copy global -> shared (16-byte aligned addresses and size),
 // completion on an mbarrier.  No multicast.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {

@@ -504,10 +504,12 @@ struct TgCfg {
     static constexpr int RING = STG * (ABYTES + XBYTES) + WST * WBYTES;
     static constexpr int NBAR = 4 * STG + 2 * WST;
     static constexpr int DEP = DQW * 32 * 4;  // per-dequant-thread scratch words (stage release)
+    // per fold warp, the f16 path's row factors of its FCOLS tokens
+    static constexpr int XFB = kPair ? 0 : NF * FCOLS * 4;
     // the 64-token layout only fits two CTAs per SM without alignment slack:
     // it relies on the 1024-byte-aligned dynamic shared-memory base (checked)
     static constexpr int SLACK = BT == 64 ? 0 : 1024;
-    static constexpr int SMEM = RING + SLACK + NBAR * 8 + 16 + DEP;
+    static constexpr int SMEM = RING + SLACK + NBAR * 8 + 16 + DEP + XFB;
     static_assert(!kPair || SMEM + 1024 <= 228 * 1024 / 2, "two CTAs per SM");
     static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
     static_assert(BT * 128 * 4 <= STG * ABYTES, "split-K partials overlay the dequantized tiles");
@@ -535,6 +537,11 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
     uint64_t* gempty = wempty + C::WST;     // accumulator folded (kdone's one arrival is the commit)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gempty + C::STG);
     uint32_t* dep_slots = tmem_slot + 4;
+    float* xf_slots = reinterpret_cast<float*>(dep_slots + C::DEP / 4);
+    volatile int* wide_fail = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    // the 128-token tile without split stores through shared memory in
+    // 16-byte chunks (rows of N bf16 must be multiples of 16 bytes)
+    const bool wide = !C::kPair && p.splits == 1 && (p.N & 7) == 0;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = blockIdx.x * C::BW, m0 = blockIdx.y * BT, split = blockIdx.z;
@@ -558,6 +565,7 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
         fence_mbar_init();
         prefetch_tmap(&tmX);
         prefetch_tmap(&tmW);
+        *wide_fail = 0;
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -717,6 +725,17 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
         const int n = n0 + r;
         const bool nvalid = n < p.N;
         const int G = p.K / 128;
+        // epilogue inputs, fetched before the stages: rho, and on the f16 path
+        // this warp's token factors (in shared memory, read back as broadcasts)
+        const float rho = p.x_scale ? *p.x_scale : 1.f;
+        float* xfw = xf_slots + fw * C::FCOLS;
+        if constexpr (F16) {
+            for (int j = lane; j < C::FCOLS; j += 32) {
+                const int m = m0 + cb + j;
+                xfw[j] = m < p.M ? p.xrow[m] : 0.f;
+            }
+            __syncwarp();
+        }
         float tot[C::FCOLS];
 #pragma unroll
         for (int j = 0; j < C::FCOLS; ++j) tot[j] = 0.f;
@@ -745,14 +764,24 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
             __syncwarp();
             if (lane == 0) mbar_arrive(&gempty[s]);
         }
-        if (p.splits == 1) {
-            const float rho = p.x_scale ? *p.x_scale : 1.f;
+        if (wide) {
+            // every MMA, and so every copy and dequantization, has completed
+            // once the last stage has been folded: the fp32 tile [128 tokens]
+            // [128 rows] * rho goes over the dequantized-code stages (row =
+            // token: the lanes' consecutive weight rows are consecutive words)
+            // and all dequant and fold warps store it below.  No loads here:
+            // a load per element would serialise on its latency.
+            float* ep = reinterpret_cast<float*>(smem);
+            if (!ok) *wide_fail = 1;
+#pragma unroll
+            for (int j = 0; j < C::FCOLS; ++j) ep[(cb + j) * 128 + r] = rho * tot[j];
+        } else if (p.splits == 1) {
             if (ok && nvalid) {
 #pragma unroll
                 for (int j = 0; j < C::FCOLS; ++j) {
                     const int m = m0 + cb + j;
                     if (m < p.M) {
-                        const float t = F16 ? tot[j] * p.xrow[m] : tot[j];
+                        const float t = F16 ? tot[j] * xfw[j] : tot[j];
                         __nv_bfloat16 y = __float2bfloat16_rn(rho * t);
                         p.Y[(size_t)m * p.N + n] = *reinterpret_cast<uint16_t*>(&y);
                     }
@@ -769,6 +798,39 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
     }
 
     if (p.splits > 1) cluster_reduce_store<BT>(p, smem_u32(smem), n0, m0);
+    if (wide && warp >= C::DQ0) {
+        // 16-byte output chunks (8 weight rows of one token) over the dequant
+        // and fold warps: the f16 path's token factor, bf16x2 converts and
+        // coalesced vector stores, all chunks' loads issued first
+        constexpr int kT = (C::DQW + C::NF) * 32, kC = BT * 16 / kT;
+        static_assert(BT * 16 % kT == 0, "whole chunks per thread");
+        named_barrier_sync(1, kT);
+        if (*wide_fail == 0) {
+            const float* ep = reinterpret_cast<const float*>(smem);
+            const int c0 = (int)threadIdx.x - C::DQ0 * 32;
+            float4 a[kC], b[kC];
+            float f[kC];
+#pragma unroll
+            for (int u = 0; u < kC; ++u) {
+                const int c = c0 + u * kT, j = c >> 4, m = m0 + j;
+                a[u] = *reinterpret_cast<const float4*>(ep + j * 128 + (c & 15) * 8);
+                b[u] = *reinterpret_cast<const float4*>(ep + j * 128 + (c & 15) * 8 + 4);
+                f[u] = F16 && m < p.M ? p.xrow[m] : 1.f;
+            }
+#pragma unroll
+            for (int u = 0; u < kC; ++u) {
+                const int c = c0 + u * kT, j = c >> 4, n = n0 + (c & 15) * 8, m = m0 + j;
+                if (m < p.M && n < p.N) {
+                    uint4 o;
+                    o.x = pack_bf16x2(a[u].x * f[u], a[u].y * f[u]);
+                    o.y = pack_bf16x2(a[u].z * f[u], a[u].w * f[u]);
+                    o.z = pack_bf16x2(b[u].x * f[u], b[u].y * f[u]);
+                    o.w = pack_bf16x2(b[u].z * f[u], b[u].w * f[u]);
+                    *reinterpret_cast<uint4*>(p.Y + (size_t)m * p.N + n) = o;
+                }
+            }
+        }
+    }
 
     tc_fence_before();
     __syncthreads();
