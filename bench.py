@@ -54,16 +54,25 @@ def read_peaks():
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def _code_only(text):
+    """C++ source without comments and blank lines (string literals kept)."""
+    import re
+    pat = re.compile(r'//[^\n]*|/\*.*?\*/|"(?:\\.|[^"\\])*"', re.S)
+    text = pat.sub(lambda m: m.group(0) if m.group(0).startswith('"') else "", text)
+    return "\n".join(l.rstrip() for l in text.splitlines() if l.strip())
+
+
 def kernel_sources_sha():
-    """Digest of the CUDA sources: per-launch DRAM traffic recorded under
-    profiles/ is valid only for the kernels it was measured on."""
+    """Digest of the CUDA sources' code (comments and blank lines dropped):
+    per-launch DRAM traffic recorded under profiles/ is valid only for the
+    kernels it was measured on."""
     import hashlib
     h = hashlib.sha256()
     d = os.path.join(ROOT, "w4a16_gemm_fp4_b200", "csrc")
     for f in sorted(os.listdir(d)):
         if f.endswith((".cu", ".cuh")):
             h.update(f.encode())
-            h.update(open(os.path.join(d, f), "rb").read())
+            h.update(_code_only(open(os.path.join(d, f), encoding="utf-8").read()).encode())
     return h.hexdigest()[:16]
 
 
