@@ -1,11 +1,13 @@
-// gemm_decode.cu -- W4A16 GEMM for skinny activations (M <= 8) on sm_100a.
+// gemm_decode.cu -- W4A16 GEMM for skinny activations on sm_100a: M <= 8
+// (the per-lane-LUT kernel, any group), M <= 16 (the group-128 kernel).
 //
 // Y[m,n] = bf16( rho * sum_k X[m,k] * v(code[n,k]) * s[n, k/g] )
 // (LLM-FP4 summary page "首个支持4-bit浮点量化的LLM来了", efficient matrix
 // multiplication: the per-group scales stay outside the 4-bit products.)
 //
 // Decode is bound by streaming the packed weights from HBM (0.5 B per
-// weight plus the scales).  Design:
+// weight plus the scales).  Design of the per-lane-LUT kernel (groups 32 and
+// 64, and group 128 beyond the group-128 kernel's K):
 //  - a CTA owns 16*R weight rows and all of K; its 8 warps split K in
 //    128-element chunks and reduce their fp32 partial sums in shared memory
 //    (fixed order, no workspace, deterministic);
@@ -171,11 +173,17 @@ __global__ void __launch_bounds__(256) gemm_decode_kernel(DecodeParams p) {
 // block takes exactly two bulk copies (its codes and its scale rows): a
 // bulk copy costs the issuing thread on the order of a hundred cycles, so
 // per-row copies would make issue, not HBM, the limit.  Every DRAM request
-// is one long contiguous run.  The activations are staged once per CTA in shared memory, already
-// in the operand form of the mma and ordered so that the four lanes sharing
-// a token read 64 contiguous bytes; where M * K is too large for that they are
-// read from L2 per chunk instead.  The warps split K into chunks and reduce
-// their fp32 sums in shared memory in warp order (deterministic).
+// is one long contiguous run.  Before its dependency wait (the weights do
+// not come from the previous kernel) thread 0 starts all of the CTA's blocks
+// towards L2, so the weight stream overlaps the previous kernel's tail.
+//
+// Activations.  They are staged once per CTA in shared memory, already in
+// the operand form of the mma and ordered so that the four lanes sharing a
+// token read 64 contiguous bytes; where M * K is too large for that they are
+// read from L2 per chunk instead.  Tokens form NT tiles of 8 mma columns
+// (NT = 2 for 9 <= M <= 16): each chunk's codes are dequantized once and
+// feed every tile's mma.  The warps split K into chunks and reduce their
+// fp32 sums in shared memory in warp order (deterministic).
 //
 // Dequantization:
 //  - E2M1: the hardware e2m1x2 -> f16x2 convert, one instruction per two

@@ -3,32 +3,37 @@
 // Y[m,n] = bf16( rho * sum_g s[n,g] * sum_{k in g} X[m,k] * v(code[n,k]) )
 // (LLM-FP4 summary page "首个支持4-bit浮点量化的LLM来了", efficient matrix
 // multiplication: the full-precision group scale stays outside the 4-bit
-// product.)  The tensor cores multiply the EXACT code values v (bf16 holds
-// every value of the three formats) by the bf16 activations with fp32
-// accumulation; each group's partial sum is scaled by s in fp32.  No
+// product.)  The tensor cores multiply the EXACT code values v (bf16 and
+// f16 hold every value of the three formats) by the 16-bit activations with
+// fp32 accumulation; each group's partial sum is scaled by s in fp32.  No
 // weight is ever rounded, so the only rounding besides fp32 accumulation
-// is the final bf16 store.
+// is the final bf16 store (and, on the f16 path, the activations' f16
+// subnormal range far below each row's maximum: see x_rows_to_f16_kernel).
 //
-// CTA tile: 128 weight rows (MMA M) x BT activation rows (MMA N), 64 k per
-// pipeline stage.  The product is computed transposed, D[n][m] = W . X^T:
-// the 128 weight rows map onto the 128 TMEM lanes, so the per-row group
-// scale is a per-lane scalar.
+// Two kernels, both with the product computed transposed, D[n][m] = W . X^T:
+// the 128 weight rows of a CTA tile (MMA M) map onto the 128 TMEM lanes, so
+// the per-row group scale is a per-lane scalar; BT activation rows are MMA N.
+//   gemm_tc_kernel<BT>        groups of 32 or 64: 64-k stages, four TMEM
+//                             group accumulators;
+//   gemm_tcg_kernel<BT, F16>  group 128: one group per stage, one TMEM
+//                             accumulator per stage (below).
 //
 // Warp roles (2 + DQW + NF warps):
-//   warp 0       TMA producer: X tile (bf16, 128-byte swizzle) and the
-//                packed code tile (uint8 [128][32], 32-byte swizzle) into a
-//                ring of shared-memory stages;
-//   warp 1       TMEM allocator and MMA issuer: one thread issues
-//                tcgen05.mma (K = 16) into one of two per-group TMEM
-//                accumulators, committing each finished group to the fold
-//                warps and each consumed stage back to the producer;
-//   DQW warps    dequantize codes into the exact bf16 values, K-major with
-//                the 128-byte swizzle (byte-plane LUT, 16-byte stores);
+//   warp 0       TMA producer: activation tiles (128-byte swizzle) and the
+//                packed code tiles (uint8, 128 rows) into shared-memory rings;
+//   warp 1       TMEM allocator and MMA issuer: one thread issues tcgen05.mma
+//                (K = 16) into the group's TMEM accumulator and commits;
+//   DQW warps    dequantize codes into exact 16-bit values, K-major with the
+//                128-byte swizzle (byte-plane LUT to bf16, or for E2M1 on the
+//                f16 path the hardware e2m1x2 -> f16x2 convert; 16-byte
+//                stores);
 //   NF warps     fold: for each group, tcgen05.ld the group accumulator and
 //                add s[n,g] * it to fp32 totals held in registers, then
-//                release the accumulator; finally the epilogue (* rho ->
-//                bf16 -> global, or fp32 split-K partials reduced in fixed
-//                order by the last CTA of the tile).
+//                release the accumulator; finally the epilogue: * rho (and
+//                the f16 path's token factor) -> bf16 -> global, directly or
+//                through shared memory with the dequant warps' help, or fp32
+//                split-K partials reduced across a CTA cluster in
+//                distributed shared memory.
 // Every mbarrier wait is bounded; a wait that gives up sets
 // FP4_DEV_WAIT_TIMEOUT and the CTA winds down normally (its copies awaited,
 // TMEM freed).  No multicast is used.
@@ -469,7 +474,7 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
 }
 
 // ---------------------------------------------------------------------------
-// Group-128 variant for small token tiles (M <= 64, BT in {16, 32, 64}).
+// Group-128 variant (BT in {16, 32, 64} two CTAs per SM; BT = 128 one).
 // A k-block is one group (128 k): the MMA thread issues its 8 K=16 steps
 // into the stage's own TMEM accumulator and commits ONCE.  That commit both
 // frees the stage (dequantized codes, activations) for reuse and hands the
