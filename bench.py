@@ -10,9 +10,12 @@ GB/s: packed codes + scales streamed per step / step time (all ranks).
 
 Also measured in the same run and reported under "parts": the quantize
 pass (GB/s), the prefill GEMM at M = 2048 (TFLOP/s) on the LLaMA-7B
-prefill workload with the pre-shift, and the format/bias search on a
-LLaMA-13B-shaped 5120x5120 matrix.  ``--impl reference`` times the CPU
-oracle on a bounded sample of the same workload, in the same unit.
+prefill workload with the pre-shift, the format/bias search on a
+LLaMA-13B-shaped 5120x5120 matrix, and passes over the full 40-layer
+LLaMA-13B-shaped linear stack (6.54 GB packed): decode at M in {1, 4, 16,
+64} (weight GB/s, tokens/s-equivalent) and prefill at M = 2048.
+``--impl reference`` times the CPU oracle on a bounded sample of the same
+workload, in the same unit.
 """
 from __future__ import annotations
 
@@ -338,6 +341,11 @@ def run_ours(args, world, rank):
     parts = {}
     if not args.no_parts and rank == 0:
         parts = run_parts(api, torch, peaks, dev, stream)
+        if not args.no_stack:
+            try:
+                parts["llama13b_stack"] = run_stack(api, torch, peaks, dev, stream)
+            except Exception as exc:  # reported, never fatal to the bench line
+                parts["llama13b_stack"] = {"error": "%s: %s" % (type(exc).__name__, exc)}
     return {
         "value": value, "ms_per_step": ms / args.steps, "roofline": roofline, "clocks": clk, "e2e": e2e,
         "gpu_launches": len(keys) * args.steps, "per_m": per_m, "parts": parts, "copies": copies,
@@ -459,6 +467,51 @@ def run_parts(api, torch, peaks, dev, stream):
                                                      True), stream, 5, warm=1)
     out["search"] = {"workload": "5120x5120 Student-t(5)*0.015, 3 formats x 8 bias candidates + pack",
                      "ms": round(ms, 3), "candidate_evals_per_s": round(24 * W.numel() / (ms * 1e-3), 0)}
+    return out
+
+
+def run_stack(api, torch, peaks, dev, stream, layers=40):
+    """The full LLaMA-13B-shaped linear stack: 40 layers x {q, k, v, o
+    5120x5120; gate, up 13824x5120; down 5120x13824}, weights drawn on the
+    GPU and quantized to E2M1 g128 fp16 scales (6.54 GB packed, far beyond
+    L2).  One pass = the 280 fp4_gemm calls in layer order; decode passes at
+    M in {1, 4, 16, 64} give weight GB/s and tokens/s-equivalent (M rows per
+    pass, linear layers only), one prefill pass at M = 2048 gives TFLOP/s."""
+    from w4a16_gemm_fp4_b200 import synth
+    mats = []
+    for layer in range(layers):
+        for _, w in synth.stack_layer_weights(layer, device=dev):
+            q = api.quantize(w, GROUP, api.E2M1)
+            mats.append((q["packed"], q["scales"], w.shape[0], w.shape[1]))
+            del w, q
+    torch.cuda.synchronize()
+    wbytes = sum(weight_bytes(N, K) for (_, _, N, K) in mats)
+    dims = sorted({K for (_, _, _, K) in mats} | {N for (_, _, N, _) in mats})
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(4)
+    out = {"workload": "llama13b_stack: %d layers x 7 matrices, E2M1 g128 fp16 scales, weights ~ N(0, 0.02^2) "
+                       "drawn on the GPU; X ~ N(0, 1) bf16" % layers,
+           "matrices": len(mats), "weight_bytes": wbytes}
+    for M in (1, 4, 16, 64, 2048):
+        xs = {d: torch.randn((M, d), generator=gen, device=dev).to(torch.bfloat16) for d in dims}
+        ys = {d: torch.empty((M, d), dtype=torch.bfloat16, device=dev) for d in dims}
+
+        def one_pass():
+            for (pk, sc, N, K) in mats:
+                api.gemm(xs[K], pk, sc, api.E2M1, GROUP, out=ys[N])
+        ms = time_graph(torch, one_pass, stream, 3 if M < 2048 else 2, warm=1)
+        if M < 2048:
+            gbs = wbytes / (ms * 1e-3) / 1e9
+            out["decode_M%d" % M] = {"ms_per_pass": round(ms, 4), "weight_gbs": round(gbs, 1),
+                                     "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                                     "tokens_per_s_equiv": round(M / (ms * 1e-3), 1)}
+        else:
+            tf = sum(2.0 * M * N * K for (_, _, N, K) in mats) / (ms * 1e-3) / 1e12
+            out["prefill_M2048"] = {"ms_per_pass": round(ms, 3), "tflops": round(tf, 1),
+                                    "frac": round(tf / peaks["bf16_tflops"], 4)}
+        del xs, ys
+    del mats
+    torch.cuda.empty_cache()
     return out
 
 
@@ -598,7 +651,8 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--no-parts", action="store_true", help="skip the quantize/prefill/search legs")
+    ap.add_argument("--no-parts", action="store_true", help="skip the quantize/prefill/search/stack legs")
+    ap.add_argument("--no-stack", action="store_true", help="skip the 40-layer 13B-shaped stack leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg")
     ap.add_argument("--soak-s", type=float, default=1.5,
