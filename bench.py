@@ -181,13 +181,21 @@ def barrier(world):
 
 
 def max_over_ranks(world, value):
+    """The largest of the ranks' values (device time: the slowest rank)."""
     if world == 1:
         return value
     import torch
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_gbs(world, bytes_per_rank_step, steps, ms_max):
+    """Weight GB/s of the whole job: the bytes every rank streamed over the
+    slowest rank's time (replicas: each rank runs the full sweep)."""
+    return world * bytes_per_rank_step * steps / (ms_max * 1e-3) / 1e9
 
 
 # --------------------------------------------------------------- our arm
@@ -308,12 +316,12 @@ def run_ours(args, world, rank):
     if st:
         raise RuntimeError("device status %#x during the timed region" % st)
 
-    total_bytes = step_weight_bytes() * args.steps * world
-    value = total_bytes / (ms * 1e-3) / 1e9
+    value = whole_job_gbs(world, step_weight_bytes(), args.steps, ms)
 
     groups = {}
     for (i, M), t in per.items():
-        eng = "decode" if M <= 8 else "tensor"
+        eng = "/".join(sorted({"decode" if api.gemm_engine_for(M, N, K, GROUP) == api.ENGINE_DECODE else "tensor"
+                               for (N, K) in SHAPES}))
         g = groups.setdefault((eng, M), {"ms": 0.0, "bytes": 0.0, "launches": 0})
         g["ms"] += t
         g["launches"] += 1
