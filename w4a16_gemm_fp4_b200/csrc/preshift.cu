@@ -12,6 +12,8 @@
 // All three passes are HBM-bound streams over X (bf16, 16-byte vectors).
 #include "common.cuh"
 
+#include <atomic>
+
 namespace fp4 {
 
 constexpr int kColsPerBlock = 512;  // 256 threads x 2 bf16 columns
@@ -161,18 +163,27 @@ static __device__ __align__(256) float g_calib_scratch[kNoAllocFloats];
 
 // Host code must not use g_calib_scratch as a device address (on the host
 // the name stands for a host-side shadow); the device address is fetched
-// once per device, with that device current, and cached.
+// once per device, with that device current, and cached.  The cache is
+// atomic so that host threads calling on different streams may race on the
+// first lookup (both store the same address).  A cached address belongs to
+// the context that was current at the lookup, like the library's other
+// per-device state: a process that resets a device must not call the
+// library on it again.
+static std::atomic<float*> g_scratch_ptrs[64];
+
 static float* noalloc_scratch_ptr() {
-    static float* ptrs[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    if (!ptrs[dev]) {
+    float* ptr = g_scratch_ptrs[dev].load(std::memory_order_acquire);
+    if (!ptr) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_calib_scratch) != cudaSuccess) return nullptr;
-        ptrs[dev] = reinterpret_cast<float*>(p);
+        ptr = reinterpret_cast<float*>(p);
+        g_scratch_ptrs[dev].store(ptr, std::memory_order_release);
     }
-    return ptrs[dev];
+    return ptr;
 }
+
 
 int noalloc_max_k() { return kNoAllocFloats; }
 
