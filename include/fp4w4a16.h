@@ -25,6 +25,11 @@
  *    of a per-device status word read by fp4_get_device_status().
  *  - Empty problems (a zero dimension) succeed without launching, except
  *    that fp4_gemm with K == 0 writes zeros to Y.
+ *  - The library keeps per-device state that it sets up on first use (the
+ *    status word's address, kernel attributes, the address of the built-in
+ *    calibration buffer).  It belongs to the context that was current then:
+ *    after cudaDeviceReset the library must not be called on that device
+ *    again in the same process.
  *  - Weight layouts produced by fp4_quantize and read by fp4_gemm:
  *      packed [N][K/2] uint8: element k of row n is nibble (k & 1) of byte
  *                             k/2, low nibble first (even k in bits 0..3);
@@ -181,26 +186,30 @@ FP4_API fp4_status fp4_preshift_calibrate_noalloc(const uint16_t *X, int M, int 
  *   fmt      the format the weights were quantized in (not AUTO).
  *   x_scale  device float (rho from fp4_preshift_calibrate) or NULL for 1.
  *   Y        [M][N] bf16 out; must not alias the inputs.
- *   workspace optional, 16-byte aligned, not overlapping the other buffers;
- *            fp4_gemm_workspace_size() bytes (0 for M <= 64; the split-K
- *            reduction of skinny problems runs between the CTAs of a
- *            thread-block cluster in distributed shared memory).  For
- *            M > 64 with E2M1 weights at group 128 it holds the activations
- *            in f16: each row is scaled by a power of two that brings its
- *            largest magnitude into [2^14, 2^15) (exact; elements more than
- *            2^31 below the row maximum round to the f16 subnormal grid)
- *            and the factor is undone in fp32 in the epilogue, so the codes
- *            convert to f16 in hardware.  Smaller or NULL: the bf16 path.
- * Engines (fp4_gemm_engine_for reports the choice): M <= 8, and M <= 16 at
- * group 128 where the decode engine can hold the activations and two weight
- * blocks in shared memory, use the decode engine (persistent CTAs stream
- * 16-row blocks of packed codes by bulk copy, dequantize in registers,
- * warp-level MMAs); larger M uses the tensor engine (TMA-staged tiles
- * dequantized in shared memory, tcgen05 MMAs into tensor memory; at group
- * 128 one 128-k group per pipeline stage).  Both multiply the exact code
- * values and apply each group scale in fp32.
- * The decode engine's E2M1 path runs its MMAs in f16: activations must lie
- * within the fp16 range (|x| < 65504); smaller than 2^-14 they lose bits.
+ *   workspace 16-byte aligned, not overlapping the other buffers, of
+ *            fp4_gemm_workspace_size() bytes.  It holds the activations
+ *            prepared once per call (f16 for E2M1, bf16 otherwise, paired
+ *            in the order the MMA operands take them) and, for the decode
+ *            engine, one partial tile per CTA piece plus one counter per
+ *            128-row tile.  E2M1 rows are scaled by a power of two that
+ *            brings their largest magnitude into [2^14, 2^15) (exact;
+ *            elements more than 2^31 below the row maximum round to the f16
+ *            subnormal grid) and the factor is undone in fp32 in the
+ *            epilogue, so every bf16 activation is accepted.  With the
+ *            automatic engine a workspace that is too small (or NULL)
+ *            falls back to the tensor engine's bf16 path.
+ * Engines (fp4_gemm_engine_for reports the choice): at group 128 M <= 64,
+ * and at groups 32/64 M <= 8, use the decode engine; larger M uses the
+ * tensor engine (TMA-staged tiles dequantized in shared memory, tcgen05
+ * MMAs into tensor memory, one group per pipeline stage).  The group-128
+ * decode engine runs one persistent CTA per SM over an even split of all
+ * (128-row tile, 2-group chunk) units: TMA streams the codes, dequantize
+ * warps write the exact code values into tensor memory as the MMA's A
+ * operand, tcgen05 MMAs multiply them by the activations, and each group's
+ * scale is applied in fp32 as the accumulator is folded; a tile split
+ * between CTAs is summed by the CTA that completes it, in CTA order, so
+ * the result does not depend on timing.  Groups 32/64 use warp-level MMAs
+ * over a lookup-table dequantization (no workspace).
  * Device status: FP4_DEV_WAIT_TIMEOUT, FP4_DEV_LAYOUT.
  * ---------------------------------------------------------------------- */
 FP4_API size_t fp4_gemm_workspace_size(int M, int N, int K);
@@ -209,9 +218,11 @@ FP4_API fp4_status fp4_gemm(const uint16_t *X, const uint8_t *packed, const void
                     const float *x_scale, uint16_t *Y, void *workspace, size_t ws_bytes,
                     cudaStream_t stream);
 
-/* fp4_gemm with an explicit engine and split-K count (0 = automatic, at
- * most 8); meant for tests and tuning.  The decode engine accepts M <= 16
- * at group 128 with K <= 24576 (two 8-token MMA tiles), otherwise M <= 8;
+/* fp4_gemm with an explicit engine and split count (0 = automatic); meant
+ * for tests and tuning.  For the tensor engine `splits` is the split-K
+ * count (at most 8); for the group-128 decode engine it is the number of
+ * CTAs.  The decode engine accepts M <= 64 at group 128 (and needs the
+ * workspace: FP4_ERR_WORKSPACE otherwise) and M <= 8 at groups 32/64;
  * larger M returns FP4_ERR_UNSUPPORTED_SHAPE. */
 FP4_API fp4_status fp4_gemm_ex(const uint16_t *X, const uint8_t *packed, const void *scales,
                        fp4_scale_dtype sdt, fp4_format fmt, int M, int N, int K, int group,

@@ -89,9 +89,8 @@ def test_gemm_argument_errors(L):
     assert g(Y=MIS) == 3
     assert g(engine=7) == 1
     assert g(splits=-1) == 1
-    assert g(M=17, engine=1) == 2         # decode engine: M <= 16 at group 128 ...
+    assert g(M=65, engine=1) == 2         # decode engine: M <= 64 at group 128 ...
     assert g(M=9, group=64, engine=1) == 2  # ... and M <= 8 otherwise
-    assert g(M=9, K=24704, engine=1) == 2
     assert g(Y=Xp) == 1                   # output aliases the input
     # empty problems succeed without touching the device
     assert g(M=0) == 0
@@ -99,20 +98,18 @@ def test_gemm_argument_errors(L):
 
 
 def test_gemm_engine_choice(L):
-    """Automatic engine: decode for M <= 8; for 9..16 rows at group 128 only
-    where the decode kernel holds the activations (16 rows x (2K + 64) B)
-    and two weight blocks in shared memory; the tensor engine otherwise."""
+    """Automatic engine: at group 128 the decode (tensor-memory) engine for
+    M <= 64 at any K; at groups 32 and 64 the decode kernel for M <= 8; the
+    tensor engine otherwise."""
     e = L.fp4_gemm_engine_for
     for K in (128, 4096, 11008, 24576, 40960):
-        assert e(1, 4096, K, 128) == 1 and e(8, 11008, K, 128) == 1 and e(8, 64, K, 32) == 1
-    assert e(12, 4096, 4096, 128) == 1
-    assert e(12, 11008, 4096, 128) == 1
-    assert e(16, 4096, 4096, 128) == 2     # one block buffer left: tensor engine
-    assert e(12, 4096, 11008, 128) == 2    # activations do not fit
-    assert e(9, 4096, 4096, 64) == 2       # group 64: decode engine takes M <= 8
-    assert e(17, 4096, 4096, 128) == 2 and e(64, 4096, 4096, 128) == 2 and e(2048, 4096, 4096, 128) == 2
+        for M in (1, 8, 12, 16, 17, 33, 64):
+            assert e(M, 4096, K, 128) == 1
+        assert e(65, 4096, K, 128) == 2 and e(2048, 11008, K, 128) == 2
+    assert e(8, 64, 4096, 32) == 1 and e(8, 4096, 4096, 64) == 1
+    assert e(9, 4096, 4096, 64) == 2 and e(9, 4096, 4096, 32) == 2
     assert e(0, 4096, 4096, 128) == 0 and e(4, 4096, 4096, 96) == 0
-    assert api.gemm_engine_for(12, 4096, 4096) == api.ENGINE_DECODE
+    assert api.gemm_engine_for(64, 4096, 4096) == api.ENGINE_DECODE
 
 
 def test_preshift_argument_errors(L):
@@ -125,10 +122,21 @@ def test_preshift_argument_errors(L):
 
 
 def test_workspace_sizes(L):
-    assert L.fp4_gemm_workspace_size(1, 4096, 4096) == 0        # decode engine: none
-    assert L.fp4_gemm_workspace_size(64, 4096, 4096) == 0       # split-K reduces in a CTA cluster
-    # the 128-token tile (M > 64) takes f16 activations: M x K halves
-    # (rounded to 256 bytes) and one fp32 factor per row
+    # decode engine (M <= 64): the activations prepared once per call (M x K
+    # halves, then one fp32 factor per row, each rounded up to 256 bytes),
+    # two fp32 partial tiles [token tile][128] per CTA (one CTA per SM: 148
+    # without a device) and one counter per 128-row tile
+    def up(b):
+        return (b + 255) // 256 * 256
+
+    def dec(M, N, K, bt):
+        tiles = (N + 127) // 128
+        chunks = tiles * ((K // 128) // (2 if (K // 128) % 2 == 0 else 1))
+        ctas = min(148, chunks)
+        return up(M * K * 2) + up(M * 4) + 2 * ctas * bt * 128 * 4 + up(tiles * 4)
+    assert L.fp4_gemm_workspace_size(1, 4096, 4096) == dec(1, 4096, 4096, 16)
+    assert L.fp4_gemm_workspace_size(33, 11008, 4096) == dec(33, 11008, 4096, 64)
+    assert L.fp4_gemm_workspace_size(64, 200, 384) == dec(64, 200, 384, 64)   # 2 tiles x 3 one-group chunks
     assert L.fp4_gemm_workspace_size(65, 4096, 4096) == ((65 * 4096 * 2 + 255) // 256) * 256 + 65 * 4
     assert L.fp4_gemm_workspace_size(2048, 4096, 4096) == 2048 * 4096 * 2 + 2048 * 4
     assert L.fp4_quantize_workspace_size(4096, 4096, 128, 1, 0) >= 8

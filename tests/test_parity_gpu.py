@@ -209,13 +209,21 @@ def test_preshift_all_zero(fp4):
 
 # ----------------------------------------------------------------------- GEMM
 
-def gemm_case(fp4, oracle_mod, seed, N, K, M, group=128, fmt=1, sdt="f16", engine=0, splits=0, rho=None):
+def small_ws():
+    """A workspace too small for the prepared activations: the GEMM then
+    converts them inside the kernel."""
+    return torch.empty(16, dtype=torch.uint8, device="cuda")
+
+
+def gemm_case(fp4, oracle_mod, seed, N, K, M, group=128, fmt=1, sdt="f16", engine=0, splits=0, rho=None,
+              workspace=None):
     W, X = synth.random_case(seed, N, K, M)
     ref_q = oracle_mod.quantize(W, group, fmt, False, None, sdt)
     res = fp4.quantize(dev_f32(W), group, fmt, False, None, sdt)
     assert_quant_equal(res, ref_q)
     xs = None if rho is None else torch.tensor([rho], dtype=torch.float32, device="cuda")
-    Y = fp4.gemm(dev_bf16(X), res["packed"], res["scales"], fmt, group, x_scale=xs, engine=engine, splits=splits)
+    Y = fp4.gemm(dev_bf16(X), res["packed"], res["scales"], fmt, group, x_scale=xs, engine=engine, splits=splits,
+                 workspace=workspace)
     Yref = oracle_mod.gemm(X, ref_q["packed"], ref_q["scales"], fmt, group, 1.0 if rho is None else rho)
     return rel_err(Y, Yref)
 
@@ -226,32 +234,75 @@ def test_gemm_decode_engine(fp4, oracle_mod, M, N, K, group):
     assert gemm_case(fp4, oracle_mod, 7 * M + N, N, K, M, group=group, engine=fp4.ENGINE_DECODE) <= TOL
 
 
-@pytest.mark.parametrize("fmt,sdt", [(0, "f16"), (2, "f32"), (1, "f32")])
-def test_gemm_decode_formats(fp4, oracle_mod, fmt, sdt):
-    assert gemm_case(fp4, oracle_mod, 3, 96, 256, 4, fmt=fmt, sdt=sdt, engine=fp4.ENGINE_DECODE, rho=0.75) <= TOL
+@pytest.mark.parametrize("M", [4, 24, 64])
+@pytest.mark.parametrize("fmt,sdt", [(0, "f16"), (2, "f32"), (1, "f32"), (0, "f32"), (2, "f16")])
+def test_gemm_decode_formats(fp4, oracle_mod, fmt, sdt, M):
+    """Every format and scale type through the decode engine: E2M1 runs its
+    codes through the hardware f16 convert (activations prepared as scaled
+    f16 rows), E1M2 and E3M0 by bit placement to bf16 (activations prepared
+    as re-paired bf16 rows)."""
+    assert gemm_case(fp4, oracle_mod, 3 + M, 96, 256, M, fmt=fmt, sdt=sdt, engine=fp4.ENGINE_DECODE, rho=0.75) <= TOL
+
+
+def test_gemm_decode_needs_workspace(fp4, oracle_mod):
+    """The decode engine prepares the activations in the workspace: forced
+    without one it refuses (FP4_ERR_WORKSPACE, nothing launched); the
+    automatic choice then takes the tensor engine, which needs none."""
+    W, X = synth.random_case(12, 200, 512, 8)
+    res = fp4.quantize(dev_f32(W), 128, 1)
+    with pytest.raises(fp4.Fp4Error) as err:
+        fp4.gemm(dev_bf16(X), res["packed"], res["scales"], 1, 128, engine=fp4.ENGINE_DECODE, workspace=small_ws())
+    assert err.value.code == 4
+    Y = fp4.gemm(dev_bf16(X), res["packed"], res["scales"], 1, 128, workspace=small_ws())
+    Yref = oracle_mod.gemm(X, res["packed"].cpu().numpy(), res["scales"].cpu().numpy(), 1, 128)
+    assert rel_err(Y, Yref) <= TOL
 
 
 @pytest.mark.parametrize("N,K,M", [
-    (10007, 256, 3),    # more blocks than two per resident CTA; ragged last block
-    (40, 6272, 2),      # one CTA of 16 warps per SM, two buffers, odd chunk count
-    (2400, 24576, 1),   # largest K of the contiguous-block path: one buffer, two blocks per CTA
-    (5000, 11008, 8),   # activations too large to stage: read from L2 per chunk, two buffers
-    (2500, 13824, 1),   # staged activations with one buffer
-    (64, 24704, 2),     # beyond it: the per-group kernel
+    (10007, 256, 3),    # many row tiles, one chunk each, ragged last tile
+    (40, 6272, 2),      # one row tile of 49 groups (odd: one-group chunks) over 49 CTAs
+    (2400, 24576, 1),   # long K
+    (5000, 11008, 8),
+    (2500, 13824, 1),
+    (64, 24704, 2),     # K of 193 groups
+    (4101, 2048, 13),
+    (600, 11008, 12),
+    (128, 128, 5),      # a single chunk of one group
 ])
 def test_gemm_decode_block_schedule(fp4, oracle_mod, N, K, M):
-    """Decode engine, group 128: the persistent walk over 16-row blocks in
-    each of its shared-memory configurations."""
+    """Decode engine, group 128: the code chunks of all row tiles split into
+    one contiguous range per CTA (whole tiles stored directly, pieces
+    reduced by the CTA that completes the tile), ragged row tiles, two- and
+    one-group chunks."""
     assert gemm_case(fp4, oracle_mod, N + K, N, K, M, engine=fp4.ENGINE_DECODE, rho=1.5) <= TOL
 
 
-@pytest.mark.parametrize("N,K,M", [(256, 512, 9), (200, 1024, 16), (1000, 4096, 16), (600, 11008, 12),
-                                    (4101, 2048, 13)])
-def test_gemm_decode_two_token_tiles(fp4, oracle_mod, N, K, M):
-    """Decode engine with 9..16 activation rows: two 8-token MMA tiles that
-    share each dequantized weight fragment (staged activations, and L2
-    reads where M*K is too large to stage)."""
+@pytest.mark.parametrize("M", [9, 16, 17, 31, 32, 33, 48, 64])
+@pytest.mark.parametrize("N,K", [(256, 512), (200, 1024), (1000, 4096)])
+def test_gemm_decode_token_tiles(fp4, oracle_mod, N, K, M):
+    """Decode engine token tiles of 16, 32 and 64 activation rows (MMA N),
+    rows beyond M zero-filled by the activation copies."""
     assert gemm_case(fp4, oracle_mod, 3 * N + M, N, K, M, engine=fp4.ENGINE_DECODE, rho=0.5) <= TOL
+
+
+@pytest.mark.parametrize("M", [1, 16, 40, 64])
+@pytest.mark.parametrize("ctas", [1, 2, 3, 5, 8, 13, 24])
+def test_gemm_decode_cta_counts(fp4, oracle_mod, ctas, M):
+    """Decode engine with a forced number of CTAs (the split-K argument):
+    3 row tiles x 8 chunks cut into 1..24 contiguous ranges, so tiles are
+    whole, split in two, or shared by several CTAs."""
+    assert gemm_case(fp4, oracle_mod, 17 + M, 300, 2048, M, engine=fp4.ENGINE_DECODE, splits=ctas,
+                     rho=2.5) <= TOL
+
+
+@pytest.mark.parametrize("ctas", [0, 7])
+def test_gemm_decode_deterministic(fp4, ctas):
+    """Pieces of a tile are added in CTA order by whichever CTA completes
+    the tile: repeated calls agree bit for bit."""
+    W, X = synth.random_case(79, 1000, 4096, 16)
+    res = fp4.quantize(dev_f32(W), 128, 1)
+    outs = [fp4.gemm(dev_bf16(X), res["packed"], res["scales"], 1, 128, engine=1, splits=ctas) for _ in range(4)]
+    assert all(torch.equal(outs[0].view(torch.int16), o.view(torch.int16)) for o in outs[1:])
 
 
 def test_gemm_decode_unaligned_scales(fp4, oracle_mod):
@@ -331,14 +382,16 @@ def test_gemm_engines_agree(fp4, oracle_mod):
 
 def wide_range_rows(seed, M, K):
     """Activation rows at magnitudes 2^-60 .. 2^60 (far outside the f16
-    range on both sides), a row of zeros, and a row alternating 2^20 and
-    2^-20 entries."""
+    range on both sides); a row alternating 2^20 and 2^-20 entries (row 1,
+    or the only row); with three or more rows, a row of zeros (row 0)."""
     rng = np.random.default_rng(seed)
     x = rng.standard_normal((M, K), dtype=np.float32)
     x *= np.exp2(rng.integers(-60, 61, M).astype(np.float32))[:, None]
-    x[0] = 0.0
-    x[1, 0::2] *= np.float32(2.0 ** 20)
-    x[1, 1::2] *= np.float32(2.0 ** -20)
+    if M >= 3:
+        x[0] = 0.0
+    alt = 1 if M >= 2 else 0
+    x[alt, 0::2] *= np.float32(2.0 ** 20)
+    x[alt, 1::2] *= np.float32(2.0 ** -20)
     return synth.to_bf16_bits(x)
 
 
@@ -390,6 +443,25 @@ def test_gemm_f16_row_lengths(fp4, oracle_mod, K):
     assert row_rel_err(Y, Yref) <= TOL
 
 
+@pytest.mark.parametrize("M", [1, 2, 8, 9, 12, 16, 33, 64])
+@pytest.mark.parametrize("N,K,fmt", [(256, 1024, 1), (200, 2048, 1), (300, 512, 0), (136, 768, 2)])
+def test_gemm_decode_wide_range(fp4, oracle_mod, M, N, K, fmt):
+    """Decode engine on activation rows 2^120 apart in magnitude (far outside
+    the f16 range on both sides), a zero row and a row alternating 2^20 and
+    2^-20: each row meets the bound against its own magnitude.  E2M1 scales
+    each activation row by a power of two into the f16 range (prepared once
+    per call) and undoes it in fp32; the other formats multiply in bf16."""
+    W, _ = synth.random_case(60 + M + N, N, K, 1)
+    X = wide_range_rows(61 + M, M, K)
+    res = fp4.quantize(dev_f32(W), 128, fmt)
+    Yref = oracle_mod.gemm(X, res["packed"].cpu().numpy(), res["scales"].cpu().numpy(), fmt, 128, 0.5)
+    xs = torch.tensor([0.5], dtype=torch.float32, device="cuda")
+    for ctas in (0, 1, 3):
+        Y = fp4.gemm(dev_bf16(X), res["packed"], res["scales"], fmt, 128, x_scale=xs, engine=fp4.ENGINE_DECODE,
+                     splits=ctas)
+        assert row_rel_err(Y, Yref) <= TOL, ctas
+
+
 def test_gemm_empty_and_k0(fp4):
     packed = torch.zeros((16, 0), dtype=torch.uint8, device="cuda")
     scales = torch.zeros((16, 0), dtype=torch.float16, device="cuda")
@@ -405,19 +477,22 @@ def test_gemm_empty_and_k0(fp4):
 
 # ---------------------------------------------------------- full-size workloads
 
-def sampled_check(fp4, oracle_mod, Xbits, packed, scales, fmt, group, Y, rho=1.0, count=384, seed=0):
+def sampled_check(fp4, oracle_mod, Xbits, packed, scales, fmt, group, Y, rho=1.0, rows=4, seed=0):
+    """Whole rows of a full-size output against the oracle, element by
+    element: rows 0 and M-1 and rows-2 random ones, every one of their N
+    outputs.  The denominator is the oracle's own max|Y_ref| over those rows
+    (at most the max over the whole output, so the check is never looser
+    than the bound), and every output of Y must be finite."""
     M, N = Y.shape
+    assert bool(torch.isfinite(Y.float()).all()), "non-finite GPU output"
     rng = np.random.default_rng(seed)
-    ms = rng.integers(0, M, count).astype(np.int32)
-    ns = rng.integers(0, N, count).astype(np.int32)
-    ms[:4] = [0, M - 1, 0, M - 1]
-    ns[:4] = [0, N - 1, N - 1, 0]
-    ref = oracle_mod.gemm_sampled(Xbits, packed, scales, fmt, group, ms, ns, rho)
-    got = Y.float().cpu().numpy().astype(np.float64)[ms, ns]
-    # the bound is relative to max|Y_ref| over the whole output; the GPU's own
-    # max|Y| stands in for it (within bf16 rounding of it)
-    denom = max(np.max(np.abs(ref)), float(Y.float().abs().max()))
-    return float(np.max(np.abs(got - ref)) / denom)
+    sel = sorted({0, M - 1} | set(rng.integers(0, M, max(rows - 2, 0)).tolist()))
+    ms = np.repeat(np.asarray(sel, np.int32), N)
+    ns = np.tile(np.arange(N, dtype=np.int32), len(sel))
+    ref = oracle_mod.gemm_sampled(Xbits, packed, scales, fmt, group, ms, ns, rho).reshape(len(sel), N)
+    got = Y.float().cpu().numpy().astype(np.float64)[sel]
+    denom = float(np.max(np.abs(ref)))
+    return float(np.max(np.abs(got - ref)) / (denom if denom > 0 else 1.0))
 
 
 def test_llama7b_decode_full(fp4, oracle_mod):
@@ -481,7 +556,7 @@ def test_llama13b_stack_layer_sample(fp4, oracle_mod):
         for M in (1, 4, 16, 64, 2048):
             Xb = synth.activations(rng, M, K)
             Y = fp4.gemm(dev_bf16(Xb), res["packed"], res["scales"], 1, 128)
-            assert sampled_check(fp4, oracle_mod, Xb, ref["packed"], ref["scales"], 1, 128, Y, count=128) <= TOL
+            assert sampled_check(fp4, oracle_mod, Xb, ref["packed"], ref["scales"], 1, 128, Y, rows=3) <= TOL
 
 
 # -------------------------------------------------------- failure detection

@@ -228,9 +228,9 @@ def gemm(X, packed, scales, fmt=E2M1, group=128, x_scale=None, out=None, engine=
     """Y = bf16(x_scale * X . dequant(W)^T).  X: [M][K] bf16 CUDA tensor.
 
     ``workspace`` defaults to a per-device buffer of fp4_gemm_workspace_size
-    bytes (the f16 activations of the 128-token tensor tile, M > 64); a
-    smaller one makes that tile run in bf16.  ``engine``/``splits`` force an
-    engine or a split-K count (0: automatic)."""
+    bytes (the activations prepared once per call); a smaller one makes the
+    kernels convert the activations themselves.  ``engine``/``splits`` force
+    an engine or a split-K count (0: automatic)."""
     M, K = X.shape
     N = packed.shape[0]
     assert packed.shape[1] * 2 == K

@@ -24,11 +24,14 @@ cudaError_t launch_calibrate(const uint16_t* X, int M, int K, int8_t* shift, flo
 cudaError_t launch_apply(const uint16_t* X, int M, int K, const int8_t* shift, const float* rho, uint16_t* Xt,
                          cudaStream_t st);
 cudaError_t launch_gemm_decode(const uint16_t* X, const uint8_t* packed, const void* scales, int sdt,
-                               const FmtTable& t, int fmt, int M, int N, int K, int group, const float* x_scale,
-                               uint16_t* Y, int* status, unsigned long long timeout_ns, cudaStream_t st);
+                               const FmtTable& t, int M, int N, int K, int group, const float* x_scale, uint16_t* Y,
+                               cudaStream_t st);
+int decode_max_m_lut();
+cudaError_t launch_gemm_ts(const uint16_t* X, void* ws, size_t ws_bytes, const uint8_t* packed, const void* scales,
+                           int sdt, int fmt, int M, int N, int K, const float* x_scale, uint16_t* Y, int ctas,
+                           int* status, unsigned long long timeout_ns, cudaStream_t st);
+size_t ts_ws_bytes(int M, int N, int K);
 size_t tc_ws_bytes(int M, int N, int K);
-int decode_max_m(int K, int group);
-bool decode_preferred(int M, int N, int K, int group);
 cudaError_t launch_gemm_tc(const uint16_t* X, const uint8_t* packed, const void* scales, int sdt, const FmtTable& t,
                            bool e2m1, int M, int N, int K, int group, const float* x_scale, uint16_t* Y, void* ws,
                            size_t ws_bytes, int splits, int* status, unsigned long long timeout_ns,
@@ -46,8 +49,12 @@ __device__ int g_fp4_status;
 
 namespace {
 
-constexpr int kDecodeMaxM = 8;
+// Largest M of the decode engine: the tensor-memory engine at group 128,
+// the per-lane-LUT kernel at groups 32 and 64.
+constexpr int kDecodeMaxM128 = 64;
 constexpr int kMaxDevices = 64;
+
+int decode_max_m(int group) { return group == 128 ? kDecodeMaxM128 : decode_max_m_lut(); }
 long long g_timeout_us = 2000000;
 
 // Value of magnitude index i (code & 7) of the format with e exponent and m
@@ -278,7 +285,7 @@ fp4_status fp4_preshift_apply(const uint16_t* X, int M, int K, const int8_t* shi
 
 size_t fp4_gemm_workspace_size(int M, int N, int K) {
     if (M <= 0 || N <= 0 || K <= 0) return 0;
-    if (M <= kDecodeMaxM) return 0;
+    if (M <= kDecodeMaxM128) return ts_ws_bytes(M, N, K);
     return tc_ws_bytes(M, N, K);
 }
 
@@ -300,15 +307,24 @@ fp4_status fp4_gemm_ex(const uint16_t* X, const uint8_t* packed, const void* sca
     if (!X) return FP4_ERR_INVALID_ARG;
     if (!aligned(X, 16)) return FP4_ERR_MISALIGNED;
     if ((const void*)Y == (const void*)X || (const void*)Y == (const void*)packed) return FP4_ERR_INVALID_ARG;
-    if (engine == FP4_ENGINE_AUTO) engine = fp4_gemm_engine_for(M, N, K, group);
-    if (engine == FP4_ENGINE_DECODE && M > decode_max_m(K, group)) return FP4_ERR_UNSUPPORTED_SHAPE;
+    const bool auto_engine = engine == FP4_ENGINE_AUTO;
+    if (auto_engine) engine = fp4_gemm_engine_for(M, N, K, group);
+    if (engine == FP4_ENGINE_DECODE && M > decode_max_m(group)) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if (engine == FP4_ENGINE_DECODE && group == 128 && (!workspace || ws_bytes < ts_ws_bytes(M, N, K))) {
+        // the decode engine prepares the activations in the workspace; without
+        // one the automatic choice takes the tensor engine
+        if (!auto_engine) return FP4_ERR_WORKSPACE;
+        engine = FP4_ENGINE_TENSOR;
+    }
     const FmtTable& t = tables().f[fmt];
     int* st = status_ptr();
     if (!st) return FP4_ERR_CUDA;
     const unsigned long long to_ns = (unsigned long long)g_timeout_us * 1000ull;
     if (engine == FP4_ENGINE_DECODE) {
-        return cuda_status(launch_gemm_decode(X, packed, scales, (int)sdt, t, (int)fmt, M, N, K, group, x_scale, Y,
-                                              st, to_ns, stream));
+        if (group == 128)
+            return cuda_status(launch_gemm_ts(X, workspace, ws_bytes, packed, scales, (int)sdt, (int)fmt, M, N, K,
+                                              x_scale, Y, splits, st, to_ns, stream));
+        return cuda_status(launch_gemm_decode(X, packed, scales, (int)sdt, t, M, N, K, group, x_scale, Y, stream));
     }
     return cuda_status(launch_gemm_tc(X, packed, scales, (int)sdt, t, fmt == FP4_E2M1, M, N, K, group, x_scale, Y,
                                       workspace, ws_bytes, splits, st, to_ns, stream));
@@ -317,7 +333,7 @@ fp4_status fp4_gemm_ex(const uint16_t* X, const uint8_t* packed, const void* sca
 fp4_engine fp4_gemm_engine_for(int M, int N, int K, int group) {
     if (M <= 0 || N <= 0 || K <= 0) return FP4_ENGINE_AUTO;
     if (group != 32 && group != 64 && group != 128) return FP4_ENGINE_AUTO;
-    return decode_preferred(M, N, K, group) ? FP4_ENGINE_DECODE : FP4_ENGINE_TENSOR;
+    return M <= decode_max_m(group) ? FP4_ENGINE_DECODE : FP4_ENGINE_TENSOR;
 }
 
 fp4_status fp4_gemm(const uint16_t* X, const uint8_t* packed, const void* scales, fp4_scale_dtype sdt,

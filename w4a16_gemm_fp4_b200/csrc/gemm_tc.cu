@@ -424,9 +424,12 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
             const float s = s_next;
             if (f + 1 < kr.nfrag)
                 s_next = nvalid ? load_scale(p.scales, p.sdt, (size_t)n * G + kr.gfirst + f + 1) : 0.f;
-            if (ok && !mbar_wait(&gfull[b], (uint32_t)(f / C::NACC) & 1u, to)) {
+            // the warp decides together whether the wait gave up: the TMEM
+            // loads below are warp-collective (.sync.aligned)
+            if (!__all_sync(0xffffffffu, mbar_wait(&gfull[b], (uint32_t)(f / C::NACC) & 1u, to))) {
                 raise_status(p.status, kStatusTimeout);
                 ok = false;
+                break;
             }
             tc_fence_after();
 #pragma unroll
@@ -440,7 +443,6 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&gempty[b]);
-            if (!ok) break;
         }
         if (p.splits == 1) {
             const float rho = p.x_scale ? *p.x_scale : 1.f;
@@ -751,7 +753,9 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
             const int s = i % C::STG;
             const float sc = s_next;
             if (i + 1 < nkb) s_next = nvalid ? load_scale(p.scales, p.sdt, (size_t)n * G + kb0 + i + 1) : 0.f;
-            if (!mbar_wait(&kdone[s], (uint32_t)(i / C::STG) & 1u, to)) {
+            // the warp decides together whether the wait gave up: the TMEM
+            // loads below are warp-collective (.sync.aligned)
+            if (!__all_sync(0xffffffffu, mbar_wait(&kdone[s], (uint32_t)(i / C::STG) & 1u, to))) {
                 raise_status(p.status, kStatusTimeout);
                 ok = false;
                 break;
@@ -875,6 +879,22 @@ bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, int elem_bytes, const v
     return r == CUDA_SUCCESS;
 }
 
+// A 3-D view {inner, mid, outer} with byte strides {mid_stride, outer_stride},
+// no swizzle (used for L2 prefetches of several consecutive segments per row).
+bool encode_3d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t mid,
+               uint64_t outer, uint64_t mid_stride, uint64_t outer_stride, uint32_t box_inner, uint32_t box_mid,
+               uint32_t box_outer) {
+    EncodeTiledFn fn = get_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {inner, mid, outer};
+    cuuint64_t strides[2] = {mid_stride, outer_stride};
+    cuuint32_t box[3] = {box_inner, box_mid, box_outer};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 int tc_token_tile(int M) {
     if (M <= 32) return 32;
     if (M <= 64) return 64;
@@ -963,13 +983,19 @@ __device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4 v, float sc) {
 
 template <int R>
 __global__ void __launch_bounds__(256) x_rows_to_f16_kernel(const uint16_t* __restrict__ X, int K,
-                                                            uint16_t* __restrict__ Xh, float* __restrict__ xrow) {
+                                                            uint16_t* __restrict__ Xh, float* __restrict__ xrow,
+                                                            int* zero, int nzero) {
     __shared__ uint32_t wmax[8];
     const int m = blockIdx.x, nv = K >> 3;
     const uint4* src = reinterpret_cast<const uint4*>(X + (size_t)m * K);
     uint4* dst = reinterpret_cast<uint4*>(Xh + (size_t)m * K);
-    pdl_wait();  // X may come from the previous kernel in the stream
+    // the GEMM that follows only sets up (and starts its weights towards L2)
+    // before its own dependency wait, so it may be launched right away
     pdl_launch_dependents();
+    pdl_wait();  // X may come from the previous kernel in the stream
+    // the decode engine's tile counters start at zero
+    if (zero && m == 0)
+        for (int i = threadIdx.x; i < nzero; i += 256) zero[i] = 0;
     uint32_t mx2 = 0;  // per-half maxima of the finite magnitudes (bf16 bits order like the values)
     uint4 v[R > 0 ? R : 1];
     if constexpr (R > 0) {
@@ -1013,11 +1039,12 @@ __global__ void __launch_bounds__(256) x_rows_to_f16_kernel(const uint16_t* __re
 }
 
 // Bytes of the f16 activations (16-byte aligned rows) and their row factors.
-static size_t xh_bytes(int M, int K) { return ((size_t)M * K * 2 + 255) & ~(size_t)255; }
+size_t xh_bytes(int M, int K) { return ((size_t)M * K * 2 + 255) & ~(size_t)255; }
 
 size_t tc_f16_ws_bytes(int M, int K) { return xh_bytes(M, K) + (size_t)M * 4; }
 
-static cudaError_t launch_x_rows_to_f16(const uint16_t* X, int M, int K, uint16_t* Xh, float* xrow, cudaStream_t st) {
+cudaError_t launch_x_rows_to_f16(const uint16_t* X, int M, int K, uint16_t* Xh, float* xrow, int* zero, int nzero,
+                                 cudaStream_t st) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)M, 1, 1);
     cfg.blockDim = dim3(256, 1, 1);
@@ -1029,11 +1056,11 @@ static cudaError_t launch_x_rows_to_f16(const uint16_t* X, int M, int K, uint16_
     cfg.numAttrs = 1;
     const int nv = K / 8;
     cudaError_t e;
-    if (nv <= 256) e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<1>, X, K, Xh, xrow);
-    else if (nv <= 512) e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<2>, X, K, Xh, xrow);
-    else if (nv <= 1024) e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<4>, X, K, Xh, xrow);
-    else if (nv <= 2048) e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<8>, X, K, Xh, xrow);
-    else e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<0>, X, K, Xh, xrow);
+    if (nv <= 256) e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<1>, X, K, Xh, xrow, zero, nzero);
+    else if (nv <= 512) e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<2>, X, K, Xh, xrow, zero, nzero);
+    else if (nv <= 1024) e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<4>, X, K, Xh, xrow, zero, nzero);
+    else if (nv <= 2048) e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<8>, X, K, Xh, xrow, zero, nzero);
+    else e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<0>, X, K, Xh, xrow, zero, nzero);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -1124,7 +1151,7 @@ cudaError_t launch_gemm_tc(const uint16_t* X, const uint8_t* packed, const void*
         p.status = status;
         p.timeout_ns = timeout_ns;
         if (f16) {
-            cudaError_t e = launch_x_rows_to_f16(X, M, K, Xh, xrow, st);
+            cudaError_t e = launch_x_rows_to_f16(X, M, K, Xh, xrow, nullptr, 0, st);
             if (e != cudaSuccess) return e;
             return launch_tcg_bt<128, true>(mx, mw, p, st);
         }
