@@ -187,29 +187,34 @@ FP4_API fp4_status fp4_preshift_calibrate_noalloc(const uint16_t *X, int M, int 
  *   x_scale  device float (rho from fp4_preshift_calibrate) or NULL for 1.
  *   Y        [M][N] bf16 out; must not alias the inputs.
  *   workspace 16-byte aligned, not overlapping the other buffers, of
- *            fp4_gemm_workspace_size() bytes.  It holds the activations
- *            prepared once per call (f16 for E2M1, bf16 otherwise, paired
- *            in the order the MMA operands take them) and, for the decode
- *            engine, one partial tile per CTA piece plus one counter per
- *            128-row tile.  E2M1 rows are scaled by a power of two that
- *            brings their largest magnitude into [2^14, 2^15) (exact;
+ *            fp4_gemm_workspace_size() bytes, ZERO-FILLED ONCE before its
+ *            first use (e.g. cudaMemsetAsync).  Its first 64 KB hold the
+ *            decode engine's per-tile counters, which every call leaves at
+ *            zero again (a call that set FP4_DEV_WAIT_TIMEOUT may not: zero
+ *            the workspace again after that error); the rest holds, per
+ *            engine, partial tiles of split tiles and activations prepared
+ *            once per call.  The tensor engine's E2M1 path stores the
+ *            activations there in f16, each row scaled by a power of two
+ *            that brings its largest magnitude into [2^14, 2^15) (exact;
  *            elements more than 2^31 below the row maximum round to the f16
- *            subnormal grid) and the factor is undone in fp32 in the
- *            epilogue, so every bf16 activation is accepted.  With the
- *            automatic engine a workspace that is too small (or NULL)
- *            falls back to the tensor engine's bf16 path.
+ *            subnormal grid), the factor undone in fp32 in the epilogue;
+ *            the decode engine does the same per 128- or 256-element slice
+ *            in shared memory.  Every bf16 activation is accepted.  With the
+ *            automatic engine a workspace that is too small (or NULL) falls
+ *            back to the tensor engine's bf16 path.
  * Engines (fp4_gemm_engine_for reports the choice): at group 128 M <= 64,
  * and at groups 32/64 M <= 8, use the decode engine; larger M uses the
  * tensor engine (TMA-staged tiles dequantized in shared memory, tcgen05
  * MMAs into tensor memory, one group per pipeline stage).  The group-128
  * decode engine runs one persistent CTA per SM over an even split of all
- * (128-row tile, 2-group chunk) units: TMA streams the codes, dequantize
- * warps write the exact code values into tensor memory as the MMA's A
- * operand, tcgen05 MMAs multiply them by the activations, and each group's
- * scale is applied in fp32 as the accumulator is folded; a tile split
- * between CTAs is summed by the CTA that completes it, in CTA order, so
- * the result does not depend on timing.  Groups 32/64 use warp-level MMAs
- * over a lookup-table dequantization (no workspace).
+ * (row tile, 16 KB code chunk) units, streamed by TMA; a tile split between
+ * CTAs is summed by the CTA that completes it, in CTA order, so the result
+ * does not depend on timing.  For M <= 16 the codes convert in registers
+ * (hardware e2m1 -> f16 for E2M1, exact bf16 bit placement otherwise) into
+ * warp-level MMAs; for 16 < M <= 64 dequantize warps write them to tensor
+ * memory as the A operand of tcgen05 MMAs.  Each group scale is applied in
+ * fp32.  Groups 32/64 use warp-level MMAs over a lookup-table
+ * dequantization (no workspace).
  * Device status: FP4_DEV_WAIT_TIMEOUT, FP4_DEV_LAYOUT.
  * ---------------------------------------------------------------------- */
 FP4_API size_t fp4_gemm_workspace_size(int M, int N, int K);

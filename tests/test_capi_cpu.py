@@ -134,10 +134,20 @@ def test_workspace_sizes(L):
         chunks = tiles * ((K // 128) // (2 if (K // 128) % 2 == 0 else 1))
         ctas = min(148, chunks)
         return up(M * K * 2) + up(M * 4) + 2 * ctas * bt * 128 * 4 + up(tiles * 4)
-    assert L.fp4_gemm_workspace_size(1, 4096, 4096) == dec(1, 4096, 4096, 16)
-    assert L.fp4_gemm_workspace_size(33, 11008, 4096) == dec(33, 11008, 4096, 64)
-    assert L.fp4_gemm_workspace_size(64, 200, 384) == dec(64, 200, 384, 64)   # 2 tiles x 3 one-group chunks
-    assert L.fp4_gemm_workspace_size(65, 4096, 4096) == ((65 * 4096 * 2 + 255) // 256) * 256 + 65 * 4
-    assert L.fp4_gemm_workspace_size(2048, 4096, 4096) == 2048 * 4096 * 2 + 2048 * 4
+    def skinny(M, N, K):  # counter block + two M x TR partial tiles per CTA
+        G = K // 128
+        tr = 128 if G % 2 == 0 else 256     # tile rows: 2-group or 1-group chunks of 16 KB
+        tiles = (N + tr - 1) // tr
+        chunks = tiles * (G // (2 if G % 2 == 0 else 1))
+        ctas = min(148, chunks)
+        return 65536 + up(2 * ctas * M * tr * 4)
+    assert L.fp4_gemm_workspace_size(1, 4096, 4096) == skinny(1, 4096, 4096)
+    assert L.fp4_gemm_workspace_size(9, 200, 384) == skinny(9, 200, 384)
+    assert L.fp4_gemm_workspace_size(16, 11008, 4096) == skinny(16, 11008, 4096)
+    assert L.fp4_gemm_workspace_size(17, 4096, 4096) == 65536 + dec(17, 4096, 4096, 32)
+    assert L.fp4_gemm_workspace_size(33, 11008, 4096) == 65536 + dec(33, 11008, 4096, 64)
+    assert L.fp4_gemm_workspace_size(64, 200, 384) == 65536 + dec(64, 200, 384, 64)   # 2 tiles x 3 one-group chunks
+    assert L.fp4_gemm_workspace_size(65, 4096, 4096) == 65536 + ((65 * 4096 * 2 + 255) // 256) * 256 + 65 * 4
+    assert L.fp4_gemm_workspace_size(2048, 4096, 4096) == 65536 + 2048 * 4096 * 2 + 2048 * 4
     assert L.fp4_quantize_workspace_size(4096, 4096, 128, 1, 0) >= 8
     assert L.fp4_preshift_workspace_size(2048, 4096) >= 4096 * 4

@@ -31,6 +31,13 @@ cudaError_t launch_gemm_ts(const uint16_t* X, void* ws, size_t ws_bytes, const u
                            int sdt, int fmt, int M, int N, int K, const float* x_scale, uint16_t* Y, int ctas,
                            int* status, unsigned long long timeout_ns, cudaStream_t st);
 size_t ts_ws_bytes(int M, int N, int K);
+cudaError_t launch_gemm_skinny(const uint16_t* X, int* cnt, void* ws, size_t ws_bytes, const uint8_t* packed,
+                               const void* scales, int sdt, int fmt, int M, int N, int K, const float* x_scale,
+                               uint16_t* Y, int ctas, int* status, unsigned long long timeout_ns, cudaStream_t st);
+size_t skinny_ws_bytes(int M, int N, int K);
+int skinny_max_m();
+int skinny_max_tiles();
+int skinny_tiles(int N, int K);
 size_t tc_ws_bytes(int M, int N, int K);
 cudaError_t launch_gemm_tc(const uint16_t* X, const uint8_t* packed, const void* scales, int sdt, const FmtTable& t,
                            bool e2m1, int M, int N, int K, int group, const float* x_scale, uint16_t* Y, void* ws,
@@ -283,10 +290,25 @@ fp4_status fp4_preshift_apply(const uint16_t* X, int M, int K, const int8_t* shi
     return cuda_status(launch_apply(X, M, K, shift, rho, Xt, stream));
 }
 
+// Every GEMM workspace starts with a block of tile counters that is zero
+// between calls (the skinny kernel's split tiles); the engines' own data
+// follows it.
+constexpr size_t kCounterBlock = 65536;
+
+static bool skinny_fits(int M, int N, int K) {
+    return M <= skinny_max_m() && K % 128 == 0 && skinny_tiles(N, K) <= skinny_max_tiles();
+}
+
 size_t fp4_gemm_workspace_size(int M, int N, int K) {
     if (M <= 0 || N <= 0 || K <= 0) return 0;
-    if (M <= kDecodeMaxM128) return ts_ws_bytes(M, N, K);
-    return tc_ws_bytes(M, N, K);
+    if (skinny_fits(M, N, K)) return kCounterBlock + skinny_ws_bytes(M, N, K);
+    if (M <= kDecodeMaxM128) return kCounterBlock + ts_ws_bytes(M, N, K);
+    return kCounterBlock + tc_ws_bytes(M, N, K);
+}
+
+// Workspace bytes (counter block included) the group-128 decode engine needs.
+static size_t decode_ws_bytes(int M, int N, int K) {
+    return kCounterBlock + (skinny_fits(M, N, K) ? skinny_ws_bytes(M, N, K) : ts_ws_bytes(M, N, K));
 }
 
 fp4_status fp4_gemm_ex(const uint16_t* X, const uint8_t* packed, const void* scales, fp4_scale_dtype sdt,
@@ -310,24 +332,32 @@ fp4_status fp4_gemm_ex(const uint16_t* X, const uint8_t* packed, const void* sca
     const bool auto_engine = engine == FP4_ENGINE_AUTO;
     if (auto_engine) engine = fp4_gemm_engine_for(M, N, K, group);
     if (engine == FP4_ENGINE_DECODE && M > decode_max_m(group)) return FP4_ERR_UNSUPPORTED_SHAPE;
-    if (engine == FP4_ENGINE_DECODE && group == 128 && (!workspace || ws_bytes < ts_ws_bytes(M, N, K))) {
-        // the decode engine prepares the activations in the workspace; without
-        // one the automatic choice takes the tensor engine
+    if (engine == FP4_ENGINE_DECODE && group == 128 && (!workspace || ws_bytes < decode_ws_bytes(M, N, K))) {
+        // the group-128 decode engine keeps its tile counters and partial
+        // tiles in the workspace; without one the automatic choice takes the
+        // tensor engine
         if (!auto_engine) return FP4_ERR_WORKSPACE;
         engine = FP4_ENGINE_TENSOR;
     }
     const FmtTable& t = tables().f[fmt];
+    // the engines' part of the workspace follows the counter block
+    void* eng_ws = workspace && ws_bytes > kCounterBlock ? static_cast<uint8_t*>(workspace) + kCounterBlock : nullptr;
+    const size_t eng_bytes = eng_ws ? ws_bytes - kCounterBlock : 0;
     int* st = status_ptr();
     if (!st) return FP4_ERR_CUDA;
     const unsigned long long to_ns = (unsigned long long)g_timeout_us * 1000ull;
     if (engine == FP4_ENGINE_DECODE) {
+        if (group == 128 && skinny_fits(M, N, K))
+            return cuda_status(launch_gemm_skinny(X, static_cast<int*>(workspace), eng_ws, eng_bytes, packed, scales,
+                                                  (int)sdt, (int)fmt, M, N, K, x_scale, Y, splits, st, to_ns,
+                                                  stream));
         if (group == 128)
-            return cuda_status(launch_gemm_ts(X, workspace, ws_bytes, packed, scales, (int)sdt, (int)fmt, M, N, K,
+            return cuda_status(launch_gemm_ts(X, eng_ws, eng_bytes, packed, scales, (int)sdt, (int)fmt, M, N, K,
                                               x_scale, Y, splits, st, to_ns, stream));
         return cuda_status(launch_gemm_decode(X, packed, scales, (int)sdt, t, M, N, K, group, x_scale, Y, stream));
     }
     return cuda_status(launch_gemm_tc(X, packed, scales, (int)sdt, t, fmt == FP4_E2M1, M, N, K, group, x_scale, Y,
-                                      workspace, ws_bytes, splits, st, to_ns, stream));
+                                      eng_ws, eng_bytes, splits, st, to_ns, stream));
 }
 
 fp4_engine fp4_gemm_engine_for(int M, int N, int K, int group) {

@@ -149,6 +149,28 @@ __device__ __forceinline__ void dequant8_exact(uint32_t w, uint32_t p[4]) {
     asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(p[3]) : "r"(q3), "r"(SC));
 }
 
+// Per-half maxima of the finite magnitudes of a bf16x2 word folded into mx2
+// (bf16 bit patterns order like the magnitudes; inf and NaN are skipped).
+__device__ __forceinline__ uint32_t finite_mag_max2(uint32_t mx2, uint32_t w) {
+    const uint32_t a = w & 0x7fff7fffu;  // magnitudes; >= 0x7f80 is inf or NaN
+    return __vmaxu2(mx2, a & __vcmpltu2(a, 0x7f807f80u));
+}
+
+// Eight bf16 values times a power of two sc -> eight f16 (round to nearest).
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4 v, float sc) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t h[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float lo = __uint_as_float(w[j] << 16) * sc, hi = __uint_as_float(w[j] & 0xffff0000u) * sc;
+        asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h[j]) : "f"(hi), "f"(lo));
+    }
+    return make_uint4(h[0], h[1], h[2], h[3]);
+}
+
+// bf16 bit pattern of v, round to nearest even.
+__device__ __forceinline__ uint16_t bf16_bits(float v) { return __bfloat16_as_ushort(__float2bfloat16_rn(v)); }
+
 __device__ __forceinline__ float load_scale(const void* scales, int sdt, size_t idx) {
     if (sdt == FP4_SCALE_F16) return __half2float(__ldg(reinterpret_cast<const __half*>(scales) + idx));
     return __ldg(reinterpret_cast<const float*>(scales) + idx);
@@ -256,6 +278,28 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// cp.async of 4 bytes from global to shared (both 4-byte aligned); only the
+// first `src_bytes` (0 or 4) are read, the rest is zero-filled.
+__device__ __forceinline__ void cp_async4_zfill(uint32_t dst, const void* src, int src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+
+// Arrival on an mbarrier when all of this thread's earlier cp.async copies
+// have landed; counts as one of the phase's expected arrivals.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// 3D tiled TMA load global -> shared, completion on an mbarrier.  No multicast.
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int c0, int c1, int c2,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
         : "memory");
 }
 

@@ -965,22 +965,6 @@ static cudaError_t launch_tc_bt(const CUtensorMap& mx, const CUtensorMap& mw, co
 //
 // R = 16-byte vectors of the row each thread keeps in registers (one read
 // of X); R = 0 reads the row twice (any K).
-__device__ __forceinline__ uint32_t finite_mag_max2(uint32_t mx2, uint32_t w) {
-    const uint32_t a = w & 0x7fff7fffu;  // magnitudes; >= 0x7f80 is inf or NaN
-    return __vmaxu2(mx2, a & __vcmpltu2(a, 0x7f807f80u));
-}
-
-__device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4 v, float sc) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t h[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const float lo = __uint_as_float(w[j] << 16) * sc, hi = __uint_as_float(w[j] & 0xffff0000u) * sc;
-        asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h[j]) : "f"(hi), "f"(lo));
-    }
-    return make_uint4(h[0], h[1], h[2], h[3]);
-}
-
 template <int R>
 __global__ void __launch_bounds__(256) x_rows_to_f16_kernel(const uint16_t* __restrict__ X, int K,
                                                             uint16_t* __restrict__ Xh, float* __restrict__ xrow,

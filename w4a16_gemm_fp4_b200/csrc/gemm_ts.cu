@@ -499,7 +499,7 @@ cudaError_t launch_x_rows_to_f16(const uint16_t* X, int M, int K, uint16_t* Xh, 
 
 int ts_token_tile(int M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
 
-static int sm_count() {
+int device_sm_count() {
     static int sms[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
@@ -526,7 +526,7 @@ static TsLayout ts_layout(int M, int N, int K, int ctas) {
     const int BT = ts_token_tile(M), G = K / 128, CG = G % 2 == 0 ? 2 : 1;
     L.tiles = (N + 127) / 128;
     L.C = L.tiles * (G / CG);
-    L.P = ctas > 0 ? ctas : sm_count();
+    L.P = ctas > 0 ? ctas : device_sm_count();
     if (L.P > L.C) L.P = L.C;
     if (L.P < 1) L.P = 1;
     L.xh = 0;
