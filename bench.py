@@ -99,10 +99,11 @@ def recorded_traffic(key):
 
 
 def gemm_kernel_name(api, M, N, K):
-    """Kernel that serves an E2M1 group-128 GEMM of this shape."""
+    """Kernel that serves an E2M1 group-128 GEMM of this shape (automatic
+    engine): the skinny decode kernel, or the tensor engine's token tile."""
     if api.gemm_engine_for(M, N, K, GROUP) == api.ENGINE_DECODE:
-        return "gemm_decode_g128_kernel"
-    return "gemm_tcg_kernel<%d>" % (16 if M <= 16 else 32 if M <= 32 else 64 if M <= 64 else 128)
+        return "gemm_skinny_kernel"
+    return "gemm_tcg_kernel<%d>" % (32 if M <= 32 else 64 if M <= 64 else 128)
 
 
 def host_cores():
@@ -250,34 +251,29 @@ def run_ours(args, world, rank):
         wss[(i, M)] = torch.zeros(max(nb, 16), dtype=torch.uint8, device=dev) if nb else None
     stream = torch.cuda.Stream()
 
-    def sweep(c, events=None):
+    def sweep(c):
         for (i, M) in keys:
             packed, scales = mats[i]["reps"][c]
-            if events is not None:
-                events[(i, M)][0].record()
             api.gemm(mats[i]["X"][M], packed, scales, api.E2M1, GROUP, out=outs[(i, M)], workspace=wss[(i, M)])
-            if events is not None:
-                events[(i, M)][1].record()
 
     with torch.cuda.stream(stream):
         for s in range(args.warmup):          # eager warm-up (also loads modules, sets attributes)
             sweep(s % copies)
     torch.cuda.synchronize()
-    # one graph per weight copy holding the 12 launches back to back; a
-    # second set with an event pair around every launch gives the per-kernel
-    # durations (event nodes serialise the launches, so they are kept out of
-    # the graphs that time the step)
+    # one graph per weight copy holding the 12 launches back to back (the
+    # timed step); per-launch durations come from separate graphs that each
+    # hold one call, back to back over the weight copies (no event nodes
+    # between launches, so the launches overlap as they do in the step)
     graphs = [capture(torch, lambda c=c: sweep(c), stream) for c in range(copies)]
-    igraphs, gevents = [], []
-    for c in range(copies):
-        evs = {k: (torch.cuda.Event(enable_timing=True, external=True),
-                   torch.cuda.Event(enable_timing=True, external=True)) for k in keys}
-        igraphs.append(capture(torch, lambda c=c, evs=evs: sweep(c, evs), stream))
-        gevents.append(evs)
+
+    def one_call(key, c):
+        i, M = key
+        packed, scales = mats[i]["reps"][c]
+        api.gemm(mats[i]["X"][M], packed, scales, api.E2M1, GROUP, out=outs[key], workspace=wss[key])
+    call_graphs = {k: capture(torch, lambda k=k: [one_call(k, c) for c in range(copies)], stream) for k in keys}
     with torch.cuda.stream(stream):
         for s in range(args.warmup):
             graphs[s % copies].replay()
-            igraphs[s % copies].replay()
     torch.cuda.synchronize()
     api.device_status(clear=True)
 
@@ -306,23 +302,28 @@ def run_ours(args, world, rank):
     barrier(world)
     clk = clocks.stop()
     ms = max_over_ranks(world, t0.elapsed_time(t1))
-    # per-launch durations over a second timed region of instrumented replays
-    per_sum = {k: 0.0 for k in keys}
-    reps = max(copies, min(args.steps, 200) // copies * copies)
+    # per-launch durations: each call's graph replayed back to back
+    per = {}
+    reps = max(3, min(40, args.steps // 50))
     with torch.cuda.stream(stream):
-        for s in range(reps):
-            igraphs[s % copies].replay()
-            if s % copies == copies - 1:
-                stream.synchronize()
-                for k in keys:
-                    per_sum[k] += sum(ev[k][0].elapsed_time(ev[k][1]) for ev in gevents)
+        for k in keys:
+            call_graphs[k].replay()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(reps):
+                call_graphs[k].replay()
+            b.record()
+            b.synchronize()
+            per[k] = a.elapsed_time(b) / (reps * copies)
     torch.cuda.synchronize()
-    per = {k: v / reps for k, v in per_sum.items()}
+    del call_graphs
     st = api.device_status(clear=True)
     if st:
         raise RuntimeError("device status %#x during the timed region" % st)
 
     value = whole_job_gbs(world, step_weight_bytes(), args.steps, ms)
+    per_sum_ms = sum(per.values())
 
     groups = {}
     for (i, M), t in per.items():
@@ -363,6 +364,7 @@ def run_ours(args, world, rank):
                 parts["llama13b_stack"] = {"error": "%s: %s" % (type(exc).__name__, exc)}
     return {
         "value": value, "ms_per_step": ms / args.steps, "roofline": roofline, "clocks": clk, "e2e": e2e,
+        "per_launch_sum_ms": per_sum_ms,
         "gpu_launches": len(keys) * args.steps, "per_m": per_m, "parts": parts, "copies": copies,
         "copy_bytes": per_copy * copies, "l2_bytes": l2,
     }
@@ -476,13 +478,34 @@ def run_parts(api, torch, peaks, dev, stream):
     ms_pro = time_graph(torch, lambda: api.preshift_apply(X, shift, rho, out=Xt), stream, 20)
     out["preshift_apply"] = {"ms": round(ms_pro, 4), "gbs": round(2 * 2 * X.numel() / (ms_pro * 1e-3) / 1e9, 1)}
     del X, Xt, qs, ys, ws_cal
-    # format / bias search on 5120x5120 Student-t weights
-    W = torch.from_numpy(synth.student_t_weights(np.random.default_rng(3), 5120, 5120)).cuda()
-    o = api.quantize(W, GROUP, api.AUTO, True)
-    ms = time_graph(torch, lambda: api.quantize_into(W, o["packed"], o["scales"], o["choice"], GROUP, api.AUTO,
-                                                     True), stream, 5, warm=1)
-    out["search"] = {"workload": "5120x5120 Student-t(5)*0.015, 3 formats x 8 bias candidates + pack",
-                     "ms": round(ms, 3), "candidate_evals_per_s": round(24 * W.numel() / (ms * 1e-3), 0)}
+    # LLaMA-13B search workload: the per-tensor format/bias search (3 formats
+    # x 8 bias candidates, then the pack) on each Student-t matrix, then the
+    # W4A16 GEMM at M = 512 on the searched weights
+    case = synth.llama13b_search()
+    X = torch.from_numpy(case["X"].view(np.int16)).cuda().view(torch.bfloat16)
+    out["search"] = {}
+    out["gemm_m512"] = {}
+    for W_np in case["W"]:
+        N, K = W_np.shape
+        W = torch.from_numpy(W_np).cuda()
+        o = api.quantize(W, GROUP, api.AUTO, True)
+        ms = time_graph(torch, lambda: api.quantize_into(W, o["packed"], o["scales"], o["choice"], GROUP,
+                                                         api.AUTO, True), stream, 5, warm=1)
+        fmt = int(o["choice"][0].item())
+        out["search"]["%dx%d" % (N, K)] = {
+            "workload": "%dx%d Student-t(5)*0.015, 3 formats x 8 bias candidates + group-128 pack" % (N, K),
+            "ms": round(ms, 3), "candidate_evals_per_s": round(24 * W.numel() / (ms * 1e-3), 0),
+            "format_chosen": fmt}
+        del W
+        Y = torch.empty((X.shape[0], N), dtype=torch.bfloat16, device=dev)
+        ms = time_graph(torch, lambda: api.gemm(X, o["packed"], o["scales"], fmt, GROUP, out=Y), stream, 20)
+        tf = 2.0 * X.shape[0] * N * K / (ms * 1e-3) / 1e12
+        out["gemm_m512"]["%dx%d" % (N, K)] = {
+            "workload": "X bf16 512x5120 ~ N(0,1) . searched %dx%d weights (format %d, g128, fp16 scales)" % (
+                N, K, fmt),
+            "ms": round(ms, 4), "tflops": round(tf, 1), "frac": round(tf / peaks["bf16_tflops"], 4),
+            "frac_of_spec": round(tf / SPEC_BF16_TFLOPS, 4)}
+        del o, Y
     return out
 
 
@@ -535,34 +558,135 @@ def run_stack(api, torch, peaks, dev, stream, layers=40):
 
 # ----------------------------------------------------------- CPU oracle
 
-def oracle_sample(budget_s=12.0):
-    """Time the CPU oracle (fp64 GEMM on dequantized weights) over the
-    decode sweep, matrix by matrix and M by M, until the budget is spent.
-    Returns (weight GB/s in the step's unit, cores, description)."""
+SAMPLE_ROW_DIV = 16  # the CPU sample: every sweep call on the first 1/16 of each matrix's rows
+
+
+def oracle_sample(row_div=SAMPLE_ROW_DIV, threads=None):
+    """Time the CPU oracle (fp64 GEMM on dequantized weights) on a bounded
+    sample of the decode sweep: all 12 calls (every M, every matrix), each
+    on the first N/row_div rows of its matrix.  The oracle's work is linear
+    in the row count, so the sample's time x row_div is the sweep's time.
+    Returns (weight GB/s of the sweep, threads used, description)."""
     import oracle
     from w4a16_gemm_fp4_b200 import synth
     oracle.build()
+    if threads is not None:
+        oracle.set_num_threads(threads)
     cores = oracle.num_threads()
     cases = synth.llama7b_decode()
-    quant = [oracle.quantize(c["W"], GROUP, oracle.E2M1) for c in cases]
-    done_bytes = 0
+    quant = [oracle.quantize(c["W"][: c["W"].shape[0] // row_div], GROUP, oracle.E2M1) for c in cases]
     t_total = 0.0
-    done = []
     for M in MS:
-        for (N, K), c, q in zip(SHAPES, cases, quant):
+        for c, q in zip(cases, quant):
             t0 = time.perf_counter()
             oracle.gemm(c["X"][M], q["packed"], q["scales"], oracle.E2M1, GROUP)
-            dt = time.perf_counter() - t0
-            t_total += dt
-            done_bytes += weight_bytes(N, K)
-            done.append("%dx%d@M=%d" % (N, K, M))
-            if t_total >= budget_s:
-                break
-        if t_total >= budget_s:
-            break
-    gbs = done_bytes / t_total / 1e9
-    return gbs, cores, "oracle fp64 GEMM on %d of 12 sweep calls (%s), %.1f s" % (len(done), ", ".join(done),
-                                                                                   t_total)
+            t_total += time.perf_counter() - t0
+    sweep_s = t_total * row_div
+    gbs = step_weight_bytes() / sweep_s / 1e9
+    return gbs, cores, ("oracle fp64 GEMM, all 12 sweep calls on the first 1/%d of each matrix's rows (%.2f s), "
+                        "scaled to the full sweep by the row count" % (row_div, t_total))
+
+
+def cpu_baselines():
+    """The oracle on all host cores and on one thread, same sample."""
+    import oracle
+    gbs, cores, desc = oracle_sample()
+    gbs1, _, desc1 = oracle_sample(threads=1)
+    oracle.set_num_threads(cores)
+    return {"value": round(gbs, 5), "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc,
+            "host_cores": host_cores(),
+            "single_thread": {"value": round(gbs1, 5), "unit": "GB/s", "cores": 1, "sample": desc1}}
+
+
+def cpu_configs(threads_list=(0, 1)):
+    """The oracle on the host cores for every configuration: configs 1-4 in
+    full (quantize/search/pack and GEMM, as the workloads define them) and
+    config 5 extrapolated from one matrix of each of its three shapes
+    (x 4, 2 and 1 per layer, x 40 layers; the M = 2048 prefill GEMM of that
+    sample is itself extrapolated from its first 64 rows, the oracle's work
+    being linear in M).  threads 0 = all host cores.  Returns a dict."""
+    import oracle
+    from w4a16_gemm_fp4_b200 import synth
+    oracle.build()
+    all_cores = oracle.num_threads()
+    out = {"host_cores": host_cores(), "runs": {}}
+
+    def t(fn):
+        t0 = time.perf_counter()
+        fn()
+        return time.perf_counter() - t0
+
+    for th in threads_list:
+        oracle.set_num_threads(th if th > 0 else all_cores)
+        r = {}
+        c1 = synth.tiny()
+        q = oracle.quantize(c1["W"], GROUP, oracle.E2M1, scale_dtype="f32")
+        r["cfg1_tiny"] = {"quantize_s": t(lambda: oracle.quantize(c1["W"], GROUP, oracle.E2M1, scale_dtype="f32")),
+                          "gemm_s": t(lambda: oracle.gemm(c1["X"], q["packed"], q["scales"], oracle.E2M1, GROUP))}
+        c2 = synth.llama7b_decode()
+        qs = []
+        tq = 0.0
+        for c in c2:
+            t0 = time.perf_counter()
+            qs.append(oracle.quantize(c["W"], GROUP, oracle.E2M1))
+            tq += time.perf_counter() - t0
+        tg = sum(t(lambda c=c, qq=qq, M=M: oracle.gemm(c["X"][M], qq["packed"], qq["scales"], oracle.E2M1, GROUP))
+                 for M in MS for c, qq in zip(c2, qs))
+        r["cfg2_llama7b_decode"] = {"quantize_s": tq, "gemm_sweep_s": tg,
+                                    "weight_gbs": step_weight_bytes() / tg / 1e9}
+        del c2, qs
+        c3 = synth.llama7b_prefill()
+        tc = t(lambda: oracle.preshift_calibrate(c3["X"]))
+        shift, rho = oracle.preshift_calibrate(c3["X"])
+        ta = t(lambda: oracle.preshift_apply(c3["X"], shift, rho))
+        Xt = oracle.preshift_apply(c3["X"], shift, rho)
+        tq = 0.0
+        tg = 0.0
+        flops = 0.0
+        for W in c3["W"]:
+            t0 = time.perf_counter()
+            qq = oracle.quantize(W, GROUP, oracle.E2M1, shift=shift)
+            tq += time.perf_counter() - t0
+            tg += t(lambda: oracle.gemm(Xt, qq["packed"], qq["scales"], oracle.E2M1, GROUP, rho))
+            flops += 2.0 * Xt.shape[0] * W.shape[0] * W.shape[1]
+        r["cfg3_llama7b_prefill"] = {"calibrate_s": tc, "apply_s": ta, "quantize_s": tq, "gemm_s": tg,
+                                     "gflops": flops / tg / 1e9}
+        del c3, Xt
+        c4 = synth.llama13b_search()
+        ts = 0.0
+        tg = 0.0
+        flops = 0.0
+        for W in c4["W"]:
+            t0 = time.perf_counter()
+            qq = oracle.quantize(W, GROUP, oracle.AUTO, bias_search=True)
+            ts += time.perf_counter() - t0
+            tg += t(lambda: oracle.gemm(c4["X"], qq["packed"], qq["scales"], qq["choice"][0], GROUP))
+            flops += 2.0 * c4["X"].shape[0] * W.shape[0] * W.shape[1]
+        r["cfg4_llama13b_search"] = {"search_and_pack_s": ts, "gemm_m512_s": tg, "gflops": flops / tg / 1e9}
+        del c4
+        # config 5: one matrix of each shape, counts per layer 4, 2, 1
+        rng = np.random.default_rng(4)
+        shapes = ((5120, 5120, 4), (13824, 5120, 2), (5120, 13824, 1))
+        per_layer = {"quantize_s": 0.0}
+        for M in (1, 4, 16, 64, 2048):
+            per_layer["gemm_M%d_s" % M] = 0.0
+        for (N, K, cnt) in shapes:
+            W = synth.normal_weights(rng, N, K)
+            t0 = time.perf_counter()
+            qq = oracle.quantize(W, GROUP, oracle.E2M1)
+            per_layer["quantize_s"] += cnt * (time.perf_counter() - t0)
+            del W
+            for M in (1, 4, 16, 64, 2048):
+                Mt = min(M, 64)
+                X = synth.activations(rng, Mt, K)
+                dt = t(lambda: oracle.gemm(X, qq["packed"], qq["scales"], oracle.E2M1, GROUP))
+                per_layer["gemm_M%d_s" % M] += cnt * dt * (M / Mt)
+        r["cfg5_llama13b_stack_extrapolated"] = {k: v * 40 for k, v in per_layer.items()}
+        r["cfg5_llama13b_stack_extrapolated"]["note"] = (
+            "one matrix of each shape timed, x {4,2,1} per layer x 40 layers; M=2048 from its first 64 rows")
+        out["runs"]["threads_%d" % (th if th > 0 else all_cores)] = r
+    oracle.set_num_threads(all_cores)
+    return out
 
 
 def run_reference(args, world, rank):
@@ -570,23 +694,29 @@ def run_reference(args, world, rank):
         return None
     import oracle
     oracle.build()
-    # each step is one bounded sample of the sweep
+    # each step is one bounded sample of the sweep: the cpu_baseline sample
+    # (1/16 of the rows) when the run is short, fewer rows when many steps
+    # are asked for, so that the run ends within a few minutes
+    n = args.warmup + args.steps
+    row_div = SAMPLE_ROW_DIV
+    while n * 1.0 * SAMPLE_ROW_DIV / row_div > 40 and row_div < 1024:
+        row_div *= 2
     vals = []
     desc = ""
     cores = 1
-    for s in range(args.warmup + args.steps):
-        gbs, cores, desc = oracle_sample(budget_s=4.0)
+    for s in range(n):
+        gbs, cores, desc = oracle_sample(row_div=row_div)
         if s >= args.warmup:
             vals.append(gbs)
     v = statistics.median(vals)
-    return {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": args.gpus,
+    return {"impl": "reference", "metric": METRIC, "value": round(v, 5), "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_weight_bytes() / (v * 1e9) * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded PCG64 draws standing in for LLaMA-7B weights/activations)",
             "config": {"workload": "llama7b_decode: W 4096x4096, 11008x4096, 4096x11008 E2M1 g128 fp16 "
                                    "scales; M in {1,8,16,64}", "l2": "n/a (CPU)"},
-            "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc},
-            "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "cpu_baseline": {"value": round(v, 5), "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc},
+            "e2e": {"value": round(v, 5), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
 def profile_case(case):
@@ -620,43 +750,58 @@ def profile_case(case):
     print("profile case %s done, device status %d" % (case, st))
 
 
-TRAFFIC_CMD = ("ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none -k regex:gemm_ "
-               "-c 12 --csv --log-file traffic.csv python bench.py --steps 1 --warmup 3 --soak-s 0 --no-parts "
-               "--no-e2e --no-cpu-baseline")
+def traffic_cmds():
+    """One counter capture per kernel of the sweep (exact name, as many
+    launches as the first eager warm-up sweep has of it), each a single-pass
+    pair of DRAM byte counters."""
+    from w4a16_gemm_fp4_b200 import api
+    counts = {}
+    for M in MS:
+        for (N, K) in SHAPES:
+            base = gemm_kernel_name(api, M, N, K).split("<")[0]
+            counts[base] = counts.get(base, 0) + 1
+    return {base: ("ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none -k regex:%s "
+                   "-c %d --csv --log-file traffic_%s.csv python bench.py --steps 1 --warmup 3 --soak-s 0 "
+                   "--no-parts --no-e2e --no-cpu-baseline" % (base, n, base))
+            for base, n in sorted(counts.items())}
 
 
-def record_traffic(csv_path):
-    """The first 12 GEMM launches of this script are the first eager warm-up
-    sweep, in key order (for M in MS, for each matrix); ncu flushes the
-    caches before each profiled launch, so the bytes are cold-cache."""
+def record_traffic(csv_paths):
+    """profiles/traffic.json from the per-kernel captures of traffic_cmds():
+    each CSV lists its kernel's launches of the first eager warm-up sweep in
+    key order (for M in MS, for each matrix); ncu flushes the caches before
+    each profiled launch, so the bytes are cold-cache."""
     import csv
     from w4a16_gemm_fp4_b200 import api
-    vals = {}
-    order = []
-    with open(csv_path) as f:
-        lines = [l for l in f if l.startswith('"')]
-    for row in csv.DictReader(lines):
-        lid = int(row["ID"])
-        if lid not in vals:
-            vals[lid] = {"name": row["Kernel Name"]}
-            order.append(lid)
-        v = float(row["Metric Value"].replace(",", ""))
-        unit = row.get("Metric Unit", "byte")
-        scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}.get(unit, 1)
-        vals[lid][row["Metric Name"]] = v * scale
     keys = [(i, M) for M in MS for i in range(len(SHAPES))]
-    if len(order) < len(keys):
-        raise SystemExit("expected %d launches in %s, found %d" % (len(keys), csv_path, len(order)))
     out = {}
-    for (i, M), lid in zip(keys, order):
-        N, K = SHAPES[i]
-        kname = gemm_kernel_name(api, M, N, K)
-        assert kname.split("<")[0] in vals[lid]["name"], (kname, vals[lid]["name"])
-        d = vals[lid]
-        out["%s %dx%d M=%d" % (kname, N, K, M)] = {
-            "dram_bytes": int(d["dram__bytes_read.sum"] + d["dram__bytes_write.sum"]),
-            "algorithmic_bytes": weight_bytes(N, K) + M * K * 2 + M * N * 2}
-    doc = {"sources_sha": kernel_sources_sha(), "command": TRAFFIC_CMD, "launches": out}
+    for path in csv_paths.split(","):
+        vals, order = {}, []
+        with open(path) as f:
+            lines = [l for l in f if l.startswith('"')]
+        for row in csv.DictReader(lines):
+            lid = int(row["ID"])
+            if lid not in vals:
+                vals[lid] = {"name": row["Kernel Name"]}
+                order.append(lid)
+            v = float(row["Metric Value"].replace(",", ""))
+            scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}.get(row.get("Metric Unit", "byte"), 1)
+            vals[lid][row["Metric Name"]] = v * scale
+        if not order:
+            raise SystemExit("no launches in " + path)
+        base = vals[order[0]]["name"].split("<")[0].split("(")[0].strip()
+        mine = [k for k in keys if gemm_kernel_name(api, k[1], *SHAPES[k[0]]).split("<")[0] in base]
+        if len(order) < len(mine):
+            raise SystemExit("expected %d launches in %s, found %d" % (len(mine), path, len(order)))
+        for (i, M), lid in zip(mine, order):
+            N, K = SHAPES[i]
+            kname = gemm_kernel_name(api, M, N, K)
+            assert kname.split("<")[0] in vals[lid]["name"], (kname, vals[lid]["name"])
+            d = vals[lid]
+            out["%s %dx%d M=%d" % (kname, N, K, M)] = {
+                "dram_bytes": int(d["dram__bytes_read.sum"] + d["dram__bytes_write.sum"]),
+                "algorithmic_bytes": weight_bytes(N, K) + M * K * 2 + M * N * 2}
+    doc = {"sources_sha": kernel_sources_sha(), "commands": traffic_cmds(), "launches": out}
     path = os.path.join(ROOT, "profiles", "traffic.json")
     with open(path, "w") as f:
         json.dump(doc, f, indent=1)
@@ -678,12 +823,22 @@ def main():
     ap.add_argument("--profile-case", metavar="CASE",
                     help="run one case a few times and exit, for ncu captures: gemm:N:K:M (E2M1 g128 fp16 "
                          "scales, synthetic weights and activations) or quantize:N:K")
-    ap.add_argument("--record-traffic", metavar="CSV",
-                    help="write profiles/traffic.json from an ncu CSV of the first 12 GEMM launches "
-                         "(dram__bytes_read.sum, dram__bytes_write.sum) of this script, then exit")
+    ap.add_argument("--cpu-configs", action="store_true",
+                    help="time the CPU oracle on every configuration (1 thread and all cores), print JSON, exit")
+    ap.add_argument("--record-traffic", metavar="CSV[,CSV]",
+                    help="write profiles/traffic.json from the per-kernel ncu CSVs of traffic_cmds() "
+                         "(dram__bytes_read.sum, dram__bytes_write.sum), then exit")
+    ap.add_argument("--traffic-cmds", action="store_true", help="print the per-kernel traffic captures, exit")
     args = ap.parse_args()
     if args.record_traffic:
         record_traffic(args.record_traffic)
+        return
+    if args.traffic_cmds:
+        for cmd in traffic_cmds().values():
+            print(cmd)
+        return
+    if args.cpu_configs:
+        print(json.dumps(cpu_configs(), indent=1), flush=True)
         return
     if args.profile_case:
         profile_case(args.profile_case)
@@ -702,10 +857,7 @@ def main():
     world, rank, local = dist_setup(args)
     res = run_ours(args, world, rank)
     if rank == 0:
-        cpu = None
-        if not args.no_cpu_baseline:
-            gbs, cores, desc = oracle_sample()
-            cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc}
+        cpu = None if args.no_cpu_baseline else cpu_baselines()
         line = {
             "metric": METRIC, "value": round(res["value"], 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(res["ms_per_step"], 5), "higher_is_better": True,
@@ -717,7 +869,10 @@ def main():
                        "l2": "weights rotate over %d copies (%.0f MB) > 4x L2 (%d MB)" % (
                            res["copies"], res["copy_bytes"] / 1e6, res["l2_bytes"] // 2 ** 20)},
             "roofline": res["roofline"], "cpu_baseline": cpu, "e2e": res["e2e"], "gpu_launches": res["gpu_launches"],
-            "clocks": res["clocks"], "per_m": res["per_m"], "parts": res["parts"],
+            "clocks": res["clocks"], "per_m": res["per_m"],
+            "per_launch_sum_ms": round(res["per_launch_sum_ms"], 5),
+            "per_launch_sum_over_step": round(res["per_launch_sum_ms"] / res["ms_per_step"], 3),
+            "parts": res["parts"],
         }
         print(json.dumps(line), flush=True)
     if world > 1:
