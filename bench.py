@@ -98,11 +98,25 @@ def recorded_traffic(key):
     return e["dram_bytes"]
 
 
+def rowblk_fits(M, K):
+    """Whether the library's group-128 row-block decode kernel takes this
+    shape (its shared-memory plan: activations staged once per CTA, 16-row
+    block buffers of codes and scale rows, the cross-warp reduction area)."""
+    if K > 24576 or M > 16:
+        return False
+
+    def smem(nw, nbuf):
+        return nbuf * (16 * (K // 2) + 16 * (K // 128) * 4) + M * (2 * K + 64) + \
+            2 * nw * 32 * 4 * 4 * (2 if M > 8 else 1) + 128
+    return any(2 * (smem(8, nb) + 1024 + 128) <= 228 * 1024 or smem(16, nb) <= 226 * 1024 for nb in (2, 1))
+
+
 def gemm_kernel_name(api, M, N, K):
     """Kernel that serves an E2M1 group-128 GEMM of this shape (automatic
-    engine): the skinny decode kernel, or the tensor engine's token tile."""
+    engine): the row-block or streaming decode kernel, or the tensor
+    engine's token tile."""
     if api.gemm_engine_for(M, N, K, GROUP) == api.ENGINE_DECODE:
-        return "gemm_skinny_kernel"
+        return "gemm_rowblk_kernel" if rowblk_fits(M, K) else "gemm_skinny_kernel"
     return "gemm_tcg_kernel<%d>" % (32 if M <= 32 else 64 if M <= 64 else 128)
 
 

@@ -97,19 +97,41 @@ def test_gemm_argument_errors(L):
     assert g(N=0) == 0
 
 
+def rowblk_two_buffers(M, K):
+    """The group-128 row-block kernel's shared-memory plan (activations staged
+    once per CTA; 16-row block buffers of codes and f32 scale rows; the
+    cross-warp reduction area): True when it runs with two block buffers."""
+    if K > 24576 or M > 16:
+        return False
+    def smem(nw, nbuf):
+        return nbuf * (16 * (K // 2) + 16 * (K // 128) * 4) + M * (2 * K + 64) + \
+            2 * nw * 32 * 4 * 4 * (2 if M > 8 else 1) + 128
+    for nbuf in (2, 1):
+        if 2 * (smem(8, nbuf) + 1024 + 128) <= 228 * 1024 or smem(16, nbuf) <= 226 * 1024:
+            return nbuf == 2
+    return False
+
+
 def test_gemm_engine_choice(L):
-    """Automatic engine: at group 128 the decode (tensor-memory) engine for
-    M <= 64 at any K; at groups 32 and 64 the decode kernel for M <= 8; the
-    tensor engine otherwise."""
+    """Automatic engine: the decode engine for M <= 8 (group 128 at any K;
+    groups 32 and 64: the lookup-table kernel), and for 9 <= M <= 16 at
+    group 128 where the row-block kernel runs with two block buffers; the
+    tensor engine otherwise (it measures faster there)."""
     e = L.fp4_gemm_engine_for
     for K in (128, 4096, 11008, 24576, 40960):
-        for M in (1, 8, 12, 16, 17, 33, 64):
+        for M in (1, 4, 8):
             assert e(M, 4096, K, 128) == 1
-        assert e(65, 4096, K, 128) == 2 and e(2048, 11008, K, 128) == 2
+        for M in (9, 16):
+            assert e(M, 4096, K, 128) == (1 if rowblk_two_buffers(M, K) else 2), (M, K)
+        for M in (17, 64, 65):
+            assert e(M, 4096, K, 128) == 2
+        assert e(2048, 11008, K, 128) == 2
+    assert rowblk_two_buffers(12, 2048) and not rowblk_two_buffers(16, 4096)
     assert e(8, 64, 4096, 32) == 1 and e(8, 4096, 4096, 64) == 1
     assert e(9, 4096, 4096, 64) == 2 and e(9, 4096, 4096, 32) == 2
     assert e(0, 4096, 4096, 128) == 0 and e(4, 4096, 4096, 96) == 0
-    assert api.gemm_engine_for(64, 4096, 4096) == api.ENGINE_DECODE
+    assert api.gemm_engine_for(8, 4096, 4096) == api.ENGINE_DECODE
+    assert api.gemm_engine_for(16, 11008, 11008) == api.ENGINE_TENSOR
 
 
 def test_preshift_argument_errors(L):

@@ -234,27 +234,33 @@ def test_gemm_decode_engine(fp4, oracle_mod, M, N, K, group):
     assert gemm_case(fp4, oracle_mod, 7 * M + N, N, K, M, group=group, engine=fp4.ENGINE_DECODE) <= TOL
 
 
-@pytest.mark.parametrize("M", [4, 24, 64])
-@pytest.mark.parametrize("fmt,sdt", [(0, "f16"), (2, "f32"), (1, "f32"), (0, "f32"), (2, "f16")])
-def test_gemm_decode_formats(fp4, oracle_mod, fmt, sdt, M):
-    """Every format and scale type through the decode engine: E2M1 runs its
-    codes through the hardware f16 convert (activations prepared as scaled
-    f16 rows), E1M2 and E3M0 by bit placement to bf16 (activations prepared
-    as re-paired bf16 rows)."""
-    assert gemm_case(fp4, oracle_mod, 3 + M, 96, 256, M, fmt=fmt, sdt=sdt, engine=fp4.ENGINE_DECODE, rho=0.75) <= TOL
+@pytest.mark.parametrize("M,splits", [(4, 0), (4, 148), (13, 0), (13, 148), (24, 0), (64, 0)])
+@pytest.mark.parametrize("fmt,sdt", [(0, "f16"), (2, "f32"), (1, "f32"), (0, "f32"), (2, "f16"), (1, "f16")])
+def test_gemm_decode_formats(fp4, oracle_mod, fmt, sdt, M, splits):
+    """Every format and scale type through every decode kernel (M <= 16:
+    row-block with splits = 0, streaming with a CTA count; M > 16: the
+    tensor-memory kernel): E2M1 runs its codes through the hardware f16
+    convert (activations scaled into the f16 range by a power of two),
+    E1M2 and E3M0 by bit placement to bf16 (activations re-paired)."""
+    assert gemm_case(fp4, oracle_mod, 3 + M, 96, 256, M, fmt=fmt, sdt=sdt, engine=fp4.ENGINE_DECODE, splits=splits,
+                     rho=0.75) <= TOL
 
 
 def test_gemm_decode_needs_workspace(fp4, oracle_mod):
-    """The decode engine prepares the activations in the workspace: forced
-    without one it refuses (FP4_ERR_WORKSPACE, nothing launched); the
-    automatic choice then takes the tensor engine, which needs none."""
+    """The streaming decode kernels keep tile counters and partials in the
+    workspace: forced without one (a CTA count selects them) the call
+    refuses (FP4_ERR_WORKSPACE, nothing launched).  The row-block kernel
+    needs none, and the automatic choice runs it."""
     W, X = synth.random_case(12, 200, 512, 8)
     res = fp4.quantize(dev_f32(W), 128, 1)
     with pytest.raises(fp4.Fp4Error) as err:
-        fp4.gemm(dev_bf16(X), res["packed"], res["scales"], 1, 128, engine=fp4.ENGINE_DECODE, workspace=small_ws())
+        fp4.gemm(dev_bf16(X), res["packed"], res["scales"], 1, 128, engine=fp4.ENGINE_DECODE, splits=148,
+                 workspace=small_ws())
     assert err.value.code == 4
-    Y = fp4.gemm(dev_bf16(X), res["packed"], res["scales"], 1, 128, workspace=small_ws())
     Yref = oracle_mod.gemm(X, res["packed"].cpu().numpy(), res["scales"].cpu().numpy(), 1, 128)
+    Y = fp4.gemm(dev_bf16(X), res["packed"], res["scales"], 1, 128, engine=fp4.ENGINE_DECODE, workspace=small_ws())
+    assert rel_err(Y, Yref) <= TOL
+    Y = fp4.gemm(dev_bf16(X), res["packed"], res["scales"], 1, 128, workspace=small_ws())
     assert rel_err(Y, Yref) <= TOL
 
 
@@ -269,12 +275,15 @@ def test_gemm_decode_needs_workspace(fp4, oracle_mod):
     (600, 11008, 12),
     (128, 128, 5),      # a single chunk of one group
 ])
-def test_gemm_decode_block_schedule(fp4, oracle_mod, N, K, M):
-    """Decode engine, group 128: the code chunks of all row tiles split into
-    one contiguous range per CTA (whole tiles stored directly, pieces
-    reduced by the CTA that completes the tile), ragged row tiles, two- and
-    one-group chunks."""
-    assert gemm_case(fp4, oracle_mod, N + K, N, K, M, engine=fp4.ENGINE_DECODE, rho=1.5) <= TOL
+@pytest.mark.parametrize("splits", [0, 148])
+def test_gemm_decode_block_schedule(fp4, oracle_mod, N, K, M, splits):
+    """Decode engine, group 128.  splits = 148: the streaming kernel, whose
+    code chunks of all row tiles split into one contiguous range per CTA
+    (whole tiles stored directly, pieces reduced by the CTA that completes
+    the tile), ragged row tiles, two- and one-group chunks.  splits = 0: the
+    row-block kernel where the activations fit it (16-row blocks walked by
+    persistent CTAs, ragged last block), the streaming kernel elsewhere."""
+    assert gemm_case(fp4, oracle_mod, N + K, N, K, M, engine=fp4.ENGINE_DECODE, splits=splits, rho=1.5) <= TOL
 
 
 @pytest.mark.parametrize("M", [9, 16, 17, 31, 32, 33, 48, 64])

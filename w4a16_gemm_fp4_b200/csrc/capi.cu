@@ -38,6 +38,11 @@ size_t skinny_ws_bytes(int M, int N, int K);
 int skinny_max_m();
 int skinny_max_tiles();
 int skinny_tiles(int N, int K);
+cudaError_t launch_gemm_rowblk(const uint16_t* X, const uint8_t* packed, const void* scales, int sdt, int fmt,
+                               int M, int N, int K, const float* x_scale, uint16_t* Y, int* status,
+                               unsigned long long timeout_ns, cudaStream_t st);
+bool rowblk_fits(int M, int K);
+bool rowblk_preferred(int M, int K);
 size_t tc_ws_bytes(int M, int N, int K);
 cudaError_t launch_gemm_tc(const uint16_t* X, const uint8_t* packed, const void* scales, int sdt, const FmtTable& t,
                            bool e2m1, int M, int N, int K, int group, const float* x_scale, uint16_t* Y, void* ws,
@@ -58,7 +63,8 @@ namespace {
 
 // Largest M of the decode engine: the tensor-memory engine at group 128,
 // the per-lane-LUT kernel at groups 32 and 64.
-constexpr int kDecodeMaxM128 = 64;
+constexpr int kDecodeMaxM128 = 64;     // decode engine on request (group 128)
+constexpr int kAutoDecodeMaxM128 = 8;  // decode engine by default (group 128)
 constexpr int kMaxDevices = 64;
 
 int decode_max_m(int group) { return group == 128 ? kDecodeMaxM128 : decode_max_m_lut(); }
@@ -332,7 +338,13 @@ fp4_status fp4_gemm_ex(const uint16_t* X, const uint8_t* packed, const void* sca
     const bool auto_engine = engine == FP4_ENGINE_AUTO;
     if (auto_engine) engine = fp4_gemm_engine_for(M, N, K, group);
     if (engine == FP4_ENGINE_DECODE && M > decode_max_m(group)) return FP4_ERR_UNSUPPORTED_SHAPE;
-    if (engine == FP4_ENGINE_DECODE && group == 128 && (!workspace || ws_bytes < decode_ws_bytes(M, N, K))) {
+    // group 128, M <= 16: the row-block kernel (no workspace) unless a CTA
+    // count is asked for or the activations do not fit it; else the
+    // streaming kernels, which keep tile counters and partials in the
+    // workspace
+    const bool rowblk = engine == FP4_ENGINE_DECODE && group == 128 && splits == 0 && rowblk_fits(M, K);
+    if (engine == FP4_ENGINE_DECODE && group == 128 && !rowblk &&
+        (!workspace || ws_bytes < decode_ws_bytes(M, N, K))) {
         // the group-128 decode engine keeps its tile counters and partial
         // tiles in the workspace; without one the automatic choice takes the
         // tensor engine
@@ -347,6 +359,9 @@ fp4_status fp4_gemm_ex(const uint16_t* X, const uint8_t* packed, const void* sca
     if (!st) return FP4_ERR_CUDA;
     const unsigned long long to_ns = (unsigned long long)g_timeout_us * 1000ull;
     if (engine == FP4_ENGINE_DECODE) {
+        if (rowblk)
+            return cuda_status(launch_gemm_rowblk(X, packed, scales, (int)sdt, (int)fmt, M, N, K, x_scale, Y, st,
+                                                  to_ns, stream));
         if (group == 128 && skinny_fits(M, N, K))
             return cuda_status(launch_gemm_skinny(X, static_cast<int*>(workspace), eng_ws, eng_bytes, packed, scales,
                                                   (int)sdt, (int)fmt, M, N, K, x_scale, Y, splits, st, to_ns,
@@ -363,6 +378,13 @@ fp4_status fp4_gemm_ex(const uint16_t* X, const uint8_t* packed, const void* sca
 fp4_engine fp4_gemm_engine_for(int M, int N, int K, int group) {
     if (M <= 0 || N <= 0 || K <= 0) return FP4_ENGINE_AUTO;
     if (group != 32 && group != 64 && group != 128) return FP4_ENGINE_AUTO;
+    // group 128: the decode engine up to 8 tokens, and up to 16 where the
+    // row-block kernel runs with two block buffers; otherwise the tensor
+    // engine's small token tiles measure faster (the decode engine stays
+    // available on request up to 64 tokens)
+    if (group == 128)
+        return M <= kAutoDecodeMaxM128 || (M <= 16 && rowblk_preferred(M, K)) ? FP4_ENGINE_DECODE
+                                                                                : FP4_ENGINE_TENSOR;
     return M <= decode_max_m(group) ? FP4_ENGINE_DECODE : FP4_ENGINE_TENSOR;
 }
 

@@ -16,7 +16,7 @@
 //     previous kernel in the stream is finishing;
 //   * a scale warp copies the chunk's group scales into the slot as the
 //     slot is refilled (cp.async), so they land with the codes;
-//   * a converter warp rewrites the chunk's activations into the order the
+//   * converter warps rewrite the chunk's activations into the order the
 //     MMA fragments pair the codes (f16 with a per-chunk power-of-two token
 //     factor for E2M1, re-paired bf16 otherwise), so that every shared
 //     access of the consumers is conflict-free;
@@ -64,7 +64,8 @@ struct SkCfg {
     static constexpr int NS = (208 * 1024) / SLOT > 16 ? 16 : (208 * 1024) / SLOT;  // ring slots
     static constexpr int NCW = 16;                       // consumer warps: 16 rows x 1 group each
     static constexpr int RBLK = TR / 16;                 // row blocks of a chunk
-    static constexpr int W0 = 3;                         // first consumer warp
+    static constexpr int CW = NT == 1 ? 2 : 4;           // activation converter warps
+    static constexpr int W0 = 2 + CW;                    // first consumer warp
     static constexpr int THREADS = (W0 + NCW) * 32;
     static constexpr int RPL = TR / 32;                  // rows per scale-warp lane
     static constexpr int SD = 4;                         // chunks of scales in flight per scale-warp lane
@@ -132,7 +133,8 @@ __global__ void __launch_bounds__(SkCfg<NT, CG>::THREADS, 1)
     using C = SkCfg<NT, CG>;
     constexpr int TR = C::TR;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned base (offset arithmetic keeps the shared address space)
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* codes = smem;                                       // [NS][CBYTES], swizzled rows
     uint8_t* xraw = codes + C::NS * C::CBYTES;                   // [NS][NTOK][128 CG] bf16 as loaded
     uint8_t* xfrag = xraw + C::NS * C::XBYTES;                   // [NS][XBYTES] fragment order
@@ -143,6 +145,8 @@ __global__ void __launch_bounds__(SkCfg<NT, CG>::THREADS, 1)
     uint64_t* xland = ready + C::NS;
     uint64_t* empty = xland + C::NS;
     volatile int* reduce_flag = reinterpret_cast<volatile int*>(empty + C::NS);
+    const uint32_t codes_a = smem_u32(codes), xraw_a = smem_u32(xraw), xfrag_a = smem_u32(xfrag),
+                   scs_a = smem_u32(scs), xfs_a = smem_u32(xfs);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int c = blockIdx.x;
@@ -153,7 +157,7 @@ __global__ void __launch_bounds__(SkCfg<NT, CG>::THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::NS; ++s) {
-            mbar_init(&ready[s], 1 + 32 + 1);  // codes (with the byte count), 32 scale lanes, the converter
+            mbar_init(&ready[s], 1 + 32 + 1);  // codes (with the byte count), 32 scale lanes, a converter
             mbar_init(&xland[s], 1);
             mbar_init(&empty[s], C::NCW);
         }
@@ -186,7 +190,7 @@ __global__ void __launch_bounds__(SkCfg<NT, CG>::THREADS, 1)
             int j = pre;
             for (; j < nch; ++j) {
                 const int s = j % C::NS, jj = j0 + j;
-                if (!mbar_wait(&empty[s], ((uint32_t)(j / C::NS) & 1u) ^ 1u, to)) {
+                if (!mbar_wait_sleep(&empty[s], ((uint32_t)(j / C::NS) & 1u) ^ 1u, to)) {
                     raise_status(p.status, kStatusTimeout);
                     break;
                 }
@@ -197,8 +201,8 @@ __global__ void __launch_bounds__(SkCfg<NT, CG>::THREADS, 1)
             }
             // every copy issued must land before the CTA leaves
             for (int i = j - C::NS < 0 ? 0 : j - C::NS; i < j; ++i)
-                if (!mbar_wait(&xland[i % C::NS], (uint32_t)(i / C::NS) & 1u, to) ||
-                    !mbar_wait(&ready[i % C::NS], (uint32_t)(i / C::NS) & 1u, to)) {
+                if (!mbar_wait_sleep(&xland[i % C::NS], (uint32_t)(i / C::NS) & 1u, to) ||
+                    !mbar_wait_sleep(&ready[i % C::NS], (uint32_t)(i / C::NS) & 1u, to)) {
                     raise_status(p.status, kStatusTimeout);
                     break;
                 }
@@ -220,7 +224,7 @@ __global__ void __launch_bounds__(SkCfg<NT, CG>::THREADS, 1)
             bool ok = true;
             for (int j = 0; j < nch && ok; ++j) {
                 const int s = j % C::NS, jj = j0 + j;
-                if (j >= C::NS && !mbar_wait(&empty[s], ((uint32_t)(j / C::NS) & 1u) ^ 1u, to)) {
+                if (j >= C::NS && !mbar_wait_sleep(&empty[s], ((uint32_t)(j / C::NS) & 1u) ^ 1u, to)) {
                     raise_status(p.status, kStatusTimeout);
                     ok = false;
                     break;
@@ -257,7 +261,7 @@ __global__ void __launch_bounds__(SkCfg<NT, CG>::THREADS, 1)
                     const int j = jb + d;
                     if (j < nch && ok) {
                         const int s = j % C::NS;
-                        if (!mbar_wait(&empty[s], ((uint32_t)(j / C::NS) & 1u) ^ 1u, to)) {
+                        if (!mbar_wait_sleep(&empty[s], ((uint32_t)(j / C::NS) & 1u) ^ 1u, to)) {
                             raise_status(p.status, kStatusTimeout);
                             ok = false;
                         } else {
@@ -272,7 +276,7 @@ __global__ void __launch_bounds__(SkCfg<NT, CG>::THREADS, 1)
                 }
             }
         }
-    } else if (warp == 2) {
+    } else if (warp < C::W0) {
         // ------------------------------------------------ activation converter
         // The chunk's activations ([NTOK][128*CG] bf16 as loaded) go to the
         // order the MMA fragments take them: 16-byte vector vv of token m
@@ -281,63 +285,69 @@ __global__ void __launch_bounds__(SkCfg<NT, CG>::THREADS, 1)
         // consumer lane (token q, quarter t) reads its group's 32 values as
         // four 16-byte pieces, eight lanes of a load phase reading 128
         // contiguous bytes.  E2M1: f16 scaled by the power of two that brings
-        // the token's largest finite magnitude in this chunk into
-        // [2^14, 2^15) (exact for every element within 2^31 of it; the
-        // consumers undo the factor in fp32).  Other formats: bf16 re-paired
-        // from (k0..k7) to (k0,k4) (k1,k5) (k2,k6) (k3,k7).  Padding tokens
-        // (M .. NTOK-1) stay zero.
+        // the token's largest magnitude in this chunk into [2^14, 2^15)
+        // (exact for every element within 2^31 of it; the consumers undo the
+        // factor in fp32; a non-finite activation makes its rows non-finite
+        // either way).  Other formats: bf16 re-paired from (k0..k7) to
+        // (k0,k4) (k1,k5) (k2,k6) (k3,k7).  Padding tokens (M .. NTOK-1) stay
+        // zero.
         constexpr int VPT = CG * 16;  // vectors per token and chunk
+        constexpr int TPW = 32 / VPT;  // tokens per warp pass: 1 (CG = 2) or 2 (CG = 1)
+        const int cv = warp - 2;
         auto unit_of = [&](int m, int vv) {
             return (((vv >> 4) * 4 + (vv & 3)) * C::NTOK + m) * 64 + ((vv >> 2) & 3) * 16;
         };
-        for (int s = 0; s < C::NS; ++s) {
+        for (int s = cv; s < C::NS; s += C::CW) {
             for (int v = p.M * VPT + lane; v < C::NTOK * VPT; v += 32)
                 *reinterpret_cast<uint4*>(xfrag + s * C::XBYTES + unit_of(v / VPT, v % VPT)) =
                     make_uint4(0u, 0u, 0u, 0u);
             for (int m = p.M + lane; m < C::NTOK; m += 32) xfs[s * C::NTOK + m] = 0.f;
         }
         const int mm = p.M < C::NTOK ? p.M : C::NTOK;
-        // E2M1: LPT lanes per token (a power of two, at least 2), each taking
-        // every LPT-th vector of its token
-        int ntp = 1;
-        while (ntp < mm) ntp <<= 1;
-        const int lpt = 32 / ntp, tm = lane / lpt, sl = lane % lpt;
-        for (int j = 0; j < nch; ++j) {
+        const int vv = lane % VPT;  // this lane's vector of each token
+        // converter warp cv takes chunks cv, cv + CW, ...: all tokens of a
+        // chunk, one vector per lane and token
+        for (int j = cv; j < nch; j += C::CW) {
             const int s = j % C::NS;
             // the slot's activations landed, so its previous round was consumed
-            if (!__all_sync(0xffffffffu, mbar_wait(&xland[s], (uint32_t)(j / C::NS) & 1u, to))) {
+            if (!__all_sync(0xffffffffu, mbar_wait_sleep(&xland[s], (uint32_t)(j / C::NS) & 1u, to))) {
                 if (lane == 0) raise_status(p.status, kStatusTimeout);
                 break;
             }
-            const uint4* src = reinterpret_cast<const uint4*>(xraw + s * C::XBYTES);
-            uint8_t* dst = xfrag + s * C::XBYTES;
-            if constexpr (XM == kSkF16) {
-                uint32_t mx2 = 0;
-                if (tm < mm)
-                    for (int vv = sl; vv < VPT; vv += lpt) {
-                        const uint4 x = src[tm * VPT + vv];
-                        mx2 = finite_mag_max2(finite_mag_max2(finite_mag_max2(finite_mag_max2(mx2, x.x), x.y),
-                                                              x.z), x.w);
+            const uint32_t src = xraw_a + s * C::XBYTES;
+            const uint32_t dst = xfrag_a + s * C::XBYTES;
+#pragma unroll 4
+            for (int m0 = 0; m0 < mm; m0 += TPW) {
+                const int m = m0 + lane / VPT;
+                const bool has = m < mm;
+                const uint4 x = has ? lds128(src + (m * VPT + vv) * 16) : make_uint4(0u, 0u, 0u, 0u);
+                uint4 o;
+                float f = 1.f;
+                if constexpr (XM == kSkF16) {
+                    // largest magnitude of the token's slice (bf16 bits order like magnitudes)
+                    const uint32_t a0 = x.x & 0x7fff7fffu, a1 = x.y & 0x7fff7fffu, a2 = x.z & 0x7fff7fffu,
+                                   a3 = x.w & 0x7fff7fffu;
+                    uint32_t mx = max(max(max(a0 & 0xffffu, a0 >> 16), max(a1 & 0xffffu, a1 >> 16)),
+                                      max(max(a2 & 0xffffu, a2 >> 16), max(a3 & 0xffffu, a3 >> 16)));
+                    if constexpr (VPT == 32) {
+                        mx = __reduce_max_sync(0xffffffffu, mx);
+                    } else {
+#pragma unroll
+                        for (int o2 = 1; o2 < VPT; o2 <<= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
                     }
-                uint32_t mx = max(mx2 & 0xffffu, mx2 >> 16);
-                for (int o = 1; o < lpt; o <<= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                const int E = (int)(mx >> 7);  // biased exponent of the maximum
-                int sh = mx == 0 ? 0 : 141 - (E < 1 ? 1 : E);
-                if (sh > 126) sh = 126;
-                const float sc = __int_as_float((127 + sh) << 23);
-                if (tm < mm) {
-                    for (int vv = sl; vv < VPT; vv += lpt)
-                        *reinterpret_cast<uint4*>(dst + unit_of(tm, vv)) = bf16x8_to_f16x8(src[tm * VPT + vv], sc);
-                    if (sl == 0) xfs[s * C::NTOK + tm] = __int_as_float((127 - sh) << 23);
-                }
-            } else {
-                for (int v = lane; v < mm * VPT; v += 32) {
-                    const uint4 x = src[v];
-                    *reinterpret_cast<uint4*>(dst + unit_of(v / VPT, v % VPT)) =
-                        make_uint4(prmt(x.x, x.z, 0x5410u), prmt(x.x, x.z, 0x7632u), prmt(x.y, x.w, 0x5410u),
+                    const int E = (int)(mx >> 7);  // biased exponent of the maximum
+                    int sh = mx == 0 ? 0 : 141 - (E < 1 ? 1 : E);
+                    if (sh > 126) sh = 126;
+                    o = bf16x8_to_f16x8(x, __int_as_float((127 + sh) << 23));
+                    f = __int_as_float((127 - sh) << 23);
+                } else {
+                    o = make_uint4(prmt(x.x, x.z, 0x5410u), prmt(x.x, x.z, 0x7632u), prmt(x.y, x.w, 0x5410u),
                                    prmt(x.y, x.w, 0x7632u));
                 }
-                for (int m = lane; m < mm; m += 32) xfs[s * C::NTOK + m] = 1.f;
+                if (has) {
+                    sts128(dst + unit_of(m, vv), o);
+                    if (vv == 0) sts_f32(xfs_a + (s * C::NTOK + m) * 4, f);
+                }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&ready[s]);
@@ -373,20 +383,18 @@ __global__ void __launch_bounds__(SkCfg<NT, CG>::THREADS, 1)
             // after a timeout the loop still walks the pieces (without
             // waiting or computing) so that every consumer warp meets the
             // same named barriers
-            if (ok && !__all_sync(0xffffffffu, mbar_wait(&ready[s], (uint32_t)(j / C::NS) & 1u, to))) {
+            if (ok && !__all_sync(0xffffffffu, mbar_wait_sleep(&ready[s], (uint32_t)(j / C::NS) & 1u, to))) {
                 if (lane == 0) raise_status(p.status, kStatusTimeout);
                 ok = false;
             }
             if (ok) {
-                const uint8_t* cb = codes + s * C::CBYTES;
-                const uint8_t* xb = xfrag + s * C::XBYTES + gg * 4 * C::NTOK * 64;
-                const uint4 wa = *reinterpret_cast<const uint4*>(cb + rA * C::RB + unit);
-                const uint4 wb = *reinterpret_cast<const uint4*>(cb + rB * C::RB + unit);
-                const uint8_t* sp = reinterpret_cast<const uint8_t*>(scs) + s * C::SBYTES;
-                const float sA = sdt16 ? __half2float(reinterpret_cast<const __half*>(sp)[rA * CG + gg])
-                                       : reinterpret_cast<const float*>(sp)[rA * CG + gg];
-                const float sB = sdt16 ? __half2float(reinterpret_cast<const __half*>(sp)[rB * CG + gg])
-                                       : reinterpret_cast<const float*>(sp)[rB * CG + gg];
+                const uint32_t cb = codes_a + s * C::CBYTES;
+                const uint32_t xb = xfrag_a + s * C::XBYTES + gg * 4 * C::NTOK * 64;
+                const uint4 wa = lds128(cb + rA * C::RB + unit);
+                const uint4 wb = lds128(cb + rB * C::RB + unit);
+                const uint32_t sp = scs_a + s * C::SBYTES;
+                const float sA = sdt16 ? lds_f16_as_f32(sp + (rA * CG + gg) * 2) : lds_f32(sp + (rA * CG + gg) * 4);
+                const float sB = sdt16 ? lds_f16_as_f32(sp + (rB * CG + gg) * 2) : lds_f32(sp + (rB * CG + gg) * 4);
                 uint32_t A0[16], A1[16];
                 codes_to_frag<XM, MANT>(wa, A0);
                 codes_to_frag<XM, MANT>(wb, A1);
@@ -395,8 +403,7 @@ __global__ void __launch_bounds__(SkCfg<NT, CG>::THREADS, 1)
                     uint32_t xw[16];
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        const uint4 v =
-                            *reinterpret_cast<const uint4*>(xb + (i * C::NTOK + 8 * jn + q) * 64 + t * 16);
+                        const uint4 v = lds128(xb + (i * C::NTOK + 8 * jn + q) * 64 + t * 16);
                         xw[4 * i] = v.x;
                         xw[4 * i + 1] = v.y;
                         xw[4 * i + 2] = v.z;
@@ -413,7 +420,8 @@ __global__ void __launch_bounds__(SkCfg<NT, CG>::THREADS, 1)
                         mma_16816<XM>(acc[k & 3], A0[2 * k], A1[2 * k], A0[2 * k + 1], A1[2 * k + 1], xw[2 * k],
                                       xw[2 * k + 1]);
                     // group scale x the chunk's token factor, in fp32
-                    const float f0 = xfs[s * C::NTOK + 8 * jn + 2 * t], f1 = xfs[s * C::NTOK + 8 * jn + 2 * t + 1];
+                    const float f0 = lds_f32(xfs_a + (s * C::NTOK + 8 * jn + 2 * t) * 4),
+                                f1 = lds_f32(xfs_a + (s * C::NTOK + 8 * jn + 2 * t + 1) * 4);
                     const float w[4] = {sA * f0, sA * f1, sB * f0, sB * f1};
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
