@@ -66,11 +66,17 @@ def test_record_traffic_reads_the_first_sweep(tree, tmp_path):
     build.build()
     api.lib()
     keys = [(i, M) for M in bench.MS for i in range(len(bench.SHAPES))]
-    names = [bench.gemm_kernel_name(api, M, *bench.SHAPES[i]).split("<")[0] + "<1, 1>" for (i, M) in keys]
+    bases = [bench.gemm_kernel_name(api, M, *bench.SHAPES[i]).split("<")[0] for (i, M) in keys]
     values = [(1000 + 10 * n, 7 * n) for n in range(len(keys))]
-    csv = tmp_path / "traffic.csv"
-    _ncu_csv(csv, names, values)
-    bench.record_traffic(str(csv))
+    # one capture per kernel (as traffic_cmds() runs them), its launches in key order
+    paths = []
+    for base in sorted(set(bases)):
+        mine = [n for n in range(len(keys)) if bases[n] == base]
+        csv = tmp_path / ("traffic_%s.csv" % base)
+        _ncu_csv(csv, [base + "<1, 1>" for _ in mine], [values[n] for n in mine])
+        paths.append(str(csv))
+    assert len(paths) == len(bench.traffic_cmds())
+    bench.record_traffic(",".join(paths))
     doc = json.loads((tree / "profiles" / "traffic.json").read_text())
     assert doc["sources_sha"] == bench.kernel_sources_sha()
     assert len(doc["launches"]) == len(keys)
