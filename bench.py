@@ -117,7 +117,7 @@ def gemm_kernel_name(api, M, N, K):
     engine's token tile."""
     if api.gemm_engine_for(M, N, K, GROUP) == api.ENGINE_DECODE:
         return "gemm_rowblk_kernel" if rowblk_fits(M, K) else "gemm_skinny_kernel"
-    return "gemm_tcg_kernel<%d>" % (32 if M <= 32 else 64 if M <= 64 else 128)
+    return "gemm_tcg_kernel<%d>" % (16 if M <= 16 else 32 if M <= 32 else 64 if M <= 64 else 128)
 
 
 def host_cores():
