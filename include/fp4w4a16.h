@@ -74,6 +74,8 @@ typedef enum fp4_scale_dtype { FP4_SCALE_F32 = 0, FP4_SCALE_F16 = 1 } fp4_scale_
 
 /* GEMM engine selection for fp4_gemm_ex (fp4_gemm always uses AUTO). */
 typedef enum fp4_engine { FP4_ENGINE_AUTO = 0, FP4_ENGINE_DECODE = 1, FP4_ENGINE_TENSOR = 2 } fp4_engine;
+/* Output activation fused into the GEMM epilogue (fp4_gemm_act). */
+typedef enum fp4_act { FP4_ACT_NONE = 0, FP4_ACT_SILU = 1, FP4_ACT_GELU = 2 } fp4_act;
 
 /* Bits of the device status word. */
 #define FP4_DEV_NONFINITE_INPUT 0x1 /* NaN/Inf met in W or X                   */
@@ -233,6 +235,24 @@ FP4_API fp4_status fp4_gemm_ex(const uint16_t *X, const uint8_t *packed, const v
                        fp4_scale_dtype sdt, fp4_format fmt, int M, int N, int K, int group,
                        const float *x_scale, uint16_t *Y, void *workspace, size_t ws_bytes,
                        fp4_engine engine, int splits, cudaStream_t stream);
+
+/* fp4_gemm_ex with an output activation applied in the epilogue, in fp32,
+ * to the finished value before the bf16 rounding (HiFloat4 page, section 5
+ * "性能优化实战案例", optimisation measures: the fused Quant-GeLU-Dequant
+ * operator; here the activations stay 16-bit, so the fusion is the
+ * activation of the layer output inside the GEMM):
+ *
+ *   Y[m,n] = bf16_rne( act( rho * sum_k X[m,k] * v(code[n,k]) * s[n,k/group] ) )
+ *
+ *   act  FP4_ACT_NONE: identity; FP4_ACT_SILU: y / (1 + exp(-y));
+ *        FP4_ACT_GELU: y * (1 + erf(y / sqrt 2)) / 2.  Anything else returns
+ *        FP4_ERR_INVALID_ARG.
+ * Every engine and kernel supports it, with the other arguments as for
+ * fp4_gemm_ex; act(y) is computed once per output after any split-K sum. */
+FP4_API fp4_status fp4_gemm_act(const uint16_t *X, const uint8_t *packed, const void *scales,
+                        fp4_scale_dtype sdt, fp4_format fmt, int M, int N, int K, int group,
+                        const float *x_scale, fp4_act act, uint16_t *Y, void *workspace, size_t ws_bytes,
+                        fp4_engine engine, int splits, cudaStream_t stream);
 
 /* Engine fp4_gemm runs for this shape (FP4_ENGINE_DECODE or
  * FP4_ENGINE_TENSOR); host-only, no device call.  Non-positive sizes or an

@@ -21,6 +21,7 @@ _HDR = os.path.join(_HERE, "fp4_oracle.h")
 _LIB = os.path.join(_HERE, "libfp4_oracle.so")
 
 E1M2, E2M1, E3M0, AUTO = 0, 1, 2, -1
+ACT_NONE, ACT_SILU, ACT_GELU = 0, 1, 2
 SCALE_F32, SCALE_F16 = 0, 1
 FORMAT_NAMES = ("E1M2", "E2M1", "E3M0")
 
@@ -201,6 +202,29 @@ def gemm(X_bf16, packed, scales, fmt, group, rho=1.0):
     Y = np.zeros((M, N), np.float64)
     _check(_L().orc_gemm(_p(X), _p(packed), _p(scales), sdt, fmt, M, N, K, group, float(rho), _p(Y)))
     return Y
+
+
+def activation(Y, act):
+    """The output activation of the fused epilogue, elementwise in fp64 on
+    the finished product Y (HiFloat4 page, section 5 "性能优化实战案例": the
+    fused Quant-GeLU-Dequant operator).  SiLU y / (1 + e^-y); GeLU in its
+    erf form y * (1 + erf(y / sqrt 2)) / 2 (Python's math.erf, double)."""
+    import math
+    Y = np.asarray(Y, np.float64)
+    if act == ACT_NONE:
+        return Y.copy()
+    if act == ACT_SILU:
+        with np.errstate(over="ignore"):
+            return Y / (1.0 + np.exp(-Y))
+    if act == ACT_GELU:
+        erf = np.vectorize(math.erf, otypes=[np.float64])
+        return 0.5 * Y * (1.0 + erf(Y / math.sqrt(2.0)))
+    raise OracleError("unknown activation %r" % (act,))
+
+
+def gemm_act(X_bf16, packed, scales, fmt, group, act, rho=1.0):
+    """act(rho * X . dequant(W)^T) in fp64: gemm() followed by activation()."""
+    return activation(gemm(X_bf16, packed, scales, fmt, group, rho), act)
 
 
 def gemm_sampled(X_bf16, packed, scales, fmt, group, ms, ns, rho=1.0):

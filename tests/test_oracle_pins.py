@@ -499,6 +499,32 @@ def test_gemm_quantization_error_is_small(oracle_mod):
     assert cos > 0.98
 
 
+def test_activation_pins(oracle_mod):
+    """The epilogue activations against facts outside the oracle: the
+    standard normal CDF at 1 and 2 (printed tables: 0.841344746068543,
+    0.977249868051821), the logistic function at 1 and ln 3 (1/(1+e^-1)
+    and exactly 3/4), zero at zero, and the odd-part identity
+    act(y) - act(-y) = y that both satisfy (Phi(y) + Phi(-y) = 1,
+    sigmoid(y) + sigmoid(-y) = 1)."""
+    import math
+    A = oracle_mod
+    g = A.activation(np.array([0.0, 1.0, 2.0, -1.0]), A.ACT_GELU)
+    np.testing.assert_allclose(g, [0.0, 0.841344746068543, 2 * 0.977249868051821, -(1 - 0.841344746068543)],
+                               rtol=1e-14, atol=1e-15)
+    s = A.activation(np.array([0.0, 1.0, math.log(3.0)]), A.ACT_SILU)
+    np.testing.assert_allclose(s, [0.0, 1.0 / (1.0 + math.exp(-1.0)), 0.75 * math.log(3.0)], rtol=1e-14, atol=0)
+    y = np.linspace(-7.0, 7.0, 57)
+    for act in (A.ACT_SILU, A.ACT_GELU):
+        np.testing.assert_allclose(A.activation(y, act) - A.activation(-y, act), y, rtol=0, atol=1e-12)
+    np.testing.assert_array_equal(A.activation(y, A.ACT_NONE), y)
+    # gemm_act is the activation of the plain product
+    W, X = synth.random_case(15, 32, 256, 3)
+    r = A.quantize(W, 128, 1)
+    Y = A.gemm(X, r["packed"], r["scales"], 1, 128, 0.5)
+    np.testing.assert_array_equal(A.gemm_act(X, r["packed"], r["scales"], 1, 128, A.ACT_GELU, 0.5),
+                                  A.activation(Y, A.ACT_GELU))
+
+
 def test_golden_tiny_digest(oracle_mod):
     """The tiny workload's oracle outputs match the committed digest."""
     import hashlib

@@ -246,6 +246,40 @@ def test_gemm_decode_formats(fp4, oracle_mod, fmt, sdt, M, splits):
                      rho=0.75) <= TOL
 
 
+@pytest.mark.parametrize("act", [1, 2])
+@pytest.mark.parametrize("M,N,K,group,engine,splits", [
+    (4, 300, 1024, 128, 1, 0),      # row-block decode kernel
+    (4, 300, 1024, 128, 1, 148),    # streaming decode kernel, whole tiles and split tiles
+    (13, 300, 1024, 128, 1, 148),   # streaming, two token tiles
+    (40, 300, 1024, 128, 1, 0),     # tensor-memory decode kernel
+    (16, 300, 1024, 128, 2, 0),     # tensor engine, 16-token tile
+    (64, 300, 2048, 128, 2, 0),     # tensor engine, 64-token tile, split K over a cluster
+    (200, 300, 1024, 128, 2, 1),    # 128-token tile, f16 path (default workspace)
+    (4, 300, 1024, 64, 1, 0),       # lookup-table decode kernel, group 64
+    (40, 300, 1024, 32, 2, 0),      # tensor engine, group 32
+])
+def test_gemm_activation(fp4, oracle_mod, act, M, N, K, group, engine, splits):
+    """The fused output activation (SiLU, GeLU) in every kernel's epilogue,
+    after any split-K sum, against the oracle's activation of its fp64
+    product; rho != 1 so that the activation sees the scaled value."""
+    W, X = synth.random_case(60 + M + act, N, K, M)
+    res = fp4.quantize(dev_f32(W), group, 1)
+    xs = torch.tensor([0.75], dtype=torch.float32, device="cuda")
+    Y = fp4.gemm(dev_bf16(X), res["packed"], res["scales"], 1, group, x_scale=xs, engine=engine, splits=splits,
+                 act=act)
+    Yref = oracle_mod.gemm_act(X, res["packed"].cpu().numpy(), res["scales"].cpu().numpy(), 1, group, act, 0.75)
+    assert rel_err(Y, Yref) <= TOL
+    assert np.all(np.isfinite(Y.float().cpu().numpy()))
+
+
+def test_gemm_activation_rejects_unknown(fp4):
+    W, X = synth.random_case(70, 64, 256, 2)
+    res = fp4.quantize(dev_f32(W), 128, 1)
+    with pytest.raises(fp4.Fp4Error) as err:
+        fp4.gemm(dev_bf16(X), res["packed"], res["scales"], 1, 128, act=3)
+    assert err.value.code == 1
+
+
 def test_gemm_decode_needs_workspace(fp4, oracle_mod):
     """The streaming decode kernels keep tile counters and partials in the
     workspace: forced without one (a CTA count selects them) the call

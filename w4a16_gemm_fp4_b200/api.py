@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(HERE, "libfp4w4a16.so")
 E1M2, E2M1, E3M0, AUTO = 0, 1, 2, -1
 SCALE_F32, SCALE_F16 = 0, 1
 ENGINE_AUTO, ENGINE_DECODE, ENGINE_TENSOR = 0, 1, 2
+ACT_NONE, ACT_SILU, ACT_GELU = 0, 1, 2
 DEV_NONFINITE_INPUT, DEV_SCALE_OVERFLOW, DEV_WAIT_TIMEOUT, DEV_LAYOUT = 1, 2, 4, 8
 
 STATUS = {0: "FP4_OK", 1: "FP4_ERR_INVALID_ARG", 2: "FP4_ERR_UNSUPPORTED_SHAPE", 3: "FP4_ERR_MISALIGNED",
@@ -26,7 +27,7 @@ STATUS = {0: "FP4_OK", 1: "FP4_ERR_INVALID_ARG", 2: "FP4_ERR_UNSUPPORTED_SHAPE",
 
 EXPORTS = ("fp4_abi_version", "fp4_status_string", "fp4_quantize_workspace_size", "fp4_quantize",
            "fp4_dequantize", "fp4_preshift_workspace_size", "fp4_preshift_calibrate", "fp4_preshift_apply",
-           "fp4_gemm_workspace_size", "fp4_gemm", "fp4_gemm_ex", "fp4_get_device_status",
+           "fp4_gemm_workspace_size", "fp4_gemm", "fp4_gemm_ex", "fp4_gemm_act", "fp4_get_device_status",
            "fp4_set_wait_timeout_us", "fp4_selftest_bounded_wait", "fp4_preshift_calibrate_noalloc",
            "fp4_gemm_engine_for")
 
@@ -65,6 +66,7 @@ def lib():
                 "fp4_gemm_workspace_size": (sz, [i, i, i]),
                 "fp4_gemm": (i, [P, P, P, i, i, i, i, i, i, P, P, P, sz, P]),
                 "fp4_gemm_ex": (i, [P, P, P, i, i, i, i, i, i, P, P, P, sz, i, i, P]),
+                "fp4_gemm_act": (i, [P, P, P, i, i, i, i, i, i, P, i, P, P, sz, i, i, P]),
                 "fp4_get_device_status": (i, [ctypes.POINTER(ctypes.c_int32), i, P]),
                 "fp4_set_wait_timeout_us": (None, [ll]),
                 "fp4_selftest_bounded_wait": (i, [ll, P]),
@@ -224,13 +226,15 @@ def gemm_engine_for(M, N, K, group=128):
 
 
 def gemm(X, packed, scales, fmt=E2M1, group=128, x_scale=None, out=None, engine=ENGINE_AUTO, splits=0,
-         workspace=None, stream=None):
-    """Y = bf16(x_scale * X . dequant(W)^T).  X: [M][K] bf16 CUDA tensor.
+         workspace=None, stream=None, act=ACT_NONE):
+    """Y = bf16(act(x_scale * X . dequant(W)^T)).  X: [M][K] bf16 CUDA tensor.
 
-    ``workspace`` defaults to a per-device buffer of fp4_gemm_workspace_size
-    bytes (the activations prepared once per call); a smaller one makes the
-    kernels convert the activations themselves.  ``engine``/``splits`` force
-    an engine or a split-K count (0: automatic)."""
+    ``workspace`` defaults to a per-device zero-filled buffer of
+    fp4_gemm_workspace_size bytes (tile counters, partial tiles, prepared
+    activations); a smaller one makes the automatic choice take the tensor
+    engine's bf16 path.  ``engine``/``splits`` force an engine or a split
+    count (0: automatic).  ``act``: ACT_NONE, ACT_SILU or ACT_GELU, applied
+    in the epilogue."""
     M, K = X.shape
     N = packed.shape[0]
     assert packed.shape[1] * 2 == K
@@ -243,8 +247,8 @@ def gemm(X, packed, scales, fmt=E2M1, group=128, x_scale=None, out=None, engine=
         ws, wsb = _workspace(X.device, "gemm").get(need)
     else:
         ws, wsb = workspace, workspace.numel() * workspace.element_size()
-    _check(L.fp4_gemm_ex(_ptr(_bits(X)), _ptr(packed), _ptr(scales), sdt, fmt, M, N, K, group, _ptr(x_scale),
-                         _ptr(_bits(out)), _ptr(ws), wsb, engine, splits, _stream(stream)), "fp4_gemm")
+    _check(L.fp4_gemm_act(_ptr(_bits(X)), _ptr(packed), _ptr(scales), sdt, fmt, M, N, K, group, _ptr(x_scale),
+                          act, _ptr(_bits(out)), _ptr(ws), wsb, engine, splits, _stream(stream)), "fp4_gemm")
     return out
 
 

@@ -25,28 +25,29 @@ cudaError_t launch_apply(const uint16_t* X, int M, int K, const int8_t* shift, c
                          cudaStream_t st);
 cudaError_t launch_gemm_decode(const uint16_t* X, const uint8_t* packed, const void* scales, int sdt,
                                const FmtTable& t, int M, int N, int K, int group, const float* x_scale, uint16_t* Y,
-                               cudaStream_t st);
+                               int act, cudaStream_t st);
 int decode_max_m_lut();
 cudaError_t launch_gemm_ts(const uint16_t* X, void* ws, size_t ws_bytes, const uint8_t* packed, const void* scales,
-                           int sdt, int fmt, int M, int N, int K, const float* x_scale, uint16_t* Y, int ctas,
-                           int* status, unsigned long long timeout_ns, cudaStream_t st);
+                           int sdt, int fmt, int M, int N, int K, const float* x_scale, uint16_t* Y, int act,
+                           int ctas, int* status, unsigned long long timeout_ns, cudaStream_t st);
 size_t ts_ws_bytes(int M, int N, int K);
 cudaError_t launch_gemm_skinny(const uint16_t* X, int* cnt, void* ws, size_t ws_bytes, const uint8_t* packed,
                                const void* scales, int sdt, int fmt, int M, int N, int K, const float* x_scale,
-                               uint16_t* Y, int ctas, int* status, unsigned long long timeout_ns, cudaStream_t st);
+                               uint16_t* Y, int act, int ctas, int* status, unsigned long long timeout_ns,
+                               cudaStream_t st);
 size_t skinny_ws_bytes(int M, int N, int K);
 int skinny_max_m();
 int skinny_max_tiles();
 int skinny_tiles(int N, int K);
 cudaError_t launch_gemm_rowblk(const uint16_t* X, const uint8_t* packed, const void* scales, int sdt, int fmt,
-                               int M, int N, int K, const float* x_scale, uint16_t* Y, int* status,
+                               int M, int N, int K, const float* x_scale, uint16_t* Y, int act, int* status,
                                unsigned long long timeout_ns, cudaStream_t st);
 bool rowblk_fits(int M, int K);
 bool rowblk_preferred(int M, int K);
 size_t tc_ws_bytes(int M, int N, int K);
 cudaError_t launch_gemm_tc(const uint16_t* X, const uint8_t* packed, const void* scales, int sdt, const FmtTable& t,
-                           bool e2m1, int M, int N, int K, int group, const float* x_scale, uint16_t* Y, void* ws,
-                           size_t ws_bytes, int splits, int* status, unsigned long long timeout_ns,
+                           bool e2m1, int M, int N, int K, int group, const float* x_scale, uint16_t* Y, int act,
+                           void* ws, size_t ws_bytes, int splits, int* status, unsigned long long timeout_ns,
                            cudaStream_t st);
 cudaError_t launch_bounded_wait_probe(int* status, unsigned long long timeout_ns, cudaStream_t st);
 int noalloc_max_k();
@@ -317,10 +318,12 @@ static size_t decode_ws_bytes(int M, int N, int K) {
     return kCounterBlock + (skinny_fits(M, N, K) ? skinny_ws_bytes(M, N, K) : ts_ws_bytes(M, N, K));
 }
 
-fp4_status fp4_gemm_ex(const uint16_t* X, const uint8_t* packed, const void* scales, fp4_scale_dtype sdt,
-                       fp4_format fmt, int M, int N, int K, int group, const float* x_scale, uint16_t* Y,
-                       void* workspace, size_t ws_bytes, fp4_engine engine, int splits, cudaStream_t stream) {
+fp4_status fp4_gemm_act(const uint16_t* X, const uint8_t* packed, const void* scales, fp4_scale_dtype sdt,
+                        fp4_format fmt, int M, int N, int K, int group, const float* x_scale, fp4_act act,
+                        uint16_t* Y, void* workspace, size_t ws_bytes, fp4_engine engine, int splits,
+                        cudaStream_t stream) {
     if (M < 0) return FP4_ERR_INVALID_ARG;
+    if (act != FP4_ACT_NONE && act != FP4_ACT_SILU && act != FP4_ACT_GELU) return FP4_ERR_INVALID_ARG;
     fp4_status s = check_weights(packed, scales, sdt, fmt, N, K, group);
     if (s != FP4_OK) return s;
     if (engine != FP4_ENGINE_AUTO && engine != FP4_ENGINE_DECODE && engine != FP4_ENGINE_TENSOR)
@@ -331,6 +334,7 @@ fp4_status fp4_gemm_ex(const uint16_t* X, const uint8_t* packed, const void* sca
     if (!aligned(Y, 16)) return FP4_ERR_MISALIGNED;
     if (x_scale && !aligned(x_scale, 4)) return FP4_ERR_MISALIGNED;
     if (workspace && !aligned(workspace, 16)) return FP4_ERR_MISALIGNED;
+    // K = 0: every output is act(0) = 0 for the supported activations
     if (K == 0) return cuda_status(cudaMemsetAsync(Y, 0, (size_t)M * N * sizeof(uint16_t), stream));
     if (!X) return FP4_ERR_INVALID_ARG;
     if (!aligned(X, 16)) return FP4_ERR_MISALIGNED;
@@ -360,19 +364,27 @@ fp4_status fp4_gemm_ex(const uint16_t* X, const uint8_t* packed, const void* sca
     const unsigned long long to_ns = (unsigned long long)g_timeout_us * 1000ull;
     if (engine == FP4_ENGINE_DECODE) {
         if (rowblk)
-            return cuda_status(launch_gemm_rowblk(X, packed, scales, (int)sdt, (int)fmt, M, N, K, x_scale, Y, st,
-                                                  to_ns, stream));
+            return cuda_status(launch_gemm_rowblk(X, packed, scales, (int)sdt, (int)fmt, M, N, K, x_scale, Y,
+                                                  (int)act, st, to_ns, stream));
         if (group == 128 && skinny_fits(M, N, K))
             return cuda_status(launch_gemm_skinny(X, static_cast<int*>(workspace), eng_ws, eng_bytes, packed, scales,
-                                                  (int)sdt, (int)fmt, M, N, K, x_scale, Y, splits, st, to_ns,
-                                                  stream));
+                                                  (int)sdt, (int)fmt, M, N, K, x_scale, Y, (int)act, splits, st,
+                                                  to_ns, stream));
         if (group == 128)
             return cuda_status(launch_gemm_ts(X, eng_ws, eng_bytes, packed, scales, (int)sdt, (int)fmt, M, N, K,
-                                              x_scale, Y, splits, st, to_ns, stream));
-        return cuda_status(launch_gemm_decode(X, packed, scales, (int)sdt, t, M, N, K, group, x_scale, Y, stream));
+                                              x_scale, Y, (int)act, splits, st, to_ns, stream));
+        return cuda_status(
+            launch_gemm_decode(X, packed, scales, (int)sdt, t, M, N, K, group, x_scale, Y, (int)act, stream));
     }
     return cuda_status(launch_gemm_tc(X, packed, scales, (int)sdt, t, fmt == FP4_E2M1, M, N, K, group, x_scale, Y,
-                                      eng_ws, eng_bytes, splits, st, to_ns, stream));
+                                      (int)act, eng_ws, eng_bytes, splits, st, to_ns, stream));
+}
+
+fp4_status fp4_gemm_ex(const uint16_t* X, const uint8_t* packed, const void* scales, fp4_scale_dtype sdt,
+                       fp4_format fmt, int M, int N, int K, int group, const float* x_scale, uint16_t* Y,
+                       void* workspace, size_t ws_bytes, fp4_engine engine, int splits, cudaStream_t stream) {
+    return fp4_gemm_act(X, packed, scales, sdt, fmt, M, N, K, group, x_scale, FP4_ACT_NONE, Y, workspace, ws_bytes,
+                        engine, splits, stream);
 }
 
 fp4_engine fp4_gemm_engine_for(int M, int N, int K, int group) {

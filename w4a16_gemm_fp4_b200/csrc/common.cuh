@@ -168,6 +168,18 @@ __device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4 v, float sc) {
     return make_uint4(h[0], h[1], h[2], h[3]);
 }
 
+// Output activation of the GEMM epilogue, applied to the finished fp32 value
+// y = rho * sum before the bf16 rounding (HiFloat4 page, section 5, fused
+// operators: the activation that follows the linear layer runs in the GEMM's
+// epilogue).  0: none; 1: SiLU y * sigmoid(y); 2: GeLU y * Phi(y), the erf
+// form.
+enum { kActNone = 0, kActSilu = 1, kActGelu = 2 };
+__device__ __forceinline__ float apply_act(float y, int act) {
+    if (act == kActSilu) return y / (1.f + expf(-y));
+    if (act == kActGelu) return 0.5f * y * (1.f + erff(y * 0.70710678118654752f));
+    return y;
+}
+
 // bf16 bit pattern of v, round to nearest even.
 __device__ __forceinline__ uint16_t bf16_bits(float v) { return __bfloat16_as_ushort(__float2bfloat16_rn(v)); }
 

@@ -36,6 +36,7 @@ struct DecodeParams {
     int M, N, K, group;
     const float* x_scale;
     uint16_t* Y;
+    int act;
 };
 
 __device__ __forceinline__ void mma_bf16_16816(float d[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -154,7 +155,7 @@ __global__ void __launch_bounds__(256) gemm_decode_kernel(DecodeParams p) {
         const int n = n0 + 16 * r + (l >> 2) + 8 * (j >> 1);
         const int m = 2 * (l & 3) + (j & 1);
         if (m < p.M && n < p.N) {
-            __nv_bfloat16 y = __float2bfloat16_rn(rho * s);
+            __nv_bfloat16 y = __float2bfloat16_rn(apply_act(rho * s, p.act));
             p.Y[(size_t)m * p.N + n] = *reinterpret_cast<uint16_t*>(&y);
         }
     }
@@ -168,8 +169,8 @@ int decode_max_m_lut() { return 8; }
 
 cudaError_t launch_gemm_decode(const uint16_t* X, const uint8_t* packed, const void* scales, int sdt,
                                const FmtTable& t, int M, int N, int K, int group, const float* x_scale, uint16_t* Y,
-                               cudaStream_t st) {
-    DecodeParams p{X, packed, scales, sdt, t, M, N, K, group, x_scale, Y};
+                               int act, cudaStream_t st) {
+    DecodeParams p{X, packed, scales, sdt, t, M, N, K, group, x_scale, Y, act};
     if (M > decode_max_m_lut()) return cudaErrorInvalidValue;
     const int R = decode_rows_per_cta(N);
     const int blocks = (N + 16 * R - 1) / (16 * R);

@@ -19,6 +19,7 @@ struct RbParams {
     int M, N, K;
     const float* x_scale;
     uint16_t* Y;
+    int act;
 };
 
 __device__ __forceinline__ uint32_t word_of(const uint4& v, int i) {
@@ -347,7 +348,7 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
             for (int w = 0; w < NW; ++w) sum += rd[((tt * NW + w) * 32 + l) * 4 + j];
             const int n = n0 + (l >> 2) + 8 * (j >> 1), m = 8 * tt + 2 * (l & 3) + (j & 1);
             if (m < p.M && n < p.N) {
-                __nv_bfloat16 y = __float2bfloat16_rn(rho * (kCvt ? row_f[m] * sum : sum));
+                __nv_bfloat16 y = __float2bfloat16_rn(apply_act(rho * (kCvt ? row_f[m] * sum : sum), p.act));
                 p.Y[(size_t)m * p.N + n] = *reinterpret_cast<uint16_t*>(&y);
             }
         }
@@ -444,10 +445,10 @@ bool rowblk_preferred(int M, int K) {
 }
 
 cudaError_t launch_gemm_rowblk(const uint16_t* X, const uint8_t* packed, const void* scales, int sdt, int fmt,
-                               int M, int N, int K, const float* x_scale, uint16_t* Y, int* status,
+                               int M, int N, int K, const float* x_scale, uint16_t* Y, int act, int* status,
                                unsigned long long timeout_ns, cudaStream_t st) {
     if (K % 128 != 0 || M <= 0 || N <= 0) return cudaErrorInvalidValue;
-    RbParams p{X, packed, scales, sdt, M, N, K, x_scale, Y};
+    RbParams p{X, packed, scales, sdt, M, N, K, x_scale, Y, act};
     const bool f16 = sdt == FP4_SCALE_F16;
     if (fmt == FP4_E1M2)
         return f16 ? launch_rb_nw<2, FP4_SCALE_F16>(p, status, timeout_ns, st)

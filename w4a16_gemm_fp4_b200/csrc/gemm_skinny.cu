@@ -49,6 +49,7 @@ struct SkParams {
     int C, P;                // code chunks, CTAs
     int* status;
     unsigned long long timeout_ns;
+    int act;                 // output activation (apply_act)
 };
 
 template <int NT, int CG>
@@ -467,8 +468,11 @@ __global__ void __launch_bounds__(SkCfg<NT, CG>::THREADS, 1)
                         for (int e = 0; e < 2; ++e) {
                             const int m = 8 * jn + 2 * t + e;
                             if (m < p.M) {
-                                if (n0 + rA < p.N) p.Y[(size_t)m * p.N + n0 + rA] = bf16_bits(rho * tot[jn][e]);
-                                if (n0 + rB < p.N) p.Y[(size_t)m * p.N + n0 + rB] = bf16_bits(rho * tot[jn][2 + e]);
+                                if (n0 + rA < p.N)
+                                    p.Y[(size_t)m * p.N + n0 + rA] = bf16_bits(apply_act(rho * tot[jn][e], p.act));
+                                if (n0 + rB < p.N)
+                                    p.Y[(size_t)m * p.N + n0 + rB] =
+                                        bf16_bits(apply_act(rho * tot[jn][2 + e], p.act));
                             }
                         }
                 }
@@ -525,8 +529,8 @@ __global__ void __launch_bounds__(SkCfg<NT, CG>::THREADS, 1)
                         }
                         const int m = qd / (TR / 4), n = n0 + (qd % (TR / 4)) * 4;
                         uint16_t* dst = p.Y + (size_t)m * p.N + n;
-                        const uint32_t y01 = pack_bf16x2(rho * sum.x, rho * sum.y),
-                                       y23 = pack_bf16x2(rho * sum.z, rho * sum.w);
+                        const uint32_t y01 = pack_bf16x2(apply_act(rho * sum.x, p.act), apply_act(rho * sum.y, p.act)),
+                                       y23 = pack_bf16x2(apply_act(rho * sum.z, p.act), apply_act(rho * sum.w, p.act));
                         if ((p.N & 3) == 0 && n + 3 < p.N) {
                             *reinterpret_cast<uint2*>(dst) = make_uint2(y01, y23);
                         } else {
@@ -636,7 +640,8 @@ static cudaError_t launch_sk_fmt(int fmt, const CUtensorMap& mw, const CUtensorM
 // one CTA per SM (at most one per code chunk).
 cudaError_t launch_gemm_skinny(const uint16_t* X, int* cnt, void* ws, size_t ws_bytes, const uint8_t* packed,
                                const void* scales, int sdt, int fmt, int M, int N, int K, const float* x_scale,
-                               uint16_t* Y, int ctas, int* status, unsigned long long timeout_ns, cudaStream_t st) {
+                               uint16_t* Y, int act, int ctas, int* status, unsigned long long timeout_ns,
+                               cudaStream_t st) {
     if (K % 128 != 0 || M <= 0 || M > 16 || N <= 0 || cnt == nullptr) return cudaErrorInvalidValue;
     if (skinny_tiles(N, K) > kSkinnyCounters) return cudaErrorInvalidValue;
     int chunks = 0;
@@ -667,6 +672,7 @@ cudaError_t launch_gemm_skinny(const uint16_t* X, int* cnt, void* ws, size_t ws_
     p.P = P;
     p.status = status;
     p.timeout_ns = timeout_ns;
+    p.act = act;
     if (CG == 2) return NT == 1 ? launch_sk_fmt<1, 2>(fmt, mw, mx, p, st) : launch_sk_fmt<2, 2>(fmt, mw, mx, p, st);
     return NT == 1 ? launch_sk_fmt<1, 1>(fmt, mw, mx, p, st) : launch_sk_fmt<2, 1>(fmt, mw, mx, p, st);
 }

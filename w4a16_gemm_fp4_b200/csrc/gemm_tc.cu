@@ -52,6 +52,7 @@ struct TcParams {
     int splits;          // CTAs along K per output tile (one cluster)
     int* status;
     unsigned long long timeout_ns;
+    int act;             // output activation (apply_act)
 };
 
 template <int BT>
@@ -159,8 +160,10 @@ __device__ __forceinline__ void cluster_reduce_store(const TcParams& p, uint32_t
                 a.z *= f;
                 a.w *= f;
             }
-            __nv_bfloat16 y[4] = {__float2bfloat16_rn(rho * a.x), __float2bfloat16_rn(rho * a.y),
-                                  __float2bfloat16_rn(rho * a.z), __float2bfloat16_rn(rho * a.w)};
+            __nv_bfloat16 y[4] = {__float2bfloat16_rn(apply_act(rho * a.x, p.act)),
+                                  __float2bfloat16_rn(apply_act(rho * a.y, p.act)),
+                                  __float2bfloat16_rn(apply_act(rho * a.z, p.act)),
+                                  __float2bfloat16_rn(apply_act(rho * a.w, p.act))};
             uint16_t* dst = p.Y + (size_t)m * p.N + n;
             if (vec_store && n + 3 < p.N) {
                 uint2 w;
@@ -451,7 +454,7 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
                 for (int j = 0; j < C::FCOLS; ++j) {
                     const int m = m0 + cb + j;
                     if (m < p.M) {
-                        __nv_bfloat16 y = __float2bfloat16_rn(rho * tot[j]);
+                        __nv_bfloat16 y = __float2bfloat16_rn(apply_act(rho * tot[j], p.act));
                         p.Y[(size_t)m * p.N + n] = *reinterpret_cast<uint16_t*>(&y);
                     }
                 }
@@ -791,7 +794,7 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
                     const int m = m0 + cb + j;
                     if (m < p.M) {
                         const float t = F16 ? tot[j] * xfw[j] : tot[j];
-                        __nv_bfloat16 y = __float2bfloat16_rn(rho * t);
+                        __nv_bfloat16 y = __float2bfloat16_rn(apply_act(rho * t, p.act));
                         p.Y[(size_t)m * p.N + n] = *reinterpret_cast<uint16_t*>(&y);
                     }
                 }
@@ -831,10 +834,10 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
                 const int c = c0 + u * kT, j = c >> 4, n = n0 + (c & 15) * 8, m = m0 + j;
                 if (m < p.M && n < p.N) {
                     uint4 o;
-                    o.x = pack_bf16x2(a[u].x * f[u], a[u].y * f[u]);
-                    o.y = pack_bf16x2(a[u].z * f[u], a[u].w * f[u]);
-                    o.z = pack_bf16x2(b[u].x * f[u], b[u].y * f[u]);
-                    o.w = pack_bf16x2(b[u].z * f[u], b[u].w * f[u]);
+                    o.x = pack_bf16x2(apply_act(a[u].x * f[u], p.act), apply_act(a[u].y * f[u], p.act));
+                    o.y = pack_bf16x2(apply_act(a[u].z * f[u], p.act), apply_act(a[u].w * f[u], p.act));
+                    o.z = pack_bf16x2(apply_act(b[u].x * f[u], p.act), apply_act(b[u].y * f[u], p.act));
+                    o.w = pack_bf16x2(apply_act(b[u].z * f[u], p.act), apply_act(b[u].w * f[u], p.act));
                     *reinterpret_cast<uint4*>(p.Y + (size_t)m * p.N + n) = o;
                 }
             }
@@ -1100,8 +1103,8 @@ int tcg_splits(int M, int N, int K) {
 }
 
 cudaError_t launch_gemm_tc(const uint16_t* X, const uint8_t* packed, const void* scales, int sdt, const FmtTable& t,
-                           bool e2m1, int M, int N, int K, int group, const float* x_scale, uint16_t* Y, void* ws,
-                           size_t ws_bytes, int splits, int* status, unsigned long long timeout_ns,
+                           bool e2m1, int M, int N, int K, int group, const float* x_scale, uint16_t* Y, int act,
+                           void* ws, size_t ws_bytes, int splits, int* status, unsigned long long timeout_ns,
                            cudaStream_t st) {
     const int BTg = tcg_token_tile(M, K, group);
     if (BTg > 0) {
@@ -1134,6 +1137,7 @@ cudaError_t launch_gemm_tc(const uint16_t* X, const uint8_t* packed, const void*
         p.splits = splits;
         p.status = status;
         p.timeout_ns = timeout_ns;
+        p.act = act;
         if (f16) {
             cudaError_t e = launch_x_rows_to_f16(X, M, K, Xh, xrow, nullptr, 0, st);
             if (e != cudaSuccess) return e;
@@ -1172,6 +1176,7 @@ cudaError_t launch_gemm_tc(const uint16_t* X, const uint8_t* packed, const void*
     p.splits = splits;
     p.status = status;
     p.timeout_ns = timeout_ns;
+    p.act = act;
     switch (BT) {
         case 32: return launch_tc_bt<32>(mx, mw, p, st);
         case 64: return launch_tc_bt<64>(mx, mw, p, st);

@@ -78,6 +78,7 @@ struct TsParams {
     int P;                 // CTAs
     int* status;
     unsigned long long timeout_ns;
+    int act;               // output activation (apply_act)
 };
 
 template <int BT, int CG>
@@ -397,7 +398,7 @@ __global__ void __launch_bounds__(TsCfg<BT, CG>::THREADS, 1)
                     for (int k = 0; k < C::FCOLS; ++k) {
                         const int m = cb + k;
                         if (m < p.M) {
-                            __nv_bfloat16 y = __float2bfloat16_rn(rho * tot[k] * xrw[k]);
+                            __nv_bfloat16 y = __float2bfloat16_rn(apply_act(rho * tot[k] * xrw[k], p.act));
                             p.Y[(size_t)m * p.N + n] = *reinterpret_cast<uint16_t*>(&y);
                         }
                     }
@@ -459,8 +460,10 @@ __global__ void __launch_bounds__(TsCfg<BT, CG>::THREADS, 1)
                             const int m = qd >> 5, n4 = t * C::BW + (qd & 31) * 4;
                             const float4 a = acc[qb];
                             if (m < p.M && n4 < p.N) {
-                                const uint32_t y01 = pack_bf16x2(rho * a.x, rho * a.y),
-                                               y23 = pack_bf16x2(rho * a.z, rho * a.w);
+                                const uint32_t y01 = pack_bf16x2(apply_act(rho * a.x, p.act),
+                                                                 apply_act(rho * a.y, p.act)),
+                                               y23 = pack_bf16x2(apply_act(rho * a.z, p.act),
+                                                                 apply_act(rho * a.w, p.act));
                                 uint16_t* dst = p.Y + (size_t)m * p.N + n4;
                                 if ((p.N & 3) == 0 && n4 + 3 < p.N) {
                                     *reinterpret_cast<uint2*>(dst) = make_uint2(y01, y23);
@@ -620,8 +623,8 @@ static cudaError_t launch_ts_fmt(int fmt, const CUtensorMap& mx, const CUtensorM
 // Decode engine (M <= 64, group 128).  ws must hold ts_ws_bytes(M, N, K)
 // bytes; ctas = 0 takes one CTA per SM (at most one per code chunk).
 cudaError_t launch_gemm_ts(const uint16_t* X, void* ws, size_t ws_bytes, const uint8_t* packed, const void* scales,
-                           int sdt, int fmt, int M, int N, int K, const float* x_scale, uint16_t* Y, int ctas,
-                           int* status, unsigned long long timeout_ns, cudaStream_t st) {
+                           int sdt, int fmt, int M, int N, int K, const float* x_scale, uint16_t* Y, int act,
+                           int ctas, int* status, unsigned long long timeout_ns, cudaStream_t st) {
     if (K % 128 != 0 || M <= 0 || M > 64 || N <= 0) return cudaErrorInvalidValue;
     const TsLayout L = ts_layout(M, N, K, ctas);
     if (ws == nullptr || ws_bytes < L.total) return cudaErrorInvalidValue;
@@ -654,6 +657,7 @@ cudaError_t launch_gemm_ts(const uint16_t* X, void* ws, size_t ws_bytes, const u
     p.P = L.P;
     p.status = status;
     p.timeout_ns = timeout_ns;
+    p.act = act;
     cudaError_t e = fmt == FP4_E2M1 ? launch_x_rows_to_f16(X, M, K, Xp, xrow, cnt, L.tiles, st)
                                     : launch_x_rows_repair(X, M, K, Xp, cnt, L.tiles, st);
     if (e != cudaSuccess) return e;
