@@ -75,7 +75,7 @@ typedef enum fp4_scale_dtype { FP4_SCALE_F32 = 0, FP4_SCALE_F16 = 1 } fp4_scale_
 /* GEMM engine selection for fp4_gemm_ex (fp4_gemm always uses AUTO). */
 typedef enum fp4_engine { FP4_ENGINE_AUTO = 0, FP4_ENGINE_DECODE = 1, FP4_ENGINE_TENSOR = 2 } fp4_engine;
 /* Output activation fused into the GEMM epilogue (fp4_gemm_act). */
-typedef enum fp4_act { FP4_ACT_NONE = 0, FP4_ACT_SILU = 1, FP4_ACT_GELU = 2 } fp4_act;
+typedef enum fp4_act { FP4_ACT_NONE = 0, FP4_ACT_SILU = 1, FP4_ACT_GELU = 2, FP4_ACT_SILU_GATE = 3 } fp4_act;
 
 /* Bits of the device status word. */
 #define FP4_DEV_NONFINITE_INPUT 0x1 /* NaN/Inf met in W or X                   */
@@ -245,10 +245,18 @@ FP4_API fp4_status fp4_gemm_ex(const uint16_t *X, const uint8_t *packed, const v
  *   Y[m,n] = bf16_rne( act( rho * sum_k X[m,k] * v(code[n,k]) * s[n,k/group] ) )
  *
  *   act  FP4_ACT_NONE: identity; FP4_ACT_SILU: y / (1 + exp(-y));
- *        FP4_ACT_GELU: y * (1 + erf(y / sqrt 2)) / 2.  Anything else returns
- *        FP4_ERR_INVALID_ARG.
- * Every engine and kernel supports it, with the other arguments as for
- * fp4_gemm_ex; act(y) is computed once per output after any split-K sum. */
+ *        FP4_ACT_GELU: y * (1 + erf(y / sqrt 2)) / 2;
+ *        FP4_ACT_SILU_GATE: gate and up projections fused in one call (the
+ *        MLP of the LLaMA-shaped workloads): the weight rows are
+ *        interleaved, row 2i the gate row and row 2i+1 the up row of output
+ *        column i (quantize [W_gate; W_up] with its rows interleaved that
+ *        way), N is even, and Y is [M][N/2] with
+ *          Y[m,i] = bf16_rne( silu(y[m,2i]) * y[m,2i+1] ),
+ *        y the product above; group 128 only (FP4_ERR_UNSUPPORTED_SHAPE
+ *        otherwise).  Anything else returns FP4_ERR_INVALID_ARG.
+ * Every engine and kernel supports NONE, SILU and GELU, with the other
+ * arguments as for fp4_gemm_ex; the group-128 kernels also SILU_GATE.  The
+ * activation is computed once per output after any split-K sum. */
 FP4_API fp4_status fp4_gemm_act(const uint16_t *X, const uint8_t *packed, const void *scales,
                         fp4_scale_dtype sdt, fp4_format fmt, int M, int N, int K, int group,
                         const float *x_scale, fp4_act act, uint16_t *Y, void *workspace, size_t ws_bytes,

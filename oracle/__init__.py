@@ -21,7 +21,7 @@ _HDR = os.path.join(_HERE, "fp4_oracle.h")
 _LIB = os.path.join(_HERE, "libfp4_oracle.so")
 
 E1M2, E2M1, E3M0, AUTO = 0, 1, 2, -1
-ACT_NONE, ACT_SILU, ACT_GELU = 0, 1, 2
+ACT_NONE, ACT_SILU, ACT_GELU, ACT_SILU_GATE = 0, 1, 2, 3
 SCALE_F32, SCALE_F16 = 0, 1
 FORMAT_NAMES = ("E1M2", "E2M1", "E3M0")
 
@@ -222,9 +222,20 @@ def activation(Y, act):
     raise OracleError("unknown activation %r" % (act,))
 
 
+def silu_gate(Y):
+    """Gate/up pairs of the fused MLP epilogue: column i of the result is
+    silu(Y[:, 2i]) * Y[:, 2i+1] (gate and up rows interleaved), in fp64."""
+    Y = np.asarray(Y, np.float64)
+    g, u = Y[:, 0::2], Y[:, 1::2]
+    with np.errstate(over="ignore"):
+        return g / (1.0 + np.exp(-g)) * u
+
+
 def gemm_act(X_bf16, packed, scales, fmt, group, act, rho=1.0):
-    """act(rho * X . dequant(W)^T) in fp64: gemm() followed by activation()."""
-    return activation(gemm(X_bf16, packed, scales, fmt, group, rho), act)
+    """act(rho * X . dequant(W)^T) in fp64: gemm() followed by activation(),
+    or by silu_gate() for ACT_SILU_GATE."""
+    Y = gemm(X_bf16, packed, scales, fmt, group, rho)
+    return silu_gate(Y) if act == ACT_SILU_GATE else activation(Y, act)
 
 
 def gemm_sampled(X_bf16, packed, scales, fmt, group, ms, ns, rho=1.0):

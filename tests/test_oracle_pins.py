@@ -523,6 +523,13 @@ def test_activation_pins(oracle_mod):
     Y = A.gemm(X, r["packed"], r["scales"], 1, 128, 0.5)
     np.testing.assert_array_equal(A.gemm_act(X, r["packed"], r["scales"], 1, 128, A.ACT_GELU, 0.5),
                                   A.activation(Y, A.ACT_GELU))
+    # gate/up pairs: silu(gate) * up, column i from rows 2i, 2i+1
+    P = np.array([[1.0, 2.0, math.log(3.0), 1.0, -3.0, 0.0]])
+    np.testing.assert_allclose(A.silu_gate(P), [[2.0 / (1.0 + math.exp(-1.0)), 0.75 * math.log(3.0), 0.0]],
+                               rtol=1e-14, atol=0)
+    G = A.gemm_act(X, r["packed"], r["scales"], 1, 128, A.ACT_SILU_GATE, 0.5)
+    assert G.shape == (3, 16)
+    np.testing.assert_array_equal(G, A.activation(Y[:, 0::2], A.ACT_SILU) * Y[:, 1::2])
 
 
 def test_golden_tiny_digest(oracle_mod):

@@ -272,11 +272,52 @@ def test_gemm_activation(fp4, oracle_mod, act, M, N, K, group, engine, splits):
     assert np.all(np.isfinite(Y.float().cpu().numpy()))
 
 
+@pytest.mark.parametrize("M,N,K,engine,splits", [
+    (4, 304, 1024, 1, 0),       # row-block decode kernel (pair in lane ^ 16)
+    (4, 304, 1024, 1, 1),       # streaming kernel, one CTA: whole tiles, 128-byte rows (pair in lane ^ 8)
+    (13, 304, 1024, 1, 148),    # streaming, two token tiles, every tile split (reducer quads)
+    (5, 600, 384, 1, 2),        # streaming, one-group chunks of 256 rows (pair in lane ^ 4) and a split tile
+    (40, 304, 1024, 1, 1),      # tensor-memory decode kernel, whole tiles (lane ^ 1)
+    (40, 304, 1024, 1, 0),      # tensor-memory decode kernel, split tiles (reducer quads)
+    (16, 304, 1024, 2, 0),      # tensor engine 16-token tile, split K over a cluster (quads)
+    (64, 304, 1024, 2, 1),      # tensor engine 64-token tile, one CTA per tile (lane ^ 1)
+    (200, 304, 1024, 2, 1),     # 128-token tile, f16 path, 16-byte output chunks
+])
+def test_gemm_silu_gate(fp4, oracle_mod, M, N, K, engine, splits):
+    """Gate and up projections fused in one call: rows 2i / 2i+1 are the gate
+    / up rows of output i, Y[m, i] = silu(y[m, 2i]) * y[m, 2i+1], in every
+    group-128 kernel's epilogue."""
+    W, X = synth.random_case(80 + M, N, K, M)
+    res = fp4.quantize(dev_f32(W), 128, 1)
+    xs = torch.tensor([1.25], dtype=torch.float32, device="cuda")
+    Y = fp4.gemm(dev_bf16(X), res["packed"], res["scales"], 1, 128, x_scale=xs, engine=engine, splits=splits,
+                 act=fp4.ACT_SILU_GATE)
+    assert tuple(Y.shape) == (M, N // 2)
+    Yref = oracle_mod.gemm_act(X, res["packed"].cpu().numpy(), res["scales"].cpu().numpy(), 1, 128,
+                               oracle_mod.ACT_SILU_GATE, 1.25)
+    assert rel_err(Y, Yref) <= TOL
+
+
+def test_gemm_silu_gate_limits(fp4):
+    """Gate/up pairs need an even row count and group 128."""
+    W, X = synth.random_case(90, 63, 256, 2)
+    res = fp4.quantize(dev_f32(W), 128, 1)
+    with pytest.raises(fp4.Fp4Error) as err:
+        fp4.gemm(dev_bf16(X), res["packed"], res["scales"], 1, 128, act=fp4.ACT_SILU_GATE,
+                 out=torch.empty((2, 31), dtype=torch.bfloat16, device="cuda"))
+    assert err.value.code == 2
+    W, X = synth.random_case(91, 64, 256, 2)
+    res = fp4.quantize(dev_f32(W), 64, 1)
+    with pytest.raises(fp4.Fp4Error) as err:
+        fp4.gemm(dev_bf16(X), res["packed"], res["scales"], 1, 64, act=fp4.ACT_SILU_GATE)
+    assert err.value.code == 2
+
+
 def test_gemm_activation_rejects_unknown(fp4):
     W, X = synth.random_case(70, 64, 256, 2)
     res = fp4.quantize(dev_f32(W), 128, 1)
     with pytest.raises(fp4.Fp4Error) as err:
-        fp4.gemm(dev_bf16(X), res["packed"], res["scales"], 1, 128, act=3)
+        fp4.gemm(dev_bf16(X), res["packed"], res["scales"], 1, 128, act=4)
     assert err.value.code == 1
 
 

@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(HERE, "libfp4w4a16.so")
 E1M2, E2M1, E3M0, AUTO = 0, 1, 2, -1
 SCALE_F32, SCALE_F16 = 0, 1
 ENGINE_AUTO, ENGINE_DECODE, ENGINE_TENSOR = 0, 1, 2
-ACT_NONE, ACT_SILU, ACT_GELU = 0, 1, 2
+ACT_NONE, ACT_SILU, ACT_GELU, ACT_SILU_GATE = 0, 1, 2, 3
 DEV_NONFINITE_INPUT, DEV_SCALE_OVERFLOW, DEV_WAIT_TIMEOUT, DEV_LAYOUT = 1, 2, 4, 8
 
 STATUS = {0: "FP4_OK", 1: "FP4_ERR_INVALID_ARG", 2: "FP4_ERR_UNSUPPORTED_SHAPE", 3: "FP4_ERR_MISALIGNED",
@@ -234,13 +234,14 @@ def gemm(X, packed, scales, fmt=E2M1, group=128, x_scale=None, out=None, engine=
     activations); a smaller one makes the automatic choice take the tensor
     engine's bf16 path.  ``engine``/``splits`` force an engine or a split
     count (0: automatic).  ``act``: ACT_NONE, ACT_SILU or ACT_GELU, applied
-    in the epilogue."""
+    in the epilogue, or ACT_SILU_GATE: rows 2i / 2i+1 of the weights are the
+    gate / up rows of output column i, and Y is [M][N/2]."""
     M, K = X.shape
     N = packed.shape[0]
     assert packed.shape[1] * 2 == K
     sdt = SCALE_F16 if scales.dtype == torch.float16 else SCALE_F32
     if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+        out = torch.empty((M, N // 2 if act == ACT_SILU_GATE else N), dtype=torch.bfloat16, device=X.device)
     L = lib()
     if workspace is None:
         need = L.fp4_gemm_workspace_size(M, N, K)

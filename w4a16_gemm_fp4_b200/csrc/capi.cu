@@ -323,7 +323,8 @@ fp4_status fp4_gemm_act(const uint16_t* X, const uint8_t* packed, const void* sc
                         uint16_t* Y, void* workspace, size_t ws_bytes, fp4_engine engine, int splits,
                         cudaStream_t stream) {
     if (M < 0) return FP4_ERR_INVALID_ARG;
-    if (act != FP4_ACT_NONE && act != FP4_ACT_SILU && act != FP4_ACT_GELU) return FP4_ERR_INVALID_ARG;
+    if (act != FP4_ACT_NONE && act != FP4_ACT_SILU && act != FP4_ACT_GELU && act != FP4_ACT_SILU_GATE)
+        return FP4_ERR_INVALID_ARG;
     fp4_status s = check_weights(packed, scales, sdt, fmt, N, K, group);
     if (s != FP4_OK) return s;
     if (engine != FP4_ENGINE_AUTO && engine != FP4_ENGINE_DECODE && engine != FP4_ENGINE_TENSOR)
@@ -334,8 +335,12 @@ fp4_status fp4_gemm_act(const uint16_t* X, const uint8_t* packed, const void* sc
     if (!aligned(Y, 16)) return FP4_ERR_MISALIGNED;
     if (x_scale && !aligned(x_scale, 4)) return FP4_ERR_MISALIGNED;
     if (workspace && !aligned(workspace, 16)) return FP4_ERR_MISALIGNED;
+    // gate/up pairs: interleaved rows (N even), group-128 kernels; Y has N/2 columns
+    const bool gated = act == FP4_ACT_SILU_GATE;
+    if (gated && (N % 2 != 0 || group != 128)) return FP4_ERR_UNSUPPORTED_SHAPE;
     // K = 0: every output is act(0) = 0 for the supported activations
-    if (K == 0) return cuda_status(cudaMemsetAsync(Y, 0, (size_t)M * N * sizeof(uint16_t), stream));
+    if (K == 0)
+        return cuda_status(cudaMemsetAsync(Y, 0, (size_t)M * (gated ? N / 2 : N) * sizeof(uint16_t), stream));
     if (!X) return FP4_ERR_INVALID_ARG;
     if (!aligned(X, 16)) return FP4_ERR_MISALIGNED;
     if ((const void*)Y == (const void*)X || (const void*)Y == (const void*)packed) return FP4_ERR_INVALID_ARG;

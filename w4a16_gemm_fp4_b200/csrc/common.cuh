@@ -173,7 +173,11 @@ __device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4 v, float sc) {
 // operators: the activation that follows the linear layer runs in the GEMM's
 // epilogue).  0: none; 1: SiLU y * sigmoid(y); 2: GeLU y * Phi(y), the erf
 // form.
-enum { kActNone = 0, kActSilu = 1, kActGelu = 2 };
+// 3: SiLU-gated pairs (SwiGLU with interleaved weights): rows 2i and 2i+1
+// of the weight matrix are the gate and up rows of output column i, and the
+// output holds N/2 columns y = silu(y[2i]) * y[2i+1] (silu_gate below).
+enum { kActNone = 0, kActSilu = 1, kActGelu = 2, kActSiluGate = 3 };
+__device__ __forceinline__ float silu_gate(float g, float u) { return g / (1.f + expf(-g)) * u; }
 __device__ __forceinline__ float apply_act(float y, int act) {
     if (act == kActSilu) return y / (1.f + expf(-y));
     if (act == kActGelu) return 0.5f * y * (1.f + erff(y * 0.70710678118654752f));

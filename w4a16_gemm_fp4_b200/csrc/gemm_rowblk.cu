@@ -347,9 +347,13 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
 #pragma unroll
             for (int w = 0; w < NW; ++w) sum += rd[((tt * NW + w) * 32 + l) * 4 + j];
             const int n = n0 + (l >> 2) + 8 * (j >> 1), m = 8 * tt + 2 * (l & 3) + (j & 1);
-            if (m < p.M && n < p.N) {
-                __nv_bfloat16 y = __float2bfloat16_rn(apply_act(rho * (kCvt ? row_f[m] * sum : sum), p.act));
-                p.Y[(size_t)m * p.N + n] = *reinterpret_cast<uint16_t*>(&y);
+            const float v = rho * (kCvt ? row_f[m] * sum : sum);
+            if (p.act == kActSiluGate) {
+                // row n ^ 1 (the other half of the gate/up pair) sits in lane ^ 16
+                const float w = __shfl_xor_sync(0xffffffffu, v, 16);
+                if (m < p.M && n + 1 < p.N && (n & 1) == 0) p.Y[(size_t)m * (p.N >> 1) + (n >> 1)] = bf16_bits(silu_gate(v, w));
+            } else if (m < p.M && n < p.N) {
+                p.Y[(size_t)m * p.N + n] = bf16_bits(apply_act(v, p.act));
             }
         }
     }

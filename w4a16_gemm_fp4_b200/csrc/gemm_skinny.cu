@@ -467,12 +467,23 @@ __global__ void __launch_bounds__(SkCfg<NT, CG>::THREADS, 1)
 #pragma unroll
                         for (int e = 0; e < 2; ++e) {
                             const int m = 8 * jn + 2 * t + e;
-                            if (m < p.M) {
-                                if (n0 + rA < p.N)
-                                    p.Y[(size_t)m * p.N + n0 + rA] = bf16_bits(apply_act(rho * tot[jn][e], p.act));
-                                if (n0 + rB < p.N)
-                                    p.Y[(size_t)m * p.N + n0 + rB] =
-                                        bf16_bits(apply_act(rho * tot[jn][2 + e], p.act));
+                            const float va = rho * tot[jn][e], vb = rho * tot[jn][2 + e];
+                            if (p.act == kActSiluGate) {
+                                // rows rA ^ 1 and rB ^ 1 are held by lane ^ 8 (128-byte
+                                // swizzle row order) or lane ^ 4 (64-byte)
+                                const int o = CG == 2 ? 8 : 4;
+                                const float wa = __shfl_xor_sync(0xffffffffu, va, o);
+                                const float wb = __shfl_xor_sync(0xffffffffu, vb, o);
+                                if (m < p.M && (rA & 1) == 0) {
+                                    const int NH = p.N >> 1;
+                                    if (n0 + rA + 1 < p.N)
+                                        p.Y[(size_t)m * NH + ((n0 + rA) >> 1)] = bf16_bits(silu_gate(va, wa));
+                                    if (n0 + rB + 1 < p.N)
+                                        p.Y[(size_t)m * NH + ((n0 + rB) >> 1)] = bf16_bits(silu_gate(vb, wb));
+                                }
+                            } else if (m < p.M) {
+                                if (n0 + rA < p.N) p.Y[(size_t)m * p.N + n0 + rA] = bf16_bits(apply_act(va, p.act));
+                                if (n0 + rB < p.N) p.Y[(size_t)m * p.N + n0 + rB] = bf16_bits(apply_act(vb, p.act));
                             }
                         }
                 }
@@ -528,6 +539,13 @@ __global__ void __launch_bounds__(SkCfg<NT, CG>::THREADS, 1)
                             }
                         }
                         const int m = qd / (TR / 4), n = n0 + (qd % (TR / 4)) * 4;
+                        if (p.act == kActSiluGate) {
+                            // the quad is two gate/up pairs
+                            uint16_t* dst = p.Y + (size_t)m * (p.N >> 1) + (n >> 1);
+                            if (n + 1 < p.N) dst[0] = bf16_bits(silu_gate(rho * sum.x, rho * sum.y));
+                            if (n + 3 < p.N) dst[1] = bf16_bits(silu_gate(rho * sum.z, rho * sum.w));
+                            continue;
+                        }
                         uint16_t* dst = p.Y + (size_t)m * p.N + n;
                         const uint32_t y01 = pack_bf16x2(apply_act(rho * sum.x, p.act), apply_act(rho * sum.y, p.act)),
                                        y23 = pack_bf16x2(apply_act(rho * sum.z, p.act), apply_act(rho * sum.w, p.act));

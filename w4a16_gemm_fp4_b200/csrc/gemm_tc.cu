@@ -160,6 +160,13 @@ __device__ __forceinline__ void cluster_reduce_store(const TcParams& p, uint32_t
                 a.z *= f;
                 a.w *= f;
             }
+            if (p.act == kActSiluGate) {
+                // 4 rows = 2 gate/up pairs
+                uint16_t* dst = p.Y + (size_t)m * (p.N >> 1) + (n >> 1);
+                if (n + 1 < p.N) dst[0] = bf16_bits(silu_gate(rho * a.x, rho * a.y));
+                if (n + 3 < p.N) dst[1] = bf16_bits(silu_gate(rho * a.z, rho * a.w));
+                continue;
+            }
             __nv_bfloat16 y[4] = {__float2bfloat16_rn(apply_act(rho * a.x, p.act)),
                                   __float2bfloat16_rn(apply_act(rho * a.y, p.act)),
                                   __float2bfloat16_rn(apply_act(rho * a.z, p.act)),
@@ -788,7 +795,17 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
 #pragma unroll
             for (int j = 0; j < C::FCOLS; ++j) ep[(cb + j) * 128 + r] = rho * tot[j];
         } else if (p.splits == 1) {
-            if (ok && nvalid) {
+            if (ok && p.act == kActSiluGate) {
+                // row n ^ 1, the other half of the gate/up pair, is lane ^ 1
+#pragma unroll
+                for (int j = 0; j < C::FCOLS; ++j) {
+                    const int m = m0 + cb + j;
+                    const float v = rho * (F16 ? tot[j] * xfw[j] : tot[j]);
+                    const float w = __shfl_xor_sync(0xffffffffu, v, 1);
+                    if (m < p.M && (n & 1) == 0 && n + 1 < p.N)
+                        p.Y[(size_t)m * (p.N >> 1) + (n >> 1)] = bf16_bits(silu_gate(v, w));
+                }
+            } else if (ok && nvalid) {
 #pragma unroll
                 for (int j = 0; j < C::FCOLS; ++j) {
                     const int m = m0 + cb + j;
@@ -832,7 +849,13 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
 #pragma unroll
             for (int u = 0; u < kC; ++u) {
                 const int c = c0 + u * kT, j = c >> 4, n = n0 + (c & 15) * 8, m = m0 + j;
-                if (m < p.M && n < p.N) {
+                if (m < p.M && n < p.N && p.act == kActSiluGate) {
+                    // 8 rows = 4 gate/up pairs -> 4 outputs (N % 8 == 0 on this path)
+                    uint2 o;
+                    o.x = pack_bf16x2(silu_gate(a[u].x * f[u], a[u].y * f[u]), silu_gate(a[u].z * f[u], a[u].w * f[u]));
+                    o.y = pack_bf16x2(silu_gate(b[u].x * f[u], b[u].y * f[u]), silu_gate(b[u].z * f[u], b[u].w * f[u]));
+                    *reinterpret_cast<uint2*>(p.Y + (size_t)m * (p.N >> 1) + (n >> 1)) = o;
+                } else if (m < p.M && n < p.N) {
                     uint4 o;
                     o.x = pack_bf16x2(apply_act(a[u].x * f[u], p.act), apply_act(a[u].y * f[u], p.act));
                     o.y = pack_bf16x2(apply_act(a[u].z * f[u], p.act), apply_act(a[u].w * f[u], p.act));

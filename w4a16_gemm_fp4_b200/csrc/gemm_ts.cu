@@ -393,7 +393,17 @@ __global__ void __launch_bounds__(TsCfg<BT, CG>::THREADS, 1)
             const int n = t * C::BW + r;
             if (seg_g0 == 0 && g == G - 1) {
                 // the whole tile is this CTA's: store it
-                if (ok && n < p.N) {
+                if (p.act == kActSiluGate) {
+                    // row n ^ 1, the other half of the gate/up pair, is lane ^ 1
+#pragma unroll
+                    for (int k = 0; k < C::FCOLS; ++k) {
+                        const int m = cb + k;
+                        const float v = rho * tot[k] * xrw[k];
+                        const float w = __shfl_xor_sync(0xffffffffu, v, 1);
+                        if (ok && m < p.M && (n & 1) == 0 && n + 1 < p.N)
+                            p.Y[(size_t)m * (p.N >> 1) + (n >> 1)] = bf16_bits(silu_gate(v, w));
+                    }
+                } else if (ok && n < p.N) {
 #pragma unroll
                     for (int k = 0; k < C::FCOLS; ++k) {
                         const int m = cb + k;
@@ -459,6 +469,15 @@ __global__ void __launch_bounds__(TsCfg<BT, CG>::THREADS, 1)
                             if (qd >= BT * 32) continue;
                             const int m = qd >> 5, n4 = t * C::BW + (qd & 31) * 4;
                             const float4 a = acc[qb];
+                            if (p.act == kActSiluGate) {
+                                // the quad is two gate/up pairs
+                                if (m < p.M) {
+                                    uint16_t* dst = p.Y + (size_t)m * (p.N >> 1) + (n4 >> 1);
+                                    if (n4 + 1 < p.N) dst[0] = bf16_bits(silu_gate(rho * a.x, rho * a.y));
+                                    if (n4 + 3 < p.N) dst[1] = bf16_bits(silu_gate(rho * a.z, rho * a.w));
+                                }
+                                continue;
+                            }
                             if (m < p.M && n4 < p.N) {
                                 const uint32_t y01 = pack_bf16x2(apply_act(rho * a.x, p.act),
                                                                  apply_act(rho * a.y, p.act)),
