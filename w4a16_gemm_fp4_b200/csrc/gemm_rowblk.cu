@@ -164,8 +164,6 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
         }
     }
     __syncthreads();
-    pdl_wait();  // inputs may come from the previous kernel in the stream
-    pdl_launch_dependents();
 
     int issued = 0;  // blocks whose copies were issued (thread 0 only)
     auto issue = [&](int it) {  // bulk copies of block `it` of this CTA into buffer it % nbuf
@@ -183,8 +181,14 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
                       (uint32_t)sc_bytes, &bar[b]);
         issued = it + 1;
     };
+    // The first buffers' copies go out before the dependency wait as well:
+    // codes and scales are inputs that no kernel still running may write
+    // (the previous kernel in the stream triggers this launch early only
+    // when it is one of these GEMMs), and the buffers are free at entry.
     if (threadIdx.x == 0)
         for (int it = 0; it < nbuf && it < iters; ++it) issue(it);
+    pdl_wait();  // the activations, rho and the output may involve the previous kernel
+    pdl_launch_dependents();
 
     {
         // The activations, once per CTA, in operand form at row pitch XP:

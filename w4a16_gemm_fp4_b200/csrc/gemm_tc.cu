@@ -13,10 +13,11 @@
 // Two kernels, both with the product computed transposed, D[n][m] = W . X^T:
 // the 128 weight rows of a CTA tile (MMA M) map onto the 128 TMEM lanes, so
 // the per-row group scale is a per-lane scalar; BT activation rows are MMA N.
-//   gemm_tc_kernel<BT>        groups of 32 or 64: 64-k stages, four TMEM
+//   gemm_tc_kernel<BT, ACT>   groups of 32 or 64: 64-k stages, four TMEM
 //                             group accumulators;
-//   gemm_tcg_kernel<BT, F16>  group 128: one group per stage, one TMEM
-//                             accumulator per stage (below).
+//   gemm_tcg_kernel<BT, F16, ACT>  group 128: one group per stage, one
+//                             TMEM accumulator per stage (below); ACT
+//                             compiles in the output activations.
 //
 // Warp roles (2 + DQW + NF warps):
 //   warp 0       TMA producer: activation tiles (128-byte swizzle) and the
@@ -118,7 +119,7 @@ __device__ __forceinline__ uint4 lds128_tc(const void* p) {
 // loads from every rank before the first add, so a slice costs a few round
 // trips to the other CTAs rather than one per output.
 template <int BT>
-__device__ __forceinline__ void cluster_reduce_store(const TcParams& p, uint32_t part, int n0, int m0) {
+__device__ __forceinline__ void cluster_reduce_store(const TcParams& p, uint32_t part, int n0, int m0, int act) {
     constexpr int kQ = 1;
     cluster_sync();
     const int rank = (int)cluster_ctarank();
@@ -160,17 +161,17 @@ __device__ __forceinline__ void cluster_reduce_store(const TcParams& p, uint32_t
                 a.z *= f;
                 a.w *= f;
             }
-            if (p.act == kActSiluGate) {
+            if (act == kActSiluGate) {
                 // 4 rows = 2 gate/up pairs
                 uint16_t* dst = p.Y + (size_t)m * (p.N >> 1) + (n >> 1);
                 if (n + 1 < p.N) dst[0] = bf16_bits(silu_gate(rho * a.x, rho * a.y));
                 if (n + 3 < p.N) dst[1] = bf16_bits(silu_gate(rho * a.z, rho * a.w));
                 continue;
             }
-            __nv_bfloat16 y[4] = {__float2bfloat16_rn(apply_act(rho * a.x, p.act)),
-                                  __float2bfloat16_rn(apply_act(rho * a.y, p.act)),
-                                  __float2bfloat16_rn(apply_act(rho * a.z, p.act)),
-                                  __float2bfloat16_rn(apply_act(rho * a.w, p.act))};
+            __nv_bfloat16 y[4] = {__float2bfloat16_rn(apply_act(rho * a.x, act)),
+                                  __float2bfloat16_rn(apply_act(rho * a.y, act)),
+                                  __float2bfloat16_rn(apply_act(rho * a.z, act)),
+                                  __float2bfloat16_rn(apply_act(rho * a.w, act))};
             uint16_t* dst = p.Y + (size_t)m * p.N + n;
             if (vec_store && n + 3 < p.N) {
                 uint2 w;
@@ -187,10 +188,11 @@ __device__ __forceinline__ void cluster_reduce_store(const TcParams& p, uint32_t
     cluster_sync();  // no CTA leaves while its partials are being read
 }
 
-template <int BT>
+template <int BT, bool ACT>
 __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, TcParams p) {
     using C = TcCfg<BT>;
+    const int act = ACT ? p.act : kActNone;  // activation epilogues: own instantiation
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* as = smem;                         // AST x ABYTES: dequantized weight tiles
@@ -461,7 +463,7 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
                 for (int j = 0; j < C::FCOLS; ++j) {
                     const int m = m0 + cb + j;
                     if (m < p.M) {
-                        __nv_bfloat16 y = __float2bfloat16_rn(apply_act(rho * tot[j], p.act));
+                        __nv_bfloat16 y = __float2bfloat16_rn(apply_act(rho * tot[j], act));
                         p.Y[(size_t)m * p.N + n] = *reinterpret_cast<uint16_t*>(&y);
                     }
                 }
@@ -477,7 +479,7 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
         }
     }
 
-    if (p.splits > 1) cluster_reduce_store<BT>(p, smem_u32(smem), n0, m0);
+    if (p.splits > 1) cluster_reduce_store<BT>(p, smem_u32(smem), n0, m0, act);
 
     tc_fence_before();
     __syncthreads();
@@ -532,10 +534,13 @@ struct TgCfg {
     static_assert(BT * 128 * 4 <= STG * ABYTES, "split-K partials overlay the dequantized tiles");
 };
 
-template <int BT, bool F16>
+template <int BT, bool F16, bool ACT>
 __global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
     gemm_tcg_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, TcParams p) {
     using C = TgCfg<BT>;
+    // The activation epilogues are a separate instantiation: compiled into
+    // the plain kernel, they cost the 128-token tile its register budget.
+    const int act = ACT ? p.act : kActNone;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     if (C::SLACK == 0 && smem != smem_raw) {
@@ -592,13 +597,28 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    pdl_wait();  // inputs may come from the previous kernel in the stream
+    // The packed codes are inputs that no kernel still running may write (the
+    // previous kernel in the stream triggers this launch early only when it
+    // is one of these GEMMs), so on the small token tiles (one wave of CTAs,
+    // which overlaps the previous kernel's tail) the first ring-full of them
+    // goes out before the dependency wait; the activations follow after it.
+    // (On the 128-token tile, many waves deep, a burst of code copies ahead
+    // of the first activation copy measured slower: 866 -> 771 TFLOP/s.)
+    const int wpre = !C::kPair ? 0 : (nkb < C::WST ? nkb : C::WST);
+    if (warp == 0 && elect_one()) {
+        for (int j = 0; j < wpre; ++j) {
+            mbar_arrive_expect_tx(&wfull[j], C::WBYTES);
+            tma_load_2d(wsr + j * C::WBYTES, &tmW, (kb0 + j) * (C::KB / 2), n0, &wfull[j]);
+        }
+    }
+    __syncwarp();
+    pdl_wait();  // the activations, rho, row factors and the output involve the previous kernel
     pdl_launch_dependents();
 
     if (warp == 0) {
         // -------------------------------------------------------- producer
         if (elect_one()) {
-            int xi = 0, wj = 0;
+            int xi = 0, wj = wpre;
             bool ok = true;
             uint64_t t_last = globaltimer_ns();
             while (ok && (xi < nkb || wj < nkb)) {
@@ -795,7 +815,7 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
 #pragma unroll
             for (int j = 0; j < C::FCOLS; ++j) ep[(cb + j) * 128 + r] = rho * tot[j];
         } else if (p.splits == 1) {
-            if (ok && p.act == kActSiluGate) {
+            if (ok && act == kActSiluGate) {
                 // row n ^ 1, the other half of the gate/up pair, is lane ^ 1
 #pragma unroll
                 for (int j = 0; j < C::FCOLS; ++j) {
@@ -811,7 +831,7 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
                     const int m = m0 + cb + j;
                     if (m < p.M) {
                         const float t = F16 ? tot[j] * xfw[j] : tot[j];
-                        __nv_bfloat16 y = __float2bfloat16_rn(apply_act(rho * t, p.act));
+                        __nv_bfloat16 y = __float2bfloat16_rn(apply_act(rho * t, act));
                         p.Y[(size_t)m * p.N + n] = *reinterpret_cast<uint16_t*>(&y);
                     }
                 }
@@ -826,7 +846,7 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
         }
     }
 
-    if (p.splits > 1) cluster_reduce_store<BT>(p, smem_u32(smem), n0, m0);
+    if (p.splits > 1) cluster_reduce_store<BT>(p, smem_u32(smem), n0, m0, act);
     if (wide && warp >= C::DQ0) {
         // 16-byte output chunks (8 weight rows of one token) over the dequant
         // and fold warps: the f16 path's token factor, bf16x2 converts and
@@ -849,7 +869,7 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
 #pragma unroll
             for (int u = 0; u < kC; ++u) {
                 const int c = c0 + u * kT, j = c >> 4, n = n0 + (c & 15) * 8, m = m0 + j;
-                if (m < p.M && n < p.N && p.act == kActSiluGate) {
+                if (m < p.M && n < p.N && act == kActSiluGate) {
                     // 8 rows = 4 gate/up pairs -> 4 outputs (N % 8 == 0 on this path)
                     uint2 o;
                     o.x = pack_bf16x2(silu_gate(a[u].x * f[u], a[u].y * f[u]), silu_gate(a[u].z * f[u], a[u].w * f[u]));
@@ -857,10 +877,10 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
                     *reinterpret_cast<uint2*>(p.Y + (size_t)m * (p.N >> 1) + (n >> 1)) = o;
                 } else if (m < p.M && n < p.N) {
                     uint4 o;
-                    o.x = pack_bf16x2(apply_act(a[u].x * f[u], p.act), apply_act(a[u].y * f[u], p.act));
-                    o.y = pack_bf16x2(apply_act(a[u].z * f[u], p.act), apply_act(a[u].w * f[u], p.act));
-                    o.z = pack_bf16x2(apply_act(b[u].x * f[u], p.act), apply_act(b[u].y * f[u], p.act));
-                    o.w = pack_bf16x2(apply_act(b[u].z * f[u], p.act), apply_act(b[u].w * f[u], p.act));
+                    o.x = pack_bf16x2(apply_act(a[u].x * f[u], act), apply_act(a[u].y * f[u], act));
+                    o.y = pack_bf16x2(apply_act(a[u].z * f[u], act), apply_act(a[u].w * f[u], act));
+                    o.z = pack_bf16x2(apply_act(b[u].x * f[u], act), apply_act(b[u].y * f[u], act));
+                    o.w = pack_bf16x2(apply_act(b[u].z * f[u], act), apply_act(b[u].w * f[u], act));
                     *reinterpret_cast<uint4*>(p.Y + (size_t)m * p.N + n) = o;
                 }
             }
@@ -956,7 +976,9 @@ static cudaError_t launch_tc_bt(const CUtensorMap& mx, const CUtensorMap& mw, co
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BT, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(gemm_tc_kernel<BT, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
@@ -975,7 +997,8 @@ static cudaError_t launch_tc_bt(const CUtensorMap& mx, const CUtensorMap& mw, co
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BT>, mx, mw, p);
+    cudaError_t e = p.act != kActNone ? cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BT, true>, mx, mw, p)
+                                      : cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BT, false>, mx, mw, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -1082,7 +1105,10 @@ static cudaError_t launch_tcg_bt(const CUtensorMap& mx, const CUtensorMap& mw, c
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_tcg_kernel<BT, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        cudaError_t e = cudaFuncSetAttribute(gemm_tcg_kernel<BT, F16, false>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(gemm_tcg_kernel<BT, F16, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
@@ -1100,7 +1126,8 @@ static cudaError_t launch_tcg_bt(const CUtensorMap& mx, const CUtensorMap& mw, c
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_tcg_kernel<BT, F16>, mx, mw, p);
+    cudaError_t e = p.act != kActNone ? cudaLaunchKernelEx(&cfg, gemm_tcg_kernel<BT, F16, true>, mx, mw, p)
+                                      : cudaLaunchKernelEx(&cfg, gemm_tcg_kernel<BT, F16, false>, mx, mw, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
