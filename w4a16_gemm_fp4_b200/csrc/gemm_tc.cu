@@ -599,12 +599,9 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
     const uint32_t tmem = *tmem_slot;
     // The packed codes are inputs that no kernel still running may write (the
     // previous kernel in the stream triggers this launch early only when it
-    // is one of these GEMMs), so on the small token tiles (one wave of CTAs,
-    // which overlaps the previous kernel's tail) the first ring-full of them
-    // goes out before the dependency wait; the activations follow after it.
-    // (On the 128-token tile, many waves deep, a burst of code copies ahead
-    // of the first activation copy measured slower: 866 -> 771 TFLOP/s.)
-    const int wpre = !C::kPair ? 0 : (nkb < C::WST ? nkb : C::WST);
+    // is one of these GEMMs), so the first ring-full of them goes out before
+    // the dependency wait; the activations follow after it.
+    const int wpre = nkb < C::WST ? nkb : C::WST;
     if (warp == 0 && elect_one()) {
         for (int j = 0; j < wpre; ++j) {
             mbar_arrive_expect_tx(&wfull[j], C::WBYTES);
