@@ -204,19 +204,32 @@ FP4_API fp4_status fp4_preshift_calibrate_noalloc(const uint16_t *X, int M, int 
  *            in shared memory.  Every bf16 activation is accepted.  With the
  *            automatic engine a workspace that is too small (or NULL) falls
  *            back to the tensor engine's bf16 path.
- * Engines (fp4_gemm_engine_for reports the choice): at group 128 M <= 64,
- * and at groups 32/64 M <= 8, use the decode engine; larger M uses the
- * tensor engine (TMA-staged tiles dequantized in shared memory, tcgen05
- * MMAs into tensor memory, one group per pipeline stage).  The group-128
- * decode engine runs one persistent CTA per SM over an even split of all
- * (row tile, 16 KB code chunk) units, streamed by TMA; a tile split between
- * CTAs is summed by the CTA that completes it, in CTA order, so the result
- * does not depend on timing.  For M <= 16 the codes convert in registers
- * (hardware e2m1 -> f16 for E2M1, exact bf16 bit placement otherwise) into
- * warp-level MMAs; for 16 < M <= 64 dequantize warps write them to tensor
- * memory as the A operand of tcgen05 MMAs.  Each group scale is applied in
- * fp32.  Groups 32/64 use warp-level MMAs over a lookup-table
- * dequantization (no workspace).
+ * Engines (fp4_gemm_engine_for reports the choice).  Group 128: the decode
+ * engine for M <= 8, and for 9 <= M <= 16 where the row-block kernel keeps
+ * two block buffers (shared-memory fit of the staged activations); the
+ * tensor engine otherwise.  Groups 32/64: the decode engine for M <= 8.
+ * The group-128 decode engine has three kernels:
+ *   - row-block (M <= 16, the activations [M][K] staged once per CTA in
+ *     shared memory): each CTA takes whole 16-row blocks over all of K,
+ *     bulk-copied; codes convert in registers (hardware e2m1 -> f16 for
+ *     E2M1, exact bf16 bit placement otherwise) into warp-level MMAs.  No
+ *     workspace.  Used when splits == 0 and the activations fit;
+ *   - streaming (M <= 16): one persistent CTA per SM over an even split of
+ *     all (row tile, 16 KB code chunk) units, streamed by TMA; a tile split
+ *     between CTAs is summed by the CTA that completes it, in CTA order, so
+ *     the result does not depend on timing.  Needs the workspace;
+ *   - tensor-memory (17 <= M <= 64, on request only): dequantize warps
+ *     write the codes to tensor memory as the A operand of tcgen05 MMAs.
+ * The tensor engine stages TMA tiles, dequantizes them in shared memory and
+ * runs tcgen05 MMAs into tensor memory, one group per pipeline stage.  Each
+ * group scale is applied in fp32.  Groups 32/64 decode through a lookup
+ * table into warp-level MMAs (no workspace).
+ * Stream order: the GEMM kernels are launched as programmatic dependents
+ * and start copying `packed` and `scales` before the kernel ahead of them
+ * in the stream has finished; X, x_scale and Y are touched only after it
+ * has.  Codes and scales written by the kernel directly ahead of a GEMM
+ * call must therefore be separated from it by another stream operation
+ * (any other kernel, copy or memset); fp4_quantize ends with such a launch.
  * Device status: FP4_DEV_WAIT_TIMEOUT, FP4_DEV_LAYOUT.
  * ---------------------------------------------------------------------- */
 FP4_API size_t fp4_gemm_workspace_size(int M, int N, int K);

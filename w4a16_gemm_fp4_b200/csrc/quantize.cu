@@ -339,6 +339,13 @@ size_t quantize_ws_bytes(long long total, bool search, bool want_sse) {
     return (size_t)quantize_grid_blocks(total) * 24 * sizeof(double);
 }
 
+// Launched after the packing pass.  The GEMM kernels start copying packed
+// codes and scales before the kernel ahead of them in the stream has
+// finished (programmatic dependent launch); with this empty launch in
+// between, a GEMM that follows fp4_quantize directly reads codes whose
+// kernel completed a full kernel boundary earlier.
+__global__ void stream_boundary_kernel() {}
+
 cudaError_t launch_quantize(const float* W, int N, int K, int group, int fmt, int bias_search,
                             const int8_t* shift, int sdt, uint8_t* packed, void* scales, int32_t* choice,
                             double* sse, void* ws, const FmtTables& tabs, int* status, cudaStream_t st) {
@@ -369,6 +376,7 @@ cudaError_t launch_quantize(const float* W, int N, int K, int group, int fmt, in
         quantize_kernel<<<pblocks, kQuantThreads, 0, st>>>(p, tabs, f0, 0, nullptr, choice, sse ? wsd : nullptr);
         if (sse) sse_single_finalize_kernel<<<1, 32, 0, st>>>(wsd, pblocks, f0, 0, sse);
     }
+    stream_boundary_kernel<<<1, 32, 0, st>>>();
     return cudaGetLastError();
 }
 
