@@ -23,6 +23,7 @@ _LIB = os.path.join(_HERE, "libfp4_oracle.so")
 E1M2, E2M1, E3M0, AUTO = 0, 1, 2, -1
 ACT_NONE, ACT_SILU, ACT_GELU, ACT_SILU_GATE = 0, 1, 2, 3
 SCALE_F32, SCALE_F16 = 0, 1
+GRAN_GROUP, GRAN_CHANNEL, GRAN_HEAD = 0, 1, 2
 FORMAT_NAMES = ("E1M2", "E2M1", "E3M0")
 
 _ERRORS = {1: "invalid argument", 2: "non-finite input", 3: "stored scale not finite", 4: "allocation failed"}
@@ -69,6 +70,11 @@ def _L():
             "orc_gemm_sampled": (i, [P, P, P, i, i, i, i, i, i, f, i, P, P, P]),
             "orc_preshift_calibrate": (i, [P, i, i, P, P]),
             "orc_preshift_apply": (i, [P, i, i, P, f, P]),
+            "orc_block_count": (i, [i, i, i, i, i]),
+            "orc_quantize_blocks": (i, [P, i, i, i, i, i, i, i, P, P, i, P, P, P, P]),
+            "orc_act_quantize": (i, [P, i, i, P, f, i, i, P, P]),
+            "orc_gemm_w4a4": (i, [P, i, f, P, P, i, i, i, i, i, i, P]),
+            "orc_gemm_w4a4_sampled": (i, [P, i, f, P, P, i, i, i, i, i, i, i, P, P, P]),
             "orc_num_threads": (i, []),
             "orc_set_num_threads": (None, [i]),
         }
@@ -269,3 +275,76 @@ def preshift_apply(X_bf16, shift, rho):
     Xt = np.zeros((M, K), np.uint16)
     _check(_L().orc_preshift_apply(_p(X), M, K, _p(shift), float(rho), _p(Xt)))
     return Xt
+
+
+def block_count(N, K, group, gran, heads=0):
+    return _L().orc_block_count(N, K, group, gran, heads)
+
+
+def quantize_blocks(W, group, gran, fmt, j=0, heads=0, shift=None, scale_dtype="f16", jforce=None):
+    """Quantize with the scale's absmax taken over a block (reading R11):
+    GRAN_GROUP (group elements of a row), GRAN_CHANNEL (a row) or GRAN_HEAD
+    (N/heads rows).  j = None searches the bias index per block; jforce
+    (int8 [blocks]) imposes one per block.  Scales come out in the
+    [N][K/group] layout, a block's scale in every slot it covers.
+
+    Returns dict(packed, scales, jmap int8 [blocks], sse float)."""
+    W = np.ascontiguousarray(W, np.float32)
+    N, K = W.shape
+    sdt = _sdt(scale_dtype)
+    nb = block_count(N, K, group, gran, heads)
+    packed = np.zeros((N, K // 2), np.uint8)
+    scales = np.zeros((N, K // group), np.float16 if sdt else np.float32)
+    jmap = np.zeros(max(nb, 0), np.int8)
+    jf = None if jforce is None else np.ascontiguousarray(jforce, np.int8)
+    if jf is not None:
+        assert jf.shape == (nb,)
+    sse = np.zeros(1, np.float64)
+    s = _shift_arr(shift, K)
+    _check(_L().orc_quantize_blocks(_p(W), N, K, group, gran, heads, fmt, -1 if j is None else j, _p(jf), _p(s),
+                                    sdt, _p(packed), _p(scales), _p(jmap), _p(sse)))
+    return {"packed": packed, "scales": scales, "jmap": jmap, "sse": float(sse[0])}
+
+
+def act_quantize(X_bf16, rho, fmt=E2M1, j=0, shift=None):
+    """4-bit activation codes with the pre-shifted bias (reading R10).
+
+    Returns (packed uint8 [M][K/2], s_a float32): X' = X * 2^-shift coded
+    against the per-tensor scale s_a = fl32(fl32(rho * c_j) / Qmax)."""
+    X = np.ascontiguousarray(X_bf16, np.uint16)
+    M, K = X.shape
+    packed = np.zeros((M, K // 2), np.uint8)
+    s_a = np.zeros(1, np.float32)
+    s = _shift_arr(shift, K)
+    _check(_L().orc_act_quantize(_p(X), M, K, _p(s), float(rho), fmt, j, _p(packed), _p(s_a)))
+    return packed, np.float32(s_a[0])
+
+
+def gemm_w4a4(apacked, afmt, s_a, packed, scales, fmt, group):
+    """Y = s_a * v_a(A) . dequant(W)^T in fp64 (reading R10)."""
+    apacked = np.ascontiguousarray(apacked, np.uint8)
+    packed = np.ascontiguousarray(packed, np.uint8)
+    scales = np.ascontiguousarray(scales)
+    M, K = apacked.shape[0], apacked.shape[1] * 2
+    N = packed.shape[0]
+    assert packed.shape[1] * 2 == K
+    sdt = SCALE_F16 if scales.dtype == np.float16 else SCALE_F32
+    Y = np.zeros((M, N), np.float64)
+    _check(_L().orc_gemm_w4a4(_p(apacked), afmt, float(s_a), _p(packed), _p(scales), sdt, fmt, M, N, K, group,
+                              _p(Y)))
+    return Y
+
+
+def gemm_w4a4_sampled(apacked, afmt, s_a, packed, scales, fmt, group, ms, ns):
+    apacked = np.ascontiguousarray(apacked, np.uint8)
+    packed = np.ascontiguousarray(packed, np.uint8)
+    scales = np.ascontiguousarray(scales)
+    M, K = apacked.shape[0], apacked.shape[1] * 2
+    N = packed.shape[0]
+    ms = np.ascontiguousarray(ms, np.int32)
+    ns = np.ascontiguousarray(ns, np.int32)
+    out = np.zeros(len(ms), np.float64)
+    sdt = SCALE_F16 if scales.dtype == np.float16 else SCALE_F32
+    _check(_L().orc_gemm_w4a4_sampled(_p(apacked), afmt, float(s_a), _p(packed), _p(scales), sdt, fmt, M, N, K,
+                                      group, len(ms), _p(ms), _p(ns), _p(out)))
+    return out

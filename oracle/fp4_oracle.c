@@ -44,6 +44,20 @@
  *  R6 pre-shift: c_k = max_m |X[m,k]|, rho = max_k c_k (1 if all zero),
  *     e_k = ceil(log2(c_k / rho)) clamped to [-126, 0] (0 when c_k == 0);
  *     W' = W * 2^e_k;  X~ = bf16(fl32(fl32(X * 2^-e_k) / rho));  Y *= rho.
+ *  R10 4-bit activations with the pre-shifted bias: the activation of
+ *     channel k is clipped to rho * 2^e_k (the calibration's per-tensor
+ *     real factor times the channel's power of two).  The power of two goes
+ *     into the weights (R6), so what is quantized is X' = fl32(X * 2^-e_k)
+ *     with ONE per-tensor scale s_a = fl32(fl32(rho * c_j) / Qmax) kept in
+ *     fp32 (R3 with A = rho); codes by R4 from q = fl32(X' / s_a).  The
+ *     product takes both scales out of the low-bit sum:
+ *       Y[m,n] = s_a * sum_k v_a(a[m,k]) * v(w[n,k]) * s[n, k/g].
+ *  R11 granularity: the absmax A of R3 is taken over a block, either g
+ *     consecutive elements of a row (group), a whole row (output channel),
+ *     or N/heads consecutive rows (an attention head); the block's scale is
+ *     stored in every group slot it covers.  Per-block search: each block
+ *     takes the bias index j minimising its own SSE (fp64, first strict
+ *     minimum, j ascending); the format stays per tensor.
  *
  * Build: gcc -O2 -fopenmp -ffp-contract=off -fno-fast-math -shared -fPIC.
  * float arithmetic below is IEEE binary32 with round-to-nearest-even
@@ -396,6 +410,225 @@ int orc_gemm_sampled(const uint16_t *X, const uint8_t *packed, const void *scale
 #pragma omp parallel for schedule(static)
     for (int i = 0; i < count; ++i)
         out[i] = gemm_one(X, packed, scales, sdt, fmt, K, g, (double)rho, ms[i], ns[i]);
+    return 0;
+}
+
+/* ---------------------------------------------------- granularity (R11) */
+
+int orc_block_count(int N, int K, int g, int gran, int heads)
+{
+    if (gran == ORC_GRAN_GROUP) return g > 0 ? N * (K / g) : 0;
+    if (gran == ORC_GRAN_CHANNEL) return N;
+    if (gran == ORC_GRAN_HEAD) return heads;
+    return 0;
+}
+
+/* Rows [r0, r1) x columns [k0, k1) of block b. */
+static void block_extent(int b, int N, int K, int g, int gran, int heads, int *r0, int *r1, int *k0,
+                         int *k1)
+{
+    if (gran == ORC_GRAN_GROUP) {
+        int G = K / g;
+        *r0 = b / G;
+        *r1 = *r0 + 1;
+        *k0 = (b % G) * g;
+        *k1 = *k0 + g;
+    } else if (gran == ORC_GRAN_CHANNEL) {
+        *r0 = b;
+        *r1 = b + 1;
+        *k0 = 0;
+        *k1 = K;
+    } else {
+        int R = N / heads;
+        *r0 = b * R;
+        *r1 = *r0 + R;
+        *k0 = 0;
+        *k1 = K;
+    }
+}
+
+/* W'[r,k] = W[r,k] * 2^shift[k] (reading R6). */
+static float folded(const float *W, int K, const int8_t *shift, int r, int k)
+{
+    float w = W[(size_t)r * K + k];
+    return shift ? w * pow2f(shift[k]) : w;
+}
+
+/* One block with bias index j: its scale, and its SSE (elements in
+ * row-major order); codes written when packed != NULL. */
+static int block_pass(const float *W, int K, const int8_t *shift, int r0, int r1, int k0, int k1,
+                      float A, int fmt, int j, int sdt, uint8_t *packed, float *s_out, uint32_t *raw,
+                      double *sse_out)
+{
+    double mags[8], qmax_d;
+    orc_format_table(fmt, mags, &qmax_d);
+    float s;
+    if (group_scale(A, orc_bias_factor(j), (float)qmax_d, sdt, &s, raw) != 0) return ORC_ERR_SCALE;
+    double sse = 0.0;
+    for (int r = r0; r < r1; ++r)
+        for (int k = k0; k < k1; ++k) {
+            float w = folded(W, K, shift, r, k);
+            int idx = 0;
+            if (s != 0.0f) {
+                float q = w / s;
+                idx = orc_nearest_index(fabs((double)q), mags);
+            }
+            int sign = signbit(w) ? 1 : 0;
+            double v = sign ? -mags[idx] : mags[idx];
+            double diff = (double)w - v * (double)s;
+            sse += diff * diff;
+            if (packed) {
+                uint8_t *byte = &packed[(size_t)r * (K / 2) + (k >> 1)];
+                int code = (sign << 3) | idx;
+                if ((k & 1) == 0) *byte = (uint8_t)((*byte & 0xf0u) | code);
+                else *byte = (uint8_t)((*byte & 0x0fu) | (code << 4));
+            }
+        }
+    *s_out = s;
+    *sse_out = sse;
+    return 0;
+}
+
+int orc_quantize_blocks(const float *W, int N, int K, int g, int gran, int heads, int fmt, int j,
+                        const int8_t *jforce, const int8_t *shift, int sdt, uint8_t *packed,
+                        void *scales, int8_t *jmap, double *sse_out)
+{
+    int rc = check_args(N, K, g);
+    if (rc) return rc;
+    if (fmt < 0 || fmt > 2 || j < -1 || j > 7) return ORC_ERR_ARG;
+    if (gran < ORC_GRAN_GROUP || gran > ORC_GRAN_HEAD) return ORC_ERR_ARG;
+    if (gran == ORC_GRAN_HEAD && (heads <= 0 || N % heads != 0)) return ORC_ERR_ARG;
+    int nb = orc_block_count(N, K, g, gran, heads);
+    int G = K / g;
+    double *bsse = (double *)calloc((size_t)(nb > 0 ? nb : 1), sizeof(double));
+    if (!bsse) return ORC_ERR_ALLOC;
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int b = 0; b < nb; ++b) {
+        int r0, r1, k0, k1;
+        block_extent(b, N, K, g, gran, heads, &r0, &r1, &k0, &k1);
+        /* the block's absmax of W' */
+        float A = 0.0f;
+        int e = 0;
+        for (int r = r0; r < r1 && !e; ++r)
+            for (int k = k0; k < k1; ++k) {
+                float w = folded(W, K, shift, r, k);
+                if (!isfinite(w)) { e = ORC_ERR_NONFINITE; break; }
+                if (fabsf(w) > A) A = fabsf(w);
+            }
+        int jb = j;
+        float s;
+        uint32_t raw;
+        double sse;
+        if (!e && jforce) jb = jforce[b];
+        else if (!e && j < 0) {
+            /* per-block search: first strict minimum, j ascending */
+            double best = INFINITY;
+            jb = 0;
+            for (int jj = 0; jj < 8 && !e; ++jj) {
+                e = block_pass(W, K, shift, r0, r1, k0, k1, A, fmt, jj, sdt, NULL, &s, &raw, &sse);
+                if (!e && sse < best) { best = sse; jb = jj; }
+            }
+        }
+        if (!e && (jb < 0 || jb > 7)) e = ORC_ERR_ARG;
+        if (!e) e = block_pass(W, K, shift, r0, r1, k0, k1, A, fmt, jb, sdt, packed, &s, &raw, &sse);
+        if (e) {
+#pragma omp atomic write
+            err = e;
+            continue;
+        }
+        bsse[b] = sse;
+        if (jmap) jmap[b] = (int8_t)jb;
+        if (scales)
+            for (int r = r0; r < r1; ++r)
+                for (int gi = k0 / g; gi < k1 / g; ++gi) {
+                    if (sdt == ORC_SCALE_F16) ((uint16_t *)scales)[(size_t)r * G + gi] = (uint16_t)raw;
+                    else ((uint32_t *)scales)[(size_t)r * G + gi] = raw;
+                }
+    }
+    double tot = 0.0;
+    for (int b = 0; b < nb; ++b) tot += bsse[b];
+    free(bsse);
+    if (err) return err;
+    if (sse_out) *sse_out = tot;
+    return 0;
+}
+
+/* ------------------------------------------------- 4-bit activations (R10) */
+
+int orc_act_quantize(const uint16_t *X, int M, int K, const int8_t *shift, float rho, int fmt, int j,
+                     uint8_t *packed, float *s_out)
+{
+    if (M < 0 || K < 0 || (K % 2) != 0 || fmt < 0 || fmt > 2 || j < 0 || j > 7) return ORC_ERR_ARG;
+    if (!(rho > 0.0f) || !isfinite(rho)) return ORC_ERR_ARG;
+    double mags[8], qmax_d;
+    orc_format_table(fmt, mags, &qmax_d);
+    float s;
+    uint32_t raw;
+    if (group_scale(rho, orc_bias_factor(j), (float)qmax_d, ORC_SCALE_F32, &s, &raw) != 0) return ORC_ERR_SCALE;
+    for (size_t i = 0; i < (size_t)M * K; ++i)
+        if (!isfinite(orc_bf16_to_f32(X[i]))) return ORC_ERR_NONFINITE;
+    for (int m = 0; m < M; ++m)
+        for (int k = 0; k < K; ++k) {
+            float x = orc_bf16_to_f32(X[(size_t)m * K + k]);
+            float xs = shift ? x * pow2f(-shift[k]) : x; /* exact unless it overflows */
+            int idx = 0;
+            if (s != 0.0f) {
+                float q = xs / s; /* fl32 */
+                idx = orc_nearest_index(fabs((double)q), mags);
+            }
+            int code = ((signbit(xs) ? 1 : 0) << 3) | idx;
+            uint8_t *byte = &packed[(size_t)m * (K / 2) + (k >> 1)];
+            if ((k & 1) == 0) *byte = (uint8_t)((*byte & 0xf0u) | code);
+            else *byte = (uint8_t)((*byte & 0x0fu) | (code << 4));
+        }
+    *s_out = s;
+    return 0;
+}
+
+/* Y[m,n] = s_a * sum_k v_a(a[m,k]) * v(w[n,k]) * s[n, k/g], fp64, k
+ * increasing: both scale factors outside the low-bit product. */
+static double w4a4_one(const uint8_t *apacked, int afmt, double s_a, const uint8_t *packed,
+                       const void *scales, int sdt, int fmt, int K, int g, int m, int n)
+{
+    int G = K / g;
+    double acc = 0.0;
+    const uint8_t *ar = apacked + (size_t)m * (K / 2);
+    const uint8_t *pr = packed + (size_t)n * (K / 2);
+    for (int k = 0; k < K; ++k) {
+        int ac = (k & 1) ? (ar[k >> 1] >> 4) : (ar[k >> 1] & 15);
+        int wc = (k & 1) ? (pr[k >> 1] >> 4) : (pr[k >> 1] & 15);
+        double w = code_times_scale(fmt, wc, (double)load_scale(scales, sdt, (size_t)n * G + k / g));
+        acc += orc_code_value(afmt, ac) * w;
+    }
+    return s_a * acc;
+}
+
+int orc_gemm_w4a4(const uint8_t *apacked, int afmt, float s_a, const uint8_t *packed,
+                  const void *scales, int sdt, int fmt, int M, int N, int K, int g, double *Y)
+{
+    if (M < 0 || afmt < 0 || afmt > 2) return ORC_ERR_ARG;
+    int rc = check_args(N, K, g);
+    if (rc) return rc;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int m = 0; m < M; ++m)
+        for (int n = 0; n < N; ++n)
+            Y[(size_t)m * N + n] = w4a4_one(apacked, afmt, (double)s_a, packed, scales, sdt, fmt, K, g, m, n);
+    return 0;
+}
+
+int orc_gemm_w4a4_sampled(const uint8_t *apacked, int afmt, float s_a, const uint8_t *packed,
+                          const void *scales, int sdt, int fmt, int M, int N, int K, int g,
+                          int count, const int32_t *ms, const int32_t *ns, double *out)
+{
+    if (afmt < 0 || afmt > 2) return ORC_ERR_ARG;
+    int rc = check_args(N, K, g);
+    if (rc) return rc;
+    for (int i = 0; i < count; ++i)
+        if (ms[i] < 0 || ms[i] >= M || ns[i] < 0 || ns[i] >= N) return ORC_ERR_ARG;
+#pragma omp parallel for schedule(static)
+    for (int i = 0; i < count; ++i)
+        out[i] = w4a4_one(apacked, afmt, (double)s_a, packed, scales, sdt, fmt, K, g, ms[i], ns[i]);
     return 0;
 }
 

@@ -39,6 +39,22 @@ int orc_gemm_sampled(const uint16_t *X, const uint8_t *packed, const void *scale
                      const int32_t *ns, double *out);
 int orc_preshift_calibrate(const uint16_t *X, int M, int K, int8_t *shift, float *rho_out);
 int orc_preshift_apply(const uint16_t *X, int M, int K, const int8_t *shift, float rho, uint16_t *Xt);
+/* granularity of the scale (reading R11) */
+#define ORC_GRAN_GROUP 0   /* g consecutive elements of a row */
+#define ORC_GRAN_CHANNEL 1 /* one output channel: a whole row */
+#define ORC_GRAN_HEAD 2    /* N/heads consecutive rows (one attention head) */
+int orc_block_count(int N, int K, int g, int gran, int heads);
+int orc_quantize_blocks(const float *W, int N, int K, int g, int gran, int heads, int fmt, int j,
+                        const int8_t *jforce, const int8_t *shift, int sdt, uint8_t *packed,
+                        void *scales, int8_t *jmap, double *sse_out);
+/* 4-bit activations with the pre-shifted bias (reading R10) */
+int orc_act_quantize(const uint16_t *X, int M, int K, const int8_t *shift, float rho, int fmt, int j,
+                     uint8_t *packed, float *s_out);
+int orc_gemm_w4a4(const uint8_t *apacked, int afmt, float s_a, const uint8_t *packed,
+                  const void *scales, int sdt, int fmt, int M, int N, int K, int g, double *Y);
+int orc_gemm_w4a4_sampled(const uint8_t *apacked, int afmt, float s_a, const uint8_t *packed,
+                          const void *scales, int sdt, int fmt, int M, int N, int K, int g,
+                          int count, const int32_t *ms, const int32_t *ns, double *out);
 int orc_num_threads(void);
 void orc_set_num_threads(int n);
 

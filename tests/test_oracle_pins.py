@@ -543,3 +543,264 @@ def test_golden_tiny_digest(oracle_mod):
     assert hashlib.sha256(r["scales"].tobytes()).hexdigest() == d["scales_sha256"]
     Y = oracle_mod.gemm(case["X"], r["packed"], r["scales"], 1, 128)
     np.testing.assert_allclose(Y[0, :8], d["y_first8"], rtol=1e-15, atol=0)
+
+
+# ------------------------------------------------ granularity blocks (reading R11)
+
+GRANS = {"group": 0, "channel": 1, "head": 2}
+
+
+def block_extents(N, K, g, gran, heads):
+    """Rows x columns of every scale block, written out per granularity."""
+    if gran == 0:
+        return [((n, n + 1), (gi * g, (gi + 1) * g)) for n in range(N) for gi in range(K // g)]
+    if gran == 1:
+        return [((n, n + 1), (0, K)) for n in range(N)]
+    R = N // heads
+    return [((h * R, (h + 1) * R), (0, K)) for h in range(heads)]
+
+
+def blocks_bruteforce(W, g, gran, heads, fmt, j, sdt):
+    """Pure-Python block quantizer: absmax over the block, scale by R3,
+    codes by R4, the scale broadcast over the block's group slots; j=None
+    takes each block's first strict SSE minimum (exact rational SSE)."""
+    N, K = W.shape
+    mags = mags_exact(fmt)
+    codes = np.zeros((N, K), np.int64)
+    scales = np.zeros((N, K // g), np.float32)
+    jmap, sses = [], []
+    for (r0, r1), (k0, k1) in block_extents(N, K, g, gran, heads):
+        blk = W[r0:r1, k0:k1]
+        A = np.max(np.abs(blk)).astype(np.float32)
+
+        def run(jj):
+            s = scale_ref(A, jj, fmt, sdt)
+            c = np.zeros(blk.shape, np.int64)
+            sse = Fr(0)
+            for (r, k), x in np.ndenumerate(blk):
+                idx = 0 if s == 0 else nearest_exact(Fr(float(f32(x / s))), mags)
+                sign = 1 if math.copysign(1.0, float(x)) < 0 else 0
+                c[r, k] = (sign << 3) | idx
+                v = -mags[idx] if sign else mags[idx]
+                sse += (Fr(float(x)) - v * Fr(float(s))) ** 2
+            return s, c, sse
+
+        if j is None:
+            runs = [run(jj) for jj in range(8)]
+            best = min(range(8), key=lambda jj: (runs[jj][2], jj))
+        else:
+            runs = {j: run(j)}
+            best = j
+        s, c, sse = runs[best]
+        codes[r0:r1, k0:k1] = c
+        scales[r0:r1, k0 // g:k1 // g] = s
+        jmap.append(best)
+        sses.append(sse)
+    return codes, scales, np.array(jmap, np.int8), sses
+
+
+@pytest.mark.parametrize("gran,heads", [("group", 0), ("channel", 0), ("head", 2), ("head", 6)])
+@pytest.mark.parametrize("fmt,sdt", [(1, "f16"), (0, "f32"), (2, "f16")])
+def test_blocks_bruteforce_fixed_j(oracle_mod, gran, heads, fmt, sdt):
+    """Codes, broadcast scales and SSE of every granularity equal the
+    pure-Python block quantizer (fixed bias index)."""
+    rng = np.random.default_rng(40 + fmt)
+    W = (rng.standard_normal((6, 96)) * 0.05 * np.exp(rng.standard_normal((6, 1)))).astype(np.float32)
+    W[1, 5] = -0.0
+    for j in (0, 5):
+        r = oracle_mod.quantize_blocks(W, 32, GRANS[gran], fmt, j, heads, None, sdt)
+        codes, scales, _, sses = blocks_bruteforce(W, 32, GRANS[gran], heads, fmt, j, sdt)
+        assert np.array_equal(unpack(r["packed"]), codes), (gran, fmt, j)
+        assert np.array_equal(r["scales"].astype(np.float32), scales)
+        tot = sum(sses, Fr(0))
+        assert abs(Fr(r["sse"]) - tot) <= tot * Fr(1, 10 ** 12) + Fr(1, 10 ** 300)
+        assert np.all(r["jmap"] == j)
+
+
+@pytest.mark.parametrize("gran,heads", [("group", 0), ("channel", 0), ("head", 3)])
+def test_blocks_search_bruteforce(oracle_mod, gran, heads):
+    """Per-block search picks each block's SSE minimum over the 8 bias
+    indices (first one on an exact tie); where two candidates are within
+    1e-9 of each other, either is accepted and the codes are checked under
+    the oracle's own pick."""
+    rng = np.random.default_rng(44)
+    W = synth.student_t_weights(rng, 6, 64, scale=0.05)
+    r = oracle_mod.quantize_blocks(W, 32, GRANS[gran], 1, None, heads, None, "f16")
+    _, _, jref, sses = blocks_bruteforce(W, 32, GRANS[gran], heads, 1, None, "f16")
+    nb = len(jref)
+    for b in range(nb):
+        if r["jmap"][b] != jref[b]:
+            # near tie: the oracle's pick must be within 1e-9 of the exact best
+            per_j = [blocks_bruteforce(W, 32, GRANS[gran], heads, 1, jj, "f16")[3][b] for jj in range(8)]
+            assert per_j[r["jmap"][b]] <= min(per_j) * (1 + Fr(1, 10 ** 9)), (b, r["jmap"][b], jref[b])
+    rf = oracle_mod.quantize_blocks(W, 32, GRANS[gran], 1, 0, heads, None, "f16", jforce=r["jmap"])
+    assert np.array_equal(rf["packed"], r["packed"]) and np.array_equal(rf["scales"], r["scales"])
+    # the per-block pick is never worse than any single bias index for the tensor
+    for jj in range(8):
+        assert r["sse"] <= oracle_mod.quantize_blocks(W, 32, GRANS[gran], 1, jj, heads, None, "f16")["sse"] * (1 + 1e-12)
+
+
+def test_blocks_degenerate_cases(oracle_mod):
+    """Granularities that coincide: channel with K == g is group; head with
+    one row per head is channel; group equals the fixed quantizer."""
+    rng = np.random.default_rng(45)
+    W = (rng.standard_normal((8, 128)) * 0.02).astype(np.float32)
+    shift = rng.integers(-3, 1, 128).astype(np.int8)
+    for sdt in ("f16", "f32"):
+        g = oracle_mod.quantize_blocks(W, 128, 0, 1, 2, 0, shift, sdt)
+        c = oracle_mod.quantize_blocks(W, 128, 1, 1, 2, 0, shift, sdt)
+        h = oracle_mod.quantize_blocks(W, 128, 2, 1, 2, 8, shift, sdt)
+        packed, scales, sse = oracle_mod.quantize_fixed(W, 128, 1, 2, shift, sdt)
+        for r in (g, c, h):
+            assert np.array_equal(r["packed"], packed) and np.array_equal(r["scales"], scales)
+            assert r["sse"] == pytest.approx(sse, rel=1e-12)
+    # group granularity at g = 32 equals the fixed quantizer at g = 32
+    g32 = oracle_mod.quantize_blocks(W, 32, 0, 0, 4, 0, None, "f16")
+    p32, s32, _ = oracle_mod.quantize_fixed(W, 32, 0, 4, None, "f16")
+    assert np.array_equal(g32["packed"], p32) and np.array_equal(g32["scales"], s32)
+
+
+def test_blocks_head_shares_the_largest_row(oracle_mod):
+    """Hand example: in a head of 2 rows whose absmax is 12 (E2M1, j = 0)
+    every slot of both rows holds s = 2, and a row of small values codes
+    against it (0.9 / 2 = 0.45 -> 0.5, code 1)."""
+    W = np.zeros((4, 64), np.float32)
+    W[0, 7] = 12.0
+    W[1, :] = 0.9
+    W[2, :] = 1.0
+    W[3, 3] = -3.0
+    r = oracle_mod.quantize_blocks(W, 32, 2, 1, 0, 2, None, "f32")
+    assert np.all(r["scales"][0:2] == 2.0)
+    assert np.all(r["scales"][2:4] == np.float32(3.0) / np.float32(6.0))
+    c = unpack(r["packed"])
+    assert c[0, 7] == 7 and np.all(c[1] == 1)
+    # rows 2-3: s = 0.5, 1.0 / 0.5 = 2 -> index 4; -3 / 0.5 = -6 -> code 0xF
+    assert np.all(c[2] == 4) and c[3, 3] == 0xF
+
+
+def test_blocks_reject_bad_heads(oracle_mod):
+    W = np.ones((6, 64), np.float32)
+    with pytest.raises(oracle_mod.OracleError):
+        oracle_mod.quantize_blocks(W, 32, 2, 1, 0, 4)
+    with pytest.raises(oracle_mod.OracleError):
+        oracle_mod.quantize_blocks(W, 32, 2, 1, 0, 0)
+
+
+# ------------------------------------------- 4-bit activations (reading R10)
+
+def act_bruteforce(X_bits, shift, rho, fmt, j):
+    """Pure-Python activation quantizer: X' = X * 2^-e (exact), one fp32
+    scale s_a = fl32(fl32(rho * c_j) / Qmax), codes by R4."""
+    mags = mags_exact(fmt)
+    s = scale_ref(np.float32(rho), j, fmt, "f32")
+    x = synth.bf16_bits_to_f32(X_bits)
+    M, K = x.shape
+    codes = np.zeros((M, K), np.int64)
+    for (m, k), v in np.ndenumerate(x):
+        xs = f32(v * f32(2.0 ** (-int(shift[k])))) if shift is not None else f32(v)
+        idx = 0 if s == 0 else nearest_exact(Fr(float(f32(xs / s))), mags)
+        sign = 1 if math.copysign(1.0, float(xs)) < 0 else 0
+        codes[m, k] = (sign << 3) | idx
+    return codes, s
+
+
+def test_act_quantize_hand_example(oracle_mod):
+    """rho = 6 gives s_a = 1 in E2M1 (j = 0): 0.5 -> 1; -1.25 (tie 1|1.5)
+    -> even index 2, negative; 2.5 (tie 2|3) -> index 4; 5 (tie 4|6) ->
+    index 6; 7 saturates to 7; -0 keeps its sign; bf16(0.24) < 0.25 -> 0;
+    bf16(0.26) > 0.25 -> 1.  A channel shift of -1 doubles its column."""
+    x = np.array([[0.5, -1.25, 2.5, 5.0, 7.0, -0.0, 0.24, 0.26]], np.float32)
+    X = synth.to_bf16_bits(x)
+    packed, s = oracle_mod.act_quantize(X, 6.0, 1, 0)
+    assert s == 1.0
+    assert list(packed[0]) == [0xA1, 0x64, 0x87, 0x10]
+    shift = np.array([0, -1, 0, 0, 0, 0, 0, 0], np.int8)
+    packed, _ = oracle_mod.act_quantize(X, 6.0, 1, 0, shift)
+    assert packed[0, 0] == 0xC1       # -2.5: tie 2|3 -> index 4, negative
+
+
+@pytest.mark.parametrize("fmt,j", [(1, 0), (1, 3), (0, 0), (2, 6)])
+def test_act_quantize_bruteforce(oracle_mod, fmt, j):
+    rng = np.random.default_rng(50 + j)
+    X, _ = synth.outlier_activations(rng, 5, 64, frac=0.05, factor=30.0)
+    shift, rho = oracle_mod.preshift_calibrate(X[:3])     # calibration rows only
+    packed, s = oracle_mod.act_quantize(X, rho, fmt, j, shift)
+    codes, sref = act_bruteforce(X, shift, rho, fmt, j)
+    assert s == sref
+    assert np.array_equal(unpack(packed), codes)
+    # without a shift
+    packed, s = oracle_mod.act_quantize(X, rho, fmt, j, None)
+    codes, _ = act_bruteforce(X, None, rho, fmt, j)
+    assert np.array_equal(unpack(packed), codes)
+
+
+def test_act_quantize_error_bound_and_saturation(oracle_mod):
+    """On its own calibration data every X' = X * 2^-e lies within half a
+    grid step (times s_a) of its code's value; values beyond the calibrated
+    range saturate to the largest magnitude."""
+    rng = np.random.default_rng(52)
+    X, _ = synth.outlier_activations(rng, 16, 256)
+    shift, rho = oracle_mod.preshift_calibrate(X)
+    packed, s = oracle_mod.act_quantize(X, rho, 1, 0, shift)
+    mags = [float(v) for v in mags_exact(1)]
+    gaps = np.diff(mags)
+    xs = synth.bf16_bits_to_f32(X).astype(np.float64) * np.exp2(-shift.astype(np.float64))
+    c = unpack(packed)
+    v = np.array(mags)[c & 7] * np.where(c >= 8, -1.0, 1.0)
+    err = np.abs(xs - v * s)
+    half = np.array([gaps[0] / 2] + [max(gaps[i - 1], gaps[min(i, 6)]) / 2 for i in range(1, 8)])[c & 7]
+    assert np.all(err <= half * s * (1 + 1e-6) + 1e-30)
+    big = synth.to_bf16_bits(np.full((1, 256), float(rho) * 8, np.float32))
+    pb, _ = oracle_mod.act_quantize(big, rho, 1, 0, None)
+    assert np.all(unpack(pb) == 7)
+    with pytest.raises(oracle_mod.OracleError):
+        oracle_mod.act_quantize(X, 0.0, 1, 0)
+    bad = X.copy()
+    bad[0, 0] = 0x7F80                  # +Inf
+    with pytest.raises(oracle_mod.OracleError):
+        oracle_mod.act_quantize(bad, rho, 1, 0)
+
+
+@pytest.mark.parametrize("afmt,fmt", [(1, 1), (0, 1), (2, 0)])
+def test_gemm_w4a4_matches_torch_fp64(oracle_mod, afmt, fmt):
+    """W4A4 product == s_a * V_a . W_hat^T by torch fp64 on independently
+    decoded activation codes and weights."""
+    rng = np.random.default_rng(53)
+    W = synth.normal_weights(rng, 24, 256)
+    X = synth.activations(rng, 7, 256)
+    shift, rho = oracle_mod.preshift_calibrate(X)
+    apacked, s_a = oracle_mod.act_quantize(X, rho, afmt, 2, shift)
+    packed, scales, _ = oracle_mod.quantize_fixed(W, 128, fmt, 0, shift, "f16")
+    vals = np.array([float(value_exact(afmt, c)) for c in range(16)])
+    Va = vals[unpack(apacked)]
+    What = dequant_independent(packed, scales, fmt, 128)
+    ref = float(s_a) * torch.matmul(torch.from_numpy(Va), torch.from_numpy(What).T).numpy()
+    Y = oracle_mod.gemm_w4a4(apacked, afmt, s_a, packed, scales, fmt, 128)
+    np.testing.assert_allclose(Y, ref, rtol=1e-12, atol=1e-12 * np.max(np.abs(ref)))
+    ms = np.array([6, 0, 3], np.int32)
+    ns = np.array([0, 23, 11], np.int32)
+    assert np.array_equal(oracle_mod.gemm_w4a4_sampled(apacked, afmt, s_a, packed, scales, fmt, 128, ms, ns),
+                          Y[ms, ns])
+
+
+def test_w4a4_tracks_the_full_precision_product(oracle_mod):
+    """Sanity of the whole 4-bit path on outlier activations: with the
+    pre-shift the W4A4 product stays close to X . W^T; without it the
+    outlier channels crush the other ones."""
+    rng = np.random.default_rng(54)
+    W = synth.normal_weights(rng, 64, 512)
+    X, _ = synth.outlier_activations(rng, 16, 512, frac=0.02, factor=50.0)
+    ref = synth.bf16_bits_to_f32(X).astype(np.float64) @ W.astype(np.float64).T
+
+    def cos(a, b):
+        return float(np.sum(a * b) / np.linalg.norm(a) / np.linalg.norm(b))
+
+    shift, rho = oracle_mod.preshift_calibrate(X)
+    ap, sa = oracle_mod.act_quantize(X, rho, 1, 0, shift)
+    wp, ws, _ = oracle_mod.quantize_fixed(W, 128, 1, 0, shift, "f16")
+    with_shift = cos(oracle_mod.gemm_w4a4(ap, 1, sa, wp, ws, 1, 128), ref)
+    z = np.zeros(512, np.int8)
+    ap0, sa0 = oracle_mod.act_quantize(X, rho, 1, 0, z)
+    wp0, ws0, _ = oracle_mod.quantize_fixed(W, 128, 1, 0, None, "f16")
+    without = cos(oracle_mod.gemm_w4a4(ap0, 1, sa0, wp0, ws0, 1, 128), ref)
+    assert with_shift > 0.9 and with_shift > without
