@@ -74,6 +74,8 @@ typedef enum fp4_scale_dtype { FP4_SCALE_F32 = 0, FP4_SCALE_F16 = 1 } fp4_scale_
 
 /* GEMM engine selection for fp4_gemm_ex (fp4_gemm always uses AUTO). */
 typedef enum fp4_engine { FP4_ENGINE_AUTO = 0, FP4_ENGINE_DECODE = 1, FP4_ENGINE_TENSOR = 2 } fp4_engine;
+/* Extent of the absmax behind one weight scale (fp4_quantize_blocks). */
+typedef enum fp4_granularity { FP4_GRAN_GROUP = 0, FP4_GRAN_CHANNEL = 1, FP4_GRAN_HEAD = 2 } fp4_granularity;
 /* Output activation fused into the GEMM epilogue (fp4_gemm_act). */
 typedef enum fp4_act { FP4_ACT_NONE = 0, FP4_ACT_SILU = 1, FP4_ACT_GELU = 2, FP4_ACT_SILU_GATE = 3 } fp4_act;
 
@@ -130,6 +132,42 @@ FP4_API fp4_status fp4_quantize(const float *W, int N, int K, int group, fp4_for
                         cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * fp4_quantize_blocks -- fp4_quantize with the scale's absmax taken over a
+ * coarser block, and the bias index chosen per block.  (Granularities of
+ * the HiFloat4 page, section 3.1 "权重量化策略", scales grouped per
+ * attention head, and of the quantization-basics page, the per-tensor /
+ * per-channel / per-token classification: per output channel; the search
+ * of the LLM-FP4 summary page applied to each block instead of the tensor.)
+ *
+ *   gran FP4_GRAN_GROUP    block = `group` consecutive k of a row (as
+ *                          fp4_quantize);
+ *        FP4_GRAN_CHANNEL  block = a whole row (one output channel);
+ *        FP4_GRAN_HEAD     block = N/heads consecutive rows (an attention
+ *                          head of a q/k/v projection); N % heads == 0.
+ *   Channel and head blocks need K % 128 == 0.
+ *   A    = max |W'| over the block; s = R(fl32(fl32(A * c_j) / Qmax_f)) as
+ *          in fp4_quantize, written to every [n][k/group] slot the block
+ *          covers, so fp4_gemm reads the result with the same `group`.
+ *   bias_index 0..7: that c_j for every block; -1: each block takes the j
+ *          with the smallest SSE over its own elements (fp64; first strict
+ *          minimum in j order; the SSE is summed in a fixed order, so the
+ *          choice does not depend on timing).  fmt is fixed (not AUTO): the
+ *          GEMM decodes one format per tensor.
+ *   jmap       device int8 [blocks] out or NULL: the bias index of each
+ *              block (blocks: N*K/group, N or heads, in row order).
+ *   workspace  fp4_quantize_blocks_workspace_size(...) bytes (NULL when
+ *              0), no initialisation; channel/head searches keep 64 bytes
+ *              per 128 weights there.
+ * Device status: FP4_DEV_NONFINITE_INPUT, FP4_DEV_SCALE_OVERFLOW.
+ * ---------------------------------------------------------------------- */
+FP4_API size_t fp4_quantize_blocks_workspace_size(int N, int K, int group, fp4_granularity gran, int heads,
+                                                  int bias_index);
+FP4_API fp4_status fp4_quantize_blocks(const float *W, int N, int K, int group, fp4_granularity gran, int heads,
+                                       fp4_format fmt, int bias_index, const int8_t *chan_shift,
+                                       fp4_scale_dtype sdt, uint8_t *packed, void *scales, int8_t *jmap,
+                                       void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * fp4_dequantize -- W_hat[n,k] = fl32(v(code[n,k]) * s[n, k/group]), the
  * weights the GEMM multiplies by (test aid).  W_hat [N][K] fp32 out.
  * ---------------------------------------------------------------------- */
@@ -176,6 +214,44 @@ FP4_API fp4_status fp4_preshift_apply(const uint16_t *X, int M, int K, const int
  * ---------------------------------------------------------------------- */
 FP4_API fp4_status fp4_preshift_calibrate_noalloc(const uint16_t *X, int M, int K, int8_t *shift, float *rho,
                                                   cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * 4-bit activations with the pre-shifted exponent bias (LLM-FP4 summary
+ * page, section on the pre-shifted exponent bias: activations are quantized
+ * with one per-tensor real factor, the per-channel powers of two having
+ * moved into the weights; efficient matrix multiplication: both scale
+ * factors are taken out of the low-bit product).
+ *
+ * fp4_act_quantize:
+ *   s_a  = fl32(fl32(rho * c_j) / Qmax_f)                    (fp32)
+ *   X'   = fl32(X[m,k] * 2^-shift[k])                        (shift NULL: X)
+ *   code = signbit(X') << 3 | nearest magnitude index of fl32(|X'| / s_a),
+ *          ties to the even index, saturating at index 7 (values beyond
+ *          the calibrated range clip to +-Qmax * s_a).
+ *   X [M][K] bf16 device, K % 8 == 0; shift [K] int8 (values in [-126, 0],
+ *   from fp4_preshift_calibrate) or NULL; rho device float (positive,
+ *   finite: else FP4_DEV_NONFINITE_INPUT and a_scale = NaN); fmt
+ *   E1M2/E2M1/E3M0; j 0..7.  packed [M][K/2] uint8 out (low nibble
+ *   first); a_scale device float out (s_a, written even when M == 0).
+ * Device status: FP4_DEV_NONFINITE_INPUT.
+ *
+ * fp4_gemm_w4a4:
+ *   Y[m,n] = bf16( act( s_a * sum_k v_a(a[m,k]) * v(w[n,k]) * s[n,k/group] ) )
+ *   apacked [M][K/2] from fp4_act_quantize in format afmt, a_scale its s_a;
+ *   the weights, act, Y and the engine choice as for fp4_gemm_act.  The
+ *   activation values (exact in bf16) are expanded into the workspace and
+ *   multiplied on the 16-bit tensor paths.
+ *   workspace  fp4_gemm_w4a4_workspace_size(M, N, K) bytes, zero-filled
+ *              once before first use (its first part is the GEMM
+ *              workspace, with the same rules).
+ * ---------------------------------------------------------------------- */
+FP4_API fp4_status fp4_act_quantize(const uint16_t *X, int M, int K, const int8_t *shift, const float *rho,
+                                    fp4_format fmt, int j, uint8_t *packed, float *a_scale, cudaStream_t stream);
+FP4_API size_t fp4_gemm_w4a4_workspace_size(int M, int N, int K);
+FP4_API fp4_status fp4_gemm_w4a4(const uint8_t *apacked, fp4_format afmt, const float *a_scale,
+                                 const uint8_t *packed, const void *scales, fp4_scale_dtype sdt, fp4_format fmt,
+                                 int M, int N, int K, int group, fp4_act act, uint16_t *Y, void *workspace,
+                                 size_t ws_bytes, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
  * fp4_gemm -- Y = bf16( x_scale * X . dequant(W)^T ), fp32 accumulation.

@@ -173,3 +173,49 @@ def test_workspace_sizes(L):
     assert L.fp4_gemm_workspace_size(2048, 4096, 4096) == 65536 + 2048 * 4096 * 2 + 2048 * 4
     assert L.fp4_quantize_workspace_size(4096, 4096, 128, 1, 0) >= 8
     assert L.fp4_preshift_workspace_size(2048, 4096) >= 4096 * 4
+
+
+def test_quantize_blocks_argument_errors(L):
+    def qb(N=8, K=256, group=128, gran=1, heads=0, fmt=1, j=0, shift=None, sdt=1, packed=FAKE, scales=FAKE,
+           jmap=None, ws=None, wsb=0):
+        return L.fp4_quantize_blocks(FAKE, N, K, group, gran, heads, fmt, j, shift, sdt, packed, scales, jmap, ws,
+                                     wsb, None)
+    assert qb(fmt=-1) == 1                     # the format is fixed
+    assert qb(j=8) == 1 and qb(j=-2) == 1
+    assert qb(gran=3) == 1
+    assert qb(gran=2, heads=0) == 1
+    assert qb(gran=2, heads=3) == 2            # N % heads
+    assert qb(K=96, group=32) == 2             # channel blocks need K % 128 == 0
+    assert qb(group=48) == 2
+    assert qb(packed=MIS) == 3
+    assert qb(N=0) == 0
+    # workspace: channel/head blocks keep their absmax (and, searched, 64 B
+    # per 128 weights + one byte per block); group blocks need none
+    def up(b):
+        return (b + 255) // 256 * 256
+    assert L.fp4_quantize_blocks_workspace_size(8, 256, 128, 0, 0, -1) == 0
+    assert L.fp4_quantize_blocks_workspace_size(8, 256, 128, 1, 0, 0) == up(8 * 4)
+    assert L.fp4_quantize_blocks_workspace_size(8, 256, 128, 2, 4, -1) == up(4 * 4) + up(8 * 256 // 128 * 64) + up(4)
+    assert qb(j=-1, ws=None) == 4
+    need = L.fp4_quantize_blocks_workspace_size(8, 256, 128, 1, 0, -1)
+    assert qb(j=-1, ws=FAKE, wsb=need - 1) == 4
+
+
+def test_act_quantize_and_w4a4_argument_errors(L):
+    aq = L.fp4_act_quantize
+    assert aq(FAKE, 4, 60, None, FAKE, 1, 0, FAKE, FAKE, None) == 2      # K % 8
+    assert aq(FAKE, 4, 64, None, None, 1, 0, FAKE, FAKE, None) == 1      # rho required
+    assert aq(FAKE, 4, 64, None, FAKE, 1, 8, FAKE, FAKE, None) == 1      # j
+    assert aq(FAKE, 4, 64, None, FAKE, -1, 0, FAKE, FAKE, None) == 1     # fixed format
+    assert aq(MIS, 4, 64, None, FAKE, 1, 0, FAKE, FAKE, None) == 3
+    assert aq(FAKE, 4, 64, MIS, FAKE, 1, 0, FAKE, FAKE, None) == 3
+    g = L.fp4_gemm_w4a4
+    need = L.fp4_gemm_w4a4_workspace_size(4, 256, 512)
+    assert need == (L.fp4_gemm_workspace_size(4, 256, 512) + 255) // 256 * 256 + 4 * 512 * 2
+    assert g(FAKE, 1, FAKE, FAKE, FAKE, 1, 1, 4, 256, 512, 128, 0, FAKE, None, 0, None) == 4
+    assert g(FAKE, 1, FAKE, FAKE, FAKE, 1, 1, 4, 256, 512, 128, 0, FAKE, FAKE, need - 16, None) == 4
+    assert g(FAKE, 5, FAKE, FAKE, FAKE, 1, 1, 4, 256, 512, 128, 0, FAKE, FAKE, need, None) == 1
+    assert g(FAKE, 1, None, FAKE, FAKE, 1, 1, 4, 256, 512, 128, 0, FAKE, FAKE, need, None) == 1
+    assert g(MIS, 1, FAKE, FAKE, FAKE, 1, 1, 4, 256, 512, 128, 0, FAKE, FAKE, need, None) == 3
+    assert g(FAKE, 1, FAKE, FAKE, FAKE, 1, 1, 4, 256, 512, 128, 4, FAKE, FAKE, need, None) == 1   # act
+    assert g(FAKE, 1, FAKE, FAKE, FAKE, 1, 1, 0, 256, 512, 128, 0, FAKE, None, 0, None) == 0      # M == 0

@@ -20,6 +20,7 @@ E1M2, E2M1, E3M0, AUTO = 0, 1, 2, -1
 SCALE_F32, SCALE_F16 = 0, 1
 ENGINE_AUTO, ENGINE_DECODE, ENGINE_TENSOR = 0, 1, 2
 ACT_NONE, ACT_SILU, ACT_GELU, ACT_SILU_GATE = 0, 1, 2, 3
+GRAN_GROUP, GRAN_CHANNEL, GRAN_HEAD = 0, 1, 2
 DEV_NONFINITE_INPUT, DEV_SCALE_OVERFLOW, DEV_WAIT_TIMEOUT, DEV_LAYOUT = 1, 2, 4, 8
 
 STATUS = {0: "FP4_OK", 1: "FP4_ERR_INVALID_ARG", 2: "FP4_ERR_UNSUPPORTED_SHAPE", 3: "FP4_ERR_MISALIGNED",
@@ -29,7 +30,8 @@ EXPORTS = ("fp4_abi_version", "fp4_status_string", "fp4_quantize_workspace_size"
            "fp4_dequantize", "fp4_preshift_workspace_size", "fp4_preshift_calibrate", "fp4_preshift_apply",
            "fp4_gemm_workspace_size", "fp4_gemm", "fp4_gemm_ex", "fp4_gemm_act", "fp4_get_device_status",
            "fp4_set_wait_timeout_us", "fp4_selftest_bounded_wait", "fp4_preshift_calibrate_noalloc",
-           "fp4_gemm_engine_for")
+           "fp4_gemm_engine_for", "fp4_quantize_blocks_workspace_size", "fp4_quantize_blocks",
+           "fp4_act_quantize", "fp4_gemm_w4a4_workspace_size", "fp4_gemm_w4a4")
 
 
 class Fp4Error(RuntimeError):
@@ -72,6 +74,11 @@ def lib():
                 "fp4_selftest_bounded_wait": (i, [ll, P]),
                 "fp4_preshift_calibrate_noalloc": (i, [P, i, i, P, P, P]),
                 "fp4_gemm_engine_for": (i, [i, i, i, i]),
+                "fp4_quantize_blocks_workspace_size": (sz, [i, i, i, i, i, i]),
+                "fp4_quantize_blocks": (i, [P, i, i, i, i, i, i, i, P, i, P, P, P, P, sz, P]),
+                "fp4_act_quantize": (i, [P, i, i, P, P, i, i, P, P, P]),
+                "fp4_gemm_w4a4_workspace_size": (sz, [i, i, i]),
+                "fp4_gemm_w4a4": (i, [P, i, P, P, P, i, i, i, i, i, i, i, P, P, sz, P]),
             }
             for name, (res, args) in sigs.items():
                 fn = getattr(L, name)
@@ -181,6 +188,35 @@ def quantize_into(W, packed, scales, choice, group=128, fmt=E2M1, bias_search=Fa
            "fp4_quantize")
 
 
+def block_count(N, K, group, gran, heads=0):
+    if gran == GRAN_GROUP:
+        return N * (K // group)
+    return N if gran == GRAN_CHANNEL else heads
+
+
+def quantize_blocks(W, group=128, gran=GRAN_CHANNEL, heads=0, fmt=E2M1, bias_index=0, chan_shift=None,
+                    scale_dtype="f16", want_jmap=True, stream=None):
+    """FP4 quantize with the scale's absmax over a group, a row (output
+    channel) or N/heads rows (attention head); bias_index -1 searches the
+    bias per block.  Returns dict(packed, scales [N][K/group], jmap int8
+    [blocks] or None), all on the device."""
+    assert W.is_cuda and W.dtype == torch.float32 and W.is_contiguous() and W.dim() == 2
+    N, K = W.shape
+    sdt = _sdt(scale_dtype)
+    dev = W.device
+    packed = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((N, K // group), dtype=torch.float16 if sdt else torch.float32, device=dev)
+    jmap = torch.empty(max(block_count(N, K, group, gran, heads), 1), dtype=torch.int8, device=dev) \
+        if want_jmap else None
+    L = lib()
+    need = L.fp4_quantize_blocks_workspace_size(N, K, group, gran, heads, bias_index)
+    ws, wsb = _workspace(dev).get(need)
+    _check(L.fp4_quantize_blocks(_ptr(W), N, K, group, gran, heads, fmt, bias_index, _ptr(chan_shift), sdt,
+                                 _ptr(packed), _ptr(scales), _ptr(jmap), _ptr(ws), wsb, _stream(stream)),
+           "fp4_quantize_blocks")
+    return {"packed": packed, "scales": scales, "jmap": jmap}
+
+
 def dequantize(packed, scales, fmt, group=128, stream=None):
     N, Kh = packed.shape
     K = 2 * Kh
@@ -250,6 +286,45 @@ def gemm(X, packed, scales, fmt=E2M1, group=128, x_scale=None, out=None, engine=
         ws, wsb = workspace, workspace.numel() * workspace.element_size()
     _check(L.fp4_gemm_act(_ptr(_bits(X)), _ptr(packed), _ptr(scales), sdt, fmt, M, N, K, group, _ptr(x_scale),
                           act, _ptr(_bits(out)), _ptr(ws), wsb, engine, splits, _stream(stream)), "fp4_gemm")
+    return out
+
+
+# ---------------------------------------------------------- 4-bit activations
+
+def act_quantize(X, rho, fmt=E2M1, j=0, shift=None, out=None, a_scale=None, stream=None):
+    """4-bit activation codes of X [M][K] bf16 against the per-tensor scale
+    s_a = fl32(fl32(rho * c_j) / Qmax) after the per-channel shift.
+    Returns (packed uint8 [M][K/2], a_scale float32 [1]) on the device."""
+    M, K = X.shape
+    if out is None:
+        out = torch.empty((M, K // 2), dtype=torch.uint8, device=X.device)
+    if a_scale is None:
+        a_scale = torch.empty(1, dtype=torch.float32, device=X.device)
+    _check(lib().fp4_act_quantize(_ptr(_bits(X)), M, K, _ptr(shift), _ptr(rho), fmt, j, _ptr(out), _ptr(a_scale),
+                                  _stream(stream)), "fp4_act_quantize")
+    return out, a_scale
+
+
+def gemm_w4a4_workspace_size(M, N, K):
+    return lib().fp4_gemm_w4a4_workspace_size(M, N, K)
+
+
+def gemm_w4a4(apacked, a_scale, packed, scales, afmt=E2M1, fmt=E2M1, group=128, act=ACT_NONE, out=None,
+              workspace=None, stream=None):
+    """Y = bf16(act(s_a * v_a(A) . dequant(W)^T)) from 4-bit activation codes."""
+    M, K = apacked.shape[0], apacked.shape[1] * 2
+    N = packed.shape[0]
+    assert packed.shape[1] * 2 == K
+    sdt = SCALE_F16 if scales.dtype == torch.float16 else SCALE_F32
+    if out is None:
+        out = torch.empty((M, N // 2 if act == ACT_SILU_GATE else N), dtype=torch.bfloat16, device=apacked.device)
+    L = lib()
+    if workspace is None:
+        ws, wsb = _workspace(apacked.device, "w4a4").get(L.fp4_gemm_w4a4_workspace_size(M, N, K))
+    else:
+        ws, wsb = workspace, workspace.numel() * workspace.element_size()
+    _check(L.fp4_gemm_w4a4(_ptr(apacked), afmt, _ptr(a_scale), _ptr(packed), _ptr(scales), sdt, fmt, M, N, K, group,
+                           act, _ptr(_bits(out)), _ptr(ws), wsb, _stream(stream)), "fp4_gemm_w4a4")
     return out
 
 

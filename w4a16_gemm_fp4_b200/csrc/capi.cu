@@ -50,6 +50,15 @@ cudaError_t launch_gemm_tc(const uint16_t* X, const uint8_t* packed, const void*
                            void* ws, size_t ws_bytes, int splits, int* status, unsigned long long timeout_ns,
                            cudaStream_t st);
 cudaError_t launch_bounded_wait_probe(int* status, unsigned long long timeout_ns, cudaStream_t st);
+size_t quantize_blocks_ws_bytes(int N, int K, int group, int gran, int heads, bool search);
+cudaError_t launch_quantize_blocks(const float* W, int N, int K, int group, int gran, int heads, int fmt, int j,
+                                   const int8_t* shift, int sdt, uint8_t* packed, void* scales, int8_t* jmap,
+                                   void* ws, const FmtTables& tabs, int* status, cudaStream_t st);
+cudaError_t launch_act_quantize(const uint16_t* X, int M, int K, const int8_t* shift, const float* rho,
+                                const FmtTables& tabs, int fmt, int j, uint8_t* packed, float* a_scale, int* status,
+                                cudaStream_t st);
+cudaError_t launch_act_expand(const uint8_t* codes, long long count, const FmtTable& t, uint16_t* out,
+                              cudaStream_t st);
 int noalloc_max_k();
 cudaError_t launch_calibrate_noalloc(const uint16_t* X, int M, int K, int8_t* shift, float* rho, int* status,
                                      cudaStream_t st);
@@ -225,6 +234,95 @@ fp4_status fp4_quantize(const float* W, int N, int K, int group, fp4_format fmt,
     }
     return cuda_status(launch_quantize(W, N, K, group, (int)fmt, bias_search, chan_shift, (int)sdt, packed, scales,
                                        choice, sse, workspace, tables(), st, stream));
+}
+
+static bool blocks_shape_ok(int N, int K, fp4_granularity gran, int heads) {
+    if (gran == FP4_GRAN_GROUP) return true;
+    if (K % 128 != 0) return false;
+    return gran == FP4_GRAN_CHANNEL || (heads > 0 && N % heads == 0);
+}
+
+size_t fp4_quantize_blocks_workspace_size(int N, int K, int group, fp4_granularity gran, int heads, int bias_index) {
+    if (N <= 0 || K <= 0 || group <= 0 || K % group != 0) return 0;
+    if (gran < FP4_GRAN_GROUP || gran > FP4_GRAN_HEAD || !blocks_shape_ok(N, K, gran, heads)) return 0;
+    return quantize_blocks_ws_bytes(N, K, group, (int)gran, heads, bias_index < 0);
+}
+
+fp4_status fp4_quantize_blocks(const float* W, int N, int K, int group, fp4_granularity gran, int heads,
+                               fp4_format fmt, int bias_index, const int8_t* chan_shift, fp4_scale_dtype sdt,
+                               uint8_t* packed, void* scales, int8_t* jmap, void* workspace, size_t ws_bytes,
+                               cudaStream_t stream) {
+    if (N < 0 || K < 0) return FP4_ERR_INVALID_ARG;
+    if (fmt < FP4_E1M2 || fmt > FP4_E3M0) return FP4_ERR_INVALID_ARG;
+    if (sdt != FP4_SCALE_F32 && sdt != FP4_SCALE_F16) return FP4_ERR_INVALID_ARG;
+    if (bias_index < -1 || bias_index > 7) return FP4_ERR_INVALID_ARG;
+    if (gran < FP4_GRAN_GROUP || gran > FP4_GRAN_HEAD) return FP4_ERR_INVALID_ARG;
+    if (gran == FP4_GRAN_HEAD && heads <= 0) return FP4_ERR_INVALID_ARG;
+    fp4_status s = check_group(K, group);
+    if (s != FP4_OK) return s;
+    if (!blocks_shape_ok(N, K, gran, heads)) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if ((long long)N * K == 0) return FP4_OK;
+    if (!W || !packed || !scales) return FP4_ERR_INVALID_ARG;
+    if (!aligned(W, 16) || !aligned(packed, 16) || !aligned(scales, 4)) return FP4_ERR_MISALIGNED;
+    if (chan_shift && !aligned(chan_shift, 16)) return FP4_ERR_MISALIGNED;
+    const size_t need = quantize_blocks_ws_bytes(N, K, group, (int)gran, heads, bias_index < 0);
+    if (need > 0 && (!workspace || ws_bytes < need)) return FP4_ERR_WORKSPACE;
+    if (workspace && !aligned(workspace, 16)) return FP4_ERR_MISALIGNED;
+    int* st = status_ptr();
+    if (!st) return FP4_ERR_CUDA;
+    return cuda_status(launch_quantize_blocks(W, N, K, group, (int)gran, heads, (int)fmt, bias_index, chan_shift,
+                                              (int)sdt, packed, scales, jmap, workspace, tables(), st, stream));
+}
+
+fp4_status fp4_act_quantize(const uint16_t* X, int M, int K, const int8_t* shift, const float* rho, fp4_format fmt,
+                            int j, uint8_t* packed, float* a_scale, cudaStream_t stream) {
+    if (M < 0 || K < 0) return FP4_ERR_INVALID_ARG;
+    if (fmt < FP4_E1M2 || fmt > FP4_E3M0 || j < 0 || j > 7) return FP4_ERR_INVALID_ARG;
+    if (K % 8 != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if (!rho || !a_scale) return FP4_ERR_INVALID_ARG;
+    if (!aligned(rho, 4) || !aligned(a_scale, 4)) return FP4_ERR_MISALIGNED;
+    if ((long long)M * K > 0) {
+        if (!X || !packed) return FP4_ERR_INVALID_ARG;
+        if (!aligned(X, 16) || !aligned(packed, 16)) return FP4_ERR_MISALIGNED;
+        if (shift && !aligned(shift, 16)) return FP4_ERR_MISALIGNED;
+    }
+    int* st = status_ptr();
+    if (!st) return FP4_ERR_CUDA;
+    return cuda_status(launch_act_quantize(X, M, K, shift, rho, tables(), (int)fmt, j, packed, a_scale, st, stream));
+}
+
+// The W4A4 workspace: the GEMM's own (counter block first), then the
+// expanded activations [M][K] bf16.
+static size_t w4a4_gemm_part(int M, int N, int K) { return (fp4_gemm_workspace_size(M, N, K) + 255) & ~(size_t)255; }
+
+size_t fp4_gemm_w4a4_workspace_size(int M, int N, int K) {
+    if (M <= 0 || N <= 0 || K <= 0) return 0;
+    return w4a4_gemm_part(M, N, K) + (((size_t)M * K * 2 + 255) & ~(size_t)255);
+}
+
+fp4_status fp4_gemm_w4a4(const uint8_t* apacked, fp4_format afmt, const float* a_scale, const uint8_t* packed,
+                         const void* scales, fp4_scale_dtype sdt, fp4_format fmt, int M, int N, int K, int group,
+                         fp4_act act, uint16_t* Y, void* workspace, size_t ws_bytes, cudaStream_t stream) {
+    if (M < 0) return FP4_ERR_INVALID_ARG;
+    if (afmt < FP4_E1M2 || afmt > FP4_E3M0) return FP4_ERR_INVALID_ARG;
+    if (act != FP4_ACT_NONE && act != FP4_ACT_SILU && act != FP4_ACT_GELU && act != FP4_ACT_SILU_GATE)
+        return FP4_ERR_INVALID_ARG;
+    fp4_status s = check_weights(packed, scales, sdt, fmt, N, K, group);
+    if (s != FP4_OK) return s;
+    if ((long long)M * N * K == 0)  // K == 0 (or nothing to write): fp4_gemm_act's own rules
+        return fp4_gemm_act(nullptr, packed, scales, sdt, fmt, M, N, K, group, a_scale, act, Y, workspace, ws_bytes,
+                            FP4_ENGINE_AUTO, 0, stream);
+    if (!apacked || !a_scale || !Y) return FP4_ERR_INVALID_ARG;
+    if (!aligned(apacked, 16) || !aligned(a_scale, 4)) return FP4_ERR_MISALIGNED;
+    if (!workspace || ws_bytes < fp4_gemm_w4a4_workspace_size(M, N, K)) return FP4_ERR_WORKSPACE;
+    if (!aligned(workspace, 16)) return FP4_ERR_MISALIGNED;
+    if ((const void*)Y == (const void*)apacked) return FP4_ERR_INVALID_ARG;
+    const size_t gpart = w4a4_gemm_part(M, N, K);
+    uint16_t* Xv = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(workspace) + gpart);
+    cudaError_t e = launch_act_expand(apacked, (long long)M * K, tables().f[afmt], Xv, stream);
+    if (e != cudaSuccess) return FP4_ERR_CUDA;
+    return fp4_gemm_act(Xv, packed, scales, sdt, fmt, M, N, K, group, a_scale, act, Y, workspace, gpart,
+                        FP4_ENGINE_AUTO, 0, stream);
 }
 
 fp4_status fp4_dequantize(const uint8_t* packed, const void* scales, fp4_scale_dtype sdt, fp4_format fmt, int N,

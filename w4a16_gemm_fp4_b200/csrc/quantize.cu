@@ -18,6 +18,8 @@
 // Arithmetic that decides a code is IEEE binary32 with round-to-nearest
 // (__fmul_rn / __fdiv_rn, never contracted), so codes and scales are
 // bit-identical to the CPU oracle.
+#include <cstring>
+
 #include "common.cuh"
 
 namespace fp4 {
@@ -324,6 +326,285 @@ __global__ void sse_single_finalize_kernel(const double* ws, int nblocks, int fm
     sse_out[fmt * 8 + j] = acc;
 }
 
+// ------------------------------------------------------ scale granularity
+// The absmax behind a scale is taken over a block: g elements of a row
+// (group, as in quantize_kernel), a whole row (output channel) or
+// rows_per_block consecutive rows (one attention head); the block's scale
+// goes into every group slot it covers, so the GEMM reads the usual
+// [N][K/group] layout.  Channel and head blocks need K % 128 == 0: a
+// 128-element unit then lies in one row, hence in one block.  With a bias
+// search each block takes the index j with the smallest SSE over its own
+// elements (first strict minimum); the format stays the tensor's.
+
+struct BlkParams {
+    QuantParams q;
+    int gran;             // FP4_GRAN_*
+    int rows_per_block;   // channel: 1, head: N / heads
+    const float* blockA;  // [blocks] absmax of W' per channel / head block
+    const int8_t* jsel;   // [blocks] bias index per channel / head block, or null
+    int8_t* jmap;         // [blocks] out: bias index per group block, or null
+    int j;                // fixed bias index, or -1: per-group search
+};
+
+__device__ __forceinline__ float warp_max(float a) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    return a;
+}
+
+// Butterfly sum over the whole warp: every lane ends with the same bits
+// (each step adds a pair in both orders, and IEEE addition commutes).
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Channel / head blocks: absmax of W' per block (float bits of a
+// non-negative value order like unsigned integers: atomicMax on the bits).
+__global__ void __launch_bounds__(kQuantThreads) block_absmax_kernel(QuantParams p, int rows_per_block,
+                                                                     unsigned* blockA) {
+    const int lane = threadIdx.x & 31;
+    const long long units = p.total / 128;
+    const long long wid = (long long)blockIdx.x * (kQuantThreads / 32) + (threadIdx.x >> 5);
+    const long long nw = (long long)gridDim.x * (kQuantThreads / 32);
+    bool bad = false;
+    for (long long u = wid; u < units; u += nw) {
+        float w[4];
+        load4(p, u * 128, w);
+        float a = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            bad |= !isfinite(w[i]);
+            a = fmaxf(a, fabsf(w[i]));
+        }
+        a = warp_max(a);
+        if (lane == 0) atomicMax(&blockA[(int)((u * 128) / p.K) / rows_per_block], __float_as_uint(a));
+    }
+    if (bad) raise_status(p.status, kStatusNonfinite);
+}
+
+// Channel / head blocks with a bias search: the 8 candidates' SSE of every
+// 128-element unit, usse[unit][j] (summed per block in unit order below,
+// so the choice does not depend on timing).
+__global__ void __launch_bounds__(kQuantThreads) block_sse_kernel(QuantParams p, FmtTables tabs, int fmt,
+                                                                  int rows_per_block, const float* blockA,
+                                                                  double* usse) {
+    const FmtTable& t = tabs.f[fmt];
+    const int lane = threadIdx.x & 31;
+    const long long units = p.total / 128;
+    const long long wid = (long long)blockIdx.x * (kQuantThreads / 32) + (threadIdx.x >> 5);
+    const long long nw = (long long)gridDim.x * (kQuantThreads / 32);
+    for (long long u = wid; u < units; u += nw) {
+        float w[4];
+        load4(p, u * 128, w);
+        const float A = blockA[(int)((u * 128) / p.K) / rows_per_block];
+#pragma unroll 1
+        for (int jj = 0; jj < 8; ++jj) {
+            bool o;
+            uint32_t raw;
+            const float s = stored_scale(A, tabs.cj[jj], t.qmax, p.sdt, &o, &raw);
+            double acc = 0.0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float v;
+                code_of(w[i], s, t, &v);
+                const double d = (double)w[i] - (double)v * (double)s;
+                acc = fma(d, d, acc);
+            }
+            acc = warp_sum(acc);
+            if (lane == jj) usse[u * 8 + jj] = acc;
+        }
+    }
+}
+
+// One warp per channel / head block: its units' SSE summed in a fixed
+// order, then the first strict minimum over j.
+__global__ void block_choose_kernel(const double* usse, long long units_per_block, int nblocks, int8_t* jsel) {
+    const int lane = threadIdx.x & 31;
+    const int b = (int)(((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+    if (b >= nblocks) return;  // whole warps leave together
+    double e[8];
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) e[jj] = 0.0;
+    for (long long v = lane; v < units_per_block; v += 32) {
+        const double* row = usse + ((long long)b * units_per_block + v) * 8;
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) e[jj] += row[jj];
+    }
+    int best = 0;
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+        e[jj] = warp_sum(e[jj]);
+        if (e[jj] < e[best]) best = jj;
+    }
+    if (lane == 0) jsel[b] = (int8_t)best;
+}
+
+// Codes and scales for every granularity: the group absmax or the block's
+// precomputed one, a fixed, chosen or (group blocks) searched bias index,
+// then scale-and-clip, compare-and-quantize and packing as in
+// quantize_kernel.
+__global__ void __launch_bounds__(kQuantThreads) quantize_blocks_kernel(BlkParams bp, FmtTables tabs, int fmt) {
+    const QuantParams& p = bp.q;
+    const FmtTable& t = tabs.f[fmt];
+    const int lane = threadIdx.x & 31;
+    const int lpg = p.group >> 2;
+    const long long units = (p.total + 127) / 128;
+    const long long wid = (long long)blockIdx.x * (kQuantThreads / 32) + (threadIdx.x >> 5);
+    const long long nw = (long long)gridDim.x * (kQuantThreads / 32);
+    bool bad = false, ovf = false;
+    for (long long u = wid; u < units; u += nw) {
+        float w[4];
+        const bool valid = load4(p, u * 128, w);
+        float a = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            bad |= valid && !isfinite(w[i]);
+            a = fmaxf(a, fabsf(w[i]));
+        }
+        const float Ag = group_absmax(a, lpg);
+        const long long off = u * 128 + 4 * lane;
+        long long blk;
+        float A;
+        if (bp.gran == FP4_GRAN_GROUP) {
+            blk = off / p.group;
+            A = Ag;
+        } else {
+            blk = valid ? (off / p.K) / bp.rows_per_block : 0;
+            A = valid ? bp.blockA[blk] : 0.f;
+        }
+        int j = bp.j;
+        if (j < 0 && bp.jsel) {
+            j = valid ? bp.jsel[blk] : 0;
+        } else if (j < 0) {
+            // per-group search: the group's SSE for every candidate (a sum
+            // over its lanes, identical bits in all of them)
+            double best = 0.0;
+            j = 0;
+#pragma unroll 1
+            for (int jj = 0; jj < 8; ++jj) {
+                bool o;
+                uint32_t raw;
+                const float s = stored_scale(A, tabs.cj[jj], t.qmax, p.sdt, &o, &raw);
+                double acc = 0.0;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float v;
+                    code_of(w[i], s, t, &v);
+                    const double d = (double)w[i] - (double)v * (double)s;
+                    acc = fma(d, d, acc);
+                }
+                for (int o2 = 1; o2 < lpg; o2 <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o2);
+                if (jj == 0 || acc < best) {
+                    best = acc;
+                    j = jj;
+                }
+            }
+        }
+        if (!valid) continue;
+        bool o;
+        uint32_t raw;
+        const float s = stored_scale(A, tabs.cj[j], t.qmax, p.sdt, &o, &raw);
+        ovf |= o;
+        uint32_t codes = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float v;
+            codes |= (uint32_t)code_of(w[i], s, t, &v) << (4 * i);
+        }
+        *reinterpret_cast<uint16_t*>(p.packed + off / 2) = (uint16_t)codes;
+        if ((lane & (lpg - 1)) == 0) {
+            const long long gi = off / p.group;
+            if (p.sdt == FP4_SCALE_F16)
+                reinterpret_cast<uint16_t*>(p.scales)[gi] = (uint16_t)raw;
+            else
+                reinterpret_cast<uint32_t*>(p.scales)[gi] = raw;
+            if (bp.jmap && bp.gran == FP4_GRAN_GROUP) bp.jmap[blk] = (int8_t)j;
+        }
+    }
+    if (bad) raise_status(p.status, kStatusNonfinite);
+    if (ovf) raise_status(p.status, kStatusScaleOverflow);
+}
+
+// ------------------------------------------------------ 4-bit activations
+// Codes of X' = X * 2^-shift[k] against one per-tensor scale
+// s_a = fl32(fl32(rho * c_j) / Qmax) (the per-channel power of two of the
+// pre-shifted exponent bias lives in the weights).  Eight elements per
+// thread: one 16-byte load of X, one 4-byte store of codes.  The nearest-
+// code decisions use the exact thresholds of code_threshold (no division
+// per element).  HBM-bound: 2 B read + 0.5 B written per element.
+__global__ void __launch_bounds__(256) act_quantize_kernel(const uint4* __restrict__ X, long long nvec, int K,
+                                                           const int8_t* __restrict__ shift,
+                                                           const float* __restrict__ rho, FmtTables tabs, int fmt,
+                                                           int j, uint32_t* __restrict__ packed, float* a_scale,
+                                                           int* status) {
+    const FmtTable& t = tabs.f[fmt];
+    const float r = *rho;
+    const bool rho_ok = r > 0.f && isfinite(r);
+    const float s = __fdiv_rn(__fmul_rn(r, tabs.cj[j]), t.qmax);
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        *a_scale = rho_ok ? s : __int_as_float(0x7fc00000);
+        if (!rho_ok) raise_status(status, kStatusNonfinite);
+    }
+    float T[7];
+#pragma unroll
+    for (int i = 0; i < 7; ++i) T[i] = code_threshold(tabs.hb[fmt][i], (tabs.tie_up[fmt] >> i) & 1u, s);
+    bool bad = false;
+    for (long long v = (long long)blockIdx.x * blockDim.x + threadIdx.x; v < nvec;
+         v += (long long)gridDim.x * blockDim.x) {
+        const uint4 x = __ldg(X + v);
+        const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+        int8_t e[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        if (shift) {
+            const uint2 sh = __ldg(reinterpret_cast<const uint2*>(shift + (v * 8) % K));
+            const uint32_t shw[2] = {sh.x, sh.y};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) e[i] = (int8_t)(shw[i >> 2] >> (8 * (i & 3)));
+        }
+        uint32_t codes = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            float xv = __uint_as_float((i & 1) ? (xw[i >> 1] & 0xffff0000u) : (xw[i >> 1] << 16));
+            bad |= !isfinite(xv);
+            if (shift) xv = __fmul_rn(xv, pow2i(-(int)e[i]));
+            const float ax = fabsf(xv);
+            int idx = 0;
+#pragma unroll
+            for (int k = 0; k < 7; ++k) idx += ax >= T[k] ? 1 : 0;
+            codes |= (uint32_t)((signbit(xv) ? 8 : 0) | idx) << (4 * i);
+        }
+        packed[v] = codes;
+    }
+    if (bad) raise_status(status, kStatusNonfinite);
+}
+
+// The values of 4-bit activation codes as bf16 (exact: every magnitude of
+// the three formats has at most 3 significant bits), for the 16-bit tensor
+// path of the W4A4 product.  Eight codes per thread: a 4-byte load, a
+// 16-byte store.
+struct CodeTable16 {
+    uint16_t v[16];
+};
+
+__global__ void __launch_bounds__(256) act_expand_kernel(const uint32_t* __restrict__ codes, long long nwords,
+                                                         CodeTable16 tab, uint4* __restrict__ out) {
+    __shared__ uint16_t tv[16];
+    if (threadIdx.x < 16) tv[threadIdx.x] = tab.v[threadIdx.x];
+    __syncthreads();
+    pdl_launch_dependents();
+    pdl_wait();  // the codes may come from the previous kernel in the stream
+    for (long long w = (long long)blockIdx.x * blockDim.x + threadIdx.x; w < nwords;
+         w += (long long)gridDim.x * blockDim.x) {
+        const uint32_t c = __ldg(codes + w);
+        uint32_t o[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            o[i] = (uint32_t)tv[(c >> (8 * i)) & 15] | ((uint32_t)tv[(c >> (8 * i + 4)) & 15] << 16);
+        out[w] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
 // ----------------------------------------------------------- host launch
 
 int quantize_grid_blocks(long long total) {
@@ -414,6 +695,115 @@ cudaError_t launch_dequantize(const uint8_t* packed, const void* scales, int sdt
     if (blocks < 1) blocks = 1;
     dequantize_kernel<<<(int)blocks, 256, 0, st>>>(reinterpret_cast<const uint32_t*>(packed), scales, sdt, t,
                                                    words, K, group, out);
+    return cudaGetLastError();
+}
+
+
+// ------------------------------------------- granularity / activations: host
+
+static long long blk_count(int N, int K, int group, int gran, int heads) {
+    if (gran == FP4_GRAN_GROUP) return (long long)N * (K / group);
+    return gran == FP4_GRAN_CHANNEL ? N : heads;
+}
+
+static size_t up256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+size_t quantize_blocks_ws_bytes(int N, int K, int group, int gran, int heads, bool search) {
+    if (gran == FP4_GRAN_GROUP || (long long)N * K == 0) return 0;
+    const long long nb = blk_count(N, K, group, gran, heads);
+    size_t b = up256((size_t)nb * 4);
+    if (search) b += up256((size_t)N * K / 128 * 8 * sizeof(double)) + up256((size_t)nb);
+    return b;
+}
+
+cudaError_t launch_quantize_blocks(const float* W, int N, int K, int group, int gran, int heads, int fmt, int j,
+                                   const int8_t* shift, int sdt, uint8_t* packed, void* scales, int8_t* jmap,
+                                   void* ws, const FmtTables& tabs, int* status, cudaStream_t st) {
+    BlkParams bp;
+    QuantParams& p = bp.q;
+    p.W = W;
+    p.shift = shift;
+    p.total = (long long)N * K;
+    p.K = K;
+    p.group = group;
+    p.sdt = sdt;
+    p.packed = packed;
+    p.scales = scales;
+    p.status = status;
+    bp.gran = gran;
+    bp.rows_per_block = gran == FP4_GRAN_HEAD ? N / heads : 1;
+    bp.blockA = nullptr;
+    bp.jsel = nullptr;
+    bp.jmap = jmap;
+    bp.j = j;
+    const long long nb = blk_count(N, K, group, gran, heads);
+    const int blocks = quantize_grid_blocks(p.total);
+    cudaError_t e = cudaSuccess;
+    if (gran != FP4_GRAN_GROUP) {
+        uint8_t* w8 = static_cast<uint8_t*>(ws);
+        float* blockA = reinterpret_cast<float*>(w8);
+        e = cudaMemsetAsync(blockA, 0, (size_t)nb * 4, st);
+        if (e != cudaSuccess) return e;
+        block_absmax_kernel<<<blocks, kQuantThreads, 0, st>>>(p, bp.rows_per_block, reinterpret_cast<unsigned*>(blockA));
+        bp.blockA = blockA;
+        if (j < 0) {
+            double* usse = reinterpret_cast<double*>(w8 + up256((size_t)nb * 4));
+            int8_t* jsel = jmap ? jmap
+                                : reinterpret_cast<int8_t*>(w8 + up256((size_t)nb * 4) +
+                                                            up256((size_t)p.total / 128 * 8 * sizeof(double)));
+            block_sse_kernel<<<blocks, kQuantThreads, 0, st>>>(p, tabs, fmt, bp.rows_per_block, blockA, usse);
+            const long long upb = (long long)bp.rows_per_block * (K / 128);
+            block_choose_kernel<<<(int)((nb * 32 + 255) / 256), 256, 0, st>>>(usse, upb, (int)nb, jsel);
+            bp.jsel = jsel;
+            bp.jmap = nullptr;
+        } else if (jmap) {
+            e = cudaMemsetAsync(jmap, j, (size_t)nb, st);
+            if (e != cudaSuccess) return e;
+            bp.jmap = nullptr;
+        }
+    }
+    quantize_blocks_kernel<<<blocks, kQuantThreads, 0, st>>>(bp, tabs, fmt);
+    stream_boundary_kernel<<<1, 32, 0, st>>>();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_act_quantize(const uint16_t* X, int M, int K, const int8_t* shift, const float* rho,
+                                const FmtTables& tabs, int fmt, int j, uint8_t* packed, float* a_scale, int* status,
+                                cudaStream_t st) {
+    const long long nvec = (long long)M * K / 8;
+    long long blocks = (nvec + 255) / 256;
+    if (blocks > 148 * 8) blocks = 148 * 8;
+    if (blocks < 1) blocks = 1;
+    act_quantize_kernel<<<(int)blocks, 256, 0, st>>>(reinterpret_cast<const uint4*>(X), nvec, K, shift, rho, tabs, fmt,
+                                                      j, reinterpret_cast<uint32_t*>(packed), a_scale, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_act_expand(const uint8_t* codes, long long count, const FmtTable& t, uint16_t* out,
+                              cudaStream_t st) {
+    CodeTable16 tab;
+    for (int c = 0; c < 16; ++c) {
+        const float v = (c & 8) ? -t.mag[c & 7] : t.mag[c & 7];
+        uint32_t b;
+        memcpy(&b, &v, 4);
+        tab.v[c] = (uint16_t)(b >> 16);  // exact: at most 3 significant bits
+    }
+    const long long nwords = count / 8;
+    long long blocks = (nwords + 255) / 256;
+    if (blocks > 148 * 8) blocks = 148 * 8;
+    if (blocks < 1) blocks = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(256);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, act_expand_kernel, reinterpret_cast<const uint32_t*>(codes), nwords, tab,
+                                       reinterpret_cast<uint4*>(out));
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
