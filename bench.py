@@ -491,7 +491,29 @@ def run_parts(api, torch, peaks, dev, stream):
     ws_cal = torch.zeros(api.lib().fp4_preshift_workspace_size(*X.shape), dtype=torch.uint8, device=dev)
     ms_pro = time_graph(torch, lambda: api.preshift_apply(X, shift, rho, out=Xt), stream, 20)
     out["preshift_apply"] = {"ms": round(ms_pro, 4), "gbs": round(2 * 2 * X.numel() / (ms_pro * 1e-3) / 1e9, 1)}
-    del X, Xt, qs, ys, ws_cal
+    # the same prefill with 4-bit activations: activation codes against the
+    # calibrated per-tensor scale (the channel powers of two are in the
+    # weights), then the W4A4 product on the same weights
+    ap, a_scale = api.act_quantize(X, rho, api.E2M1, 0, shift)
+    ms_aq = time_graph(torch, lambda: api.act_quantize(X, rho, api.E2M1, 0, shift, out=ap, a_scale=a_scale),
+                       stream, 20)
+    aq_bytes = 2.5 * X.numel()
+    out["act_quantize"] = {"workload": "X bf16 2048x4096 (1% outlier channels x50) -> E2M1 codes, pre-shift on",
+                           "ms": round(ms_aq, 4), "gbs": round(aq_bytes / (ms_aq * 1e-3) / 1e9, 1),
+                           "frac_hbm": round(aq_bytes / (ms_aq * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
+    ws4 = torch.zeros(max(api.gemm_w4a4_workspace_size(X.shape[0], N, K) for (N, K) in
+                          ((4096, 4096), (11008, 4096))), dtype=torch.uint8, device=dev)
+
+    def prefill_w4a4():
+        api.act_quantize(X, rho, api.E2M1, 0, shift, out=ap, a_scale=a_scale)
+        for q, y in zip(qs, ys):
+            api.gemm_w4a4(ap, a_scale, q["packed"], q["scales"], api.E2M1, api.E2M1, GROUP, out=y, workspace=ws4)
+    ms = time_graph(torch, prefill_w4a4, stream, 20)
+    tf = flops / (ms * 1e-3) / 1e12
+    out["w4a4_prefill"] = {"workload": "LLaMA-7B prefill in W4A4: act_quantize of X 2048x4096 + the product on "
+                                       "W 4096x4096 + 11008x4096; each call includes its activation expansion",
+                           "ms": round(ms, 4), "tflops": round(tf, 1), "frac": round(tf / peaks["bf16_tflops"], 4)}
+    del X, Xt, qs, ys, ws_cal, ap, a_scale, ws4
     # LLaMA-13B search workload: the per-tensor format/bias search (3 formats
     # x 8 bias candidates, then the pack) on each Student-t matrix, then the
     # W4A16 GEMM at M = 512 on the searched weights
@@ -520,6 +542,22 @@ def run_parts(api, torch, peaks, dev, stream):
             "ms": round(ms, 4), "tflops": round(tf, 1), "frac": round(tf / peaks["bf16_tflops"], 4),
             "frac_of_spec": round(tf / SPEC_BF16_TFLOPS, 4)}
         del o, Y
+    # scale granularity on the 13B projections: one scale per attention
+    # head (40 heads of 128 rows) with the bias searched per head on the q
+    # projection, and one per output channel on the gate projection
+    out["quantize_blocks"] = {}
+    for (W_np, gran, heads, bias, name) in ((case["W"][0], api.GRAN_HEAD, 40, -1, "head40_search"),
+                                            (case["W"][1], api.GRAN_CHANNEL, 0, 0, "channel")):
+        N, K = W_np.shape
+        W = torch.from_numpy(W_np).cuda()
+        ms = time_graph(torch, lambda: api.quantize_blocks(W, GROUP, gran, heads, api.E2M1, bias), stream, 5,
+                        warm=1)
+        out["quantize_blocks"]["%dx%d_%s" % (N, K, name)] = {
+            "workload": "%dx%d Student-t(5)*0.015, E2M1, scales per %s%s" % (
+                N, K, "attention head (40 x 128 rows)" if heads else "output channel",
+                ", bias index searched per block" if bias < 0 else ""),
+            "ms": round(ms, 4), "weight_gbs_read": round(4.0 * N * K / (ms * 1e-3) / 1e9, 1)}
+        del W
     return out
 
 
@@ -635,13 +673,17 @@ def cpu_baselines():
             "single_thread": {"value": round(gbs1, 5), "unit": "GB/s", "cores": 1, "sample": desc1}}
 
 
-def cpu_configs(threads_list=(0, 1)):
-    """The oracle on the host cores for every configuration: configs 1-4 in
-    full (quantize/search/pack and GEMM, as the workloads define them) and
-    config 5 extrapolated from one matrix of each of its three shapes
-    (x 4, 2 and 1 per layer, x 40 layers; the M = 2048 prefill GEMM of that
-    sample is itself extrapolated from its first 64 rows, the oracle's work
-    being linear in M).  threads 0 = all host cores.  Returns a dict."""
+def cpu_configs(threads_list=(0, 1), emit=None, single_row_div=16):
+    """The oracle on the host cores for every configuration: configs 1-4
+    (quantize/search/pack and GEMM, as the workloads define them) and config
+    5 extrapolated from one matrix of each of its three shapes (x 4, 2 and 1
+    per layer, x 40 layers; its M = 2048 prefill GEMM from the first 64
+    rows, the oracle's work being linear in M).  threads 0 = all host
+    cores: everything in full.  At one thread the quantizers run in full and
+    each GEMM on the first 1/single_row_div of its weight rows, scaled by
+    the row count (the oracle GEMM is linear in N), so the run stays within
+    tens of minutes.  emit(record) receives each configuration's record as
+    soon as it is done; the dict of all records is returned."""
     import oracle
     from w4a16_gemm_fp4_b200 import synth
     oracle.build()
@@ -654,12 +696,26 @@ def cpu_configs(threads_list=(0, 1)):
         return time.perf_counter() - t0
 
     for th in threads_list:
-        oracle.set_num_threads(th if th > 0 else all_cores)
+        nth = th if th > 0 else all_cores
+        oracle.set_num_threads(nth)
+        div = 1 if nth == all_cores and th == 0 else single_row_div
         r = {}
+
+        def done(name, rec):
+            rec["threads"] = nth
+            rec["gemm_row_sample"] = "full" if div == 1 else "first 1/%d of the weight rows, x%d" % (div, div)
+            r[name] = rec
+            if emit:
+                emit({"config": name, **rec})
+
+        def gemm_s(X, q, N, fmt=oracle.E2M1, rho=1.0):
+            n = max(1, N // div)
+            return t(lambda: oracle.gemm(X, q["packed"][:n], q["scales"][:n], fmt, GROUP, rho)) * (N / n)
+
         c1 = synth.tiny()
         q = oracle.quantize(c1["W"], GROUP, oracle.E2M1, scale_dtype="f32")
-        r["cfg1_tiny"] = {"quantize_s": t(lambda: oracle.quantize(c1["W"], GROUP, oracle.E2M1, scale_dtype="f32")),
-                          "gemm_s": t(lambda: oracle.gemm(c1["X"], q["packed"], q["scales"], oracle.E2M1, GROUP))}
+        done("cfg1_tiny", {"quantize_s": t(lambda: oracle.quantize(c1["W"], GROUP, oracle.E2M1, scale_dtype="f32")),
+                           "gemm_s": t(lambda: oracle.gemm(c1["X"], q["packed"], q["scales"], oracle.E2M1, GROUP))})
         c2 = synth.llama7b_decode()
         qs = []
         tq = 0.0
@@ -667,10 +723,9 @@ def cpu_configs(threads_list=(0, 1)):
             t0 = time.perf_counter()
             qs.append(oracle.quantize(c["W"], GROUP, oracle.E2M1))
             tq += time.perf_counter() - t0
-        tg = sum(t(lambda c=c, qq=qq, M=M: oracle.gemm(c["X"][M], qq["packed"], qq["scales"], oracle.E2M1, GROUP))
-                 for M in MS for c, qq in zip(c2, qs))
-        r["cfg2_llama7b_decode"] = {"quantize_s": tq, "gemm_sweep_s": tg,
-                                    "weight_gbs": step_weight_bytes() / tg / 1e9}
+        tg = sum(gemm_s(c["X"][M], qq, c["W"].shape[0]) for M in MS for c, qq in zip(c2, qs))
+        done("cfg2_llama7b_decode", {"quantize_s": tq, "gemm_sweep_s": tg,
+                                     "weight_gbs": step_weight_bytes() / tg / 1e9})
         del c2, qs
         c3 = synth.llama7b_prefill()
         tc = t(lambda: oracle.preshift_calibrate(c3["X"]))
@@ -684,10 +739,10 @@ def cpu_configs(threads_list=(0, 1)):
             t0 = time.perf_counter()
             qq = oracle.quantize(W, GROUP, oracle.E2M1, shift=shift)
             tq += time.perf_counter() - t0
-            tg += t(lambda: oracle.gemm(Xt, qq["packed"], qq["scales"], oracle.E2M1, GROUP, rho))
+            tg += gemm_s(Xt, qq, W.shape[0], rho=rho)
             flops += 2.0 * Xt.shape[0] * W.shape[0] * W.shape[1]
-        r["cfg3_llama7b_prefill"] = {"calibrate_s": tc, "apply_s": ta, "quantize_s": tq, "gemm_s": tg,
-                                     "gflops": flops / tg / 1e9}
+        done("cfg3_llama7b_prefill", {"calibrate_s": tc, "apply_s": ta, "quantize_s": tq, "gemm_s": tg,
+                                      "gflops": flops / tg / 1e9})
         del c3, Xt
         c4 = synth.llama13b_search()
         ts = 0.0
@@ -697,9 +752,9 @@ def cpu_configs(threads_list=(0, 1)):
             t0 = time.perf_counter()
             qq = oracle.quantize(W, GROUP, oracle.AUTO, bias_search=True)
             ts += time.perf_counter() - t0
-            tg += t(lambda: oracle.gemm(c4["X"], qq["packed"], qq["scales"], qq["choice"][0], GROUP))
+            tg += gemm_s(c4["X"], qq, W.shape[0], fmt=qq["choice"][0])
             flops += 2.0 * c4["X"].shape[0] * W.shape[0] * W.shape[1]
-        r["cfg4_llama13b_search"] = {"search_and_pack_s": ts, "gemm_m512_s": tg, "gflops": flops / tg / 1e9}
+        done("cfg4_llama13b_search", {"search_and_pack_s": ts, "gemm_m512_s": tg, "gflops": flops / tg / 1e9})
         del c4
         # config 5: one matrix of each shape, counts per layer 4, 2, 1
         rng = np.random.default_rng(4)
@@ -716,12 +771,11 @@ def cpu_configs(threads_list=(0, 1)):
             for M in (1, 4, 16, 64, 2048):
                 Mt = min(M, 64)
                 X = synth.activations(rng, Mt, K)
-                dt = t(lambda: oracle.gemm(X, qq["packed"], qq["scales"], oracle.E2M1, GROUP))
-                per_layer["gemm_M%d_s" % M] += cnt * dt * (M / Mt)
-        r["cfg5_llama13b_stack_extrapolated"] = {k: v * 40 for k, v in per_layer.items()}
-        r["cfg5_llama13b_stack_extrapolated"]["note"] = (
-            "one matrix of each shape timed, x {4,2,1} per layer x 40 layers; M=2048 from its first 64 rows")
-        out["runs"]["threads_%d" % (th if th > 0 else all_cores)] = r
+                per_layer["gemm_M%d_s" % M] += cnt * gemm_s(X, qq, N) * (M / Mt)
+        rec = {k: v * 40 for k, v in per_layer.items()}
+        rec["note"] = "one matrix of each shape timed, x {4,2,1} per layer x 40 layers; M=2048 from its first 64 rows"
+        done("cfg5_llama13b_stack_extrapolated", rec)
+        out["runs"]["threads_%d" % nth] = r
     oracle.set_num_threads(all_cores)
     return out
 
@@ -875,7 +929,7 @@ def main():
             print(cmd)
         return
     if args.cpu_configs:
-        print(json.dumps(cpu_configs(), indent=1), flush=True)
+        cpu_configs(emit=lambda rec: print(json.dumps(rec), flush=True))
         return
     if args.profile_case:
         profile_case(args.profile_case)
