@@ -134,10 +134,11 @@ FP4_API fp4_status fp4_quantize(const float *W, int N, int K, int group, fp4_for
 /* ------------------------------------------------------------------------
  * fp4_quantize_blocks -- fp4_quantize with the scale's absmax taken over a
  * coarser block, and the bias index chosen per block.  (Granularities of
- * the HiFloat4 page, section 3.1 "权重量化策略", scales grouped per
- * attention head, and of the quantization-basics page, the per-tensor /
- * per-channel / per-token classification: per output channel; the search
- * of the LLM-FP4 summary page applied to each block instead of the tensor.)
+ * the HiFloat4 page, section 3.1 "权重量化策略": scales grouped per
+ * attention head; of the "量化技术详解" page, section "量化分类" by
+ * granularity, and the per_channel option of the 4-bit float tutorial,
+ * section 4.2: one scale per output channel; the search of the LLM-FP4
+ * summary page applied to each block instead of the whole tensor.)
  *
  *   gran FP4_GRAN_GROUP    block = `group` consecutive k of a row (as
  *                          fp4_quantize);
