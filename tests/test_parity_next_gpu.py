@@ -271,3 +271,29 @@ def test_w4a4_llama7b_prefill_full(fp4, oracle_mod):
     yref = oracle_mod.gemm_w4a4_sampled(ap, 1, s_a, wp, ws, 1, 128, ms, ns).reshape(len(sel), N)
     got = Y.float().cpu().numpy().astype(np.float64)[sel]
     assert float(np.max(np.abs(got - yref)) / np.max(np.abs(yref))) <= TOL
+
+
+@pytest.mark.parametrize("M,N,K", [(65, 256, 512), (128, 384, 1024), (300, 200, 768), (2048, 256, 4096)])
+def test_gemm_w4a4_native_matches_expand(fp4, oracle_mod, M, N, K):
+    """E2M1 x E2M1 from M = 65 runs on kind::f8f6f4 MMAs with no
+    dequantization; codes at a 16- (not 32-) byte offset take the expanding
+    16-bit path.  Both meet the bound against the oracle."""
+    ap, s_a, wp, ws, gap, gs = w4a4_case(fp4, oracle_mod, 98 + M, M, N, K)
+    gw, gsc = torch.from_numpy(wp).cuda(), torch.from_numpy(ws).cuda()
+    ref = oracle_mod.gemm_w4a4(ap, 1, s_a, wp, ws, 1, 128)
+    Yn = fp4.gemm_w4a4(gap, gs, gw, gsc, 1, 1, 128)
+    buf = torch.empty(gap.numel() + 16, dtype=torch.uint8, device="cuda")
+    shifted = buf[16:].view(gap.shape)
+    shifted.copy_(gap)
+    assert shifted.data_ptr() % 32 == 16
+    Ye = fp4.gemm_w4a4(shifted, gs, gw, gsc, 1, 1, 128)
+    assert rel_err(Yn, ref) <= TOL and rel_err(Ye, ref) <= TOL
+
+
+@pytest.mark.parametrize("M", [65, 200])
+def test_gemm_w4a4_native_ragged_and_formats(fp4, oracle_mod, M):
+    """Ragged N and M tails on the native path, fp32 weight scales, a
+    shifted activation bias index."""
+    ap, s_a, wp, ws, gap, gs = w4a4_case(fp4, oracle_mod, 99, M, 130, 384, 1, 1, 5, "f32")
+    Y = fp4.gemm_w4a4(gap, gs, torch.from_numpy(wp).cuda(), torch.from_numpy(ws).cuda(), 1, 1, 128)
+    assert rel_err(Y, oracle_mod.gemm_w4a4(ap, 1, s_a, wp, ws, 1, 128)) <= TOL

@@ -59,6 +59,10 @@ cudaError_t launch_act_quantize(const uint16_t* X, int M, int K, const int8_t* s
                                 cudaStream_t st);
 cudaError_t launch_act_expand(const uint8_t* codes, long long count, const FmtTable& t, uint16_t* out,
                               cudaStream_t st);
+bool w4a4_native_fits(int afmt, int fmt, int M, int N, int K, int group, const void* apacked, const void* packed);
+cudaError_t launch_gemm_w4a4(const uint8_t* apacked, const float* a_scale, const uint8_t* packed, const void* scales,
+                             int sdt, int M, int N, int K, uint16_t* Y, int act, int* status,
+                             unsigned long long timeout_ns, cudaStream_t st);
 int noalloc_max_k();
 cudaError_t launch_calibrate_noalloc(const uint16_t* X, int M, int K, int8_t* shift, float* rho, int* status,
                                      cudaStream_t st);
@@ -317,6 +321,14 @@ fp4_status fp4_gemm_w4a4(const uint8_t* apacked, fp4_format afmt, const float* a
     if (!workspace || ws_bytes < fp4_gemm_w4a4_workspace_size(M, N, K)) return FP4_ERR_WORKSPACE;
     if (!aligned(workspace, 16)) return FP4_ERR_MISALIGNED;
     if ((const void*)Y == (const void*)apacked) return FP4_ERR_INVALID_ARG;
+    if (act == FP4_ACT_SILU_GATE && (N % 2 != 0 || group != 128)) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if (w4a4_native_fits((int)afmt, (int)fmt, M, N, K, group, apacked, packed)) {
+        // E2M1 x E2M1 from M = 65: both code tiles straight into kind::f8f6f4 MMAs
+        int* st = status_ptr();
+        if (!st) return FP4_ERR_CUDA;
+        return cuda_status(launch_gemm_w4a4(apacked, a_scale, packed, scales, (int)sdt, M, N, K, Y, (int)act, st,
+                                            (unsigned long long)g_timeout_us * 1000ull, stream));
+    }
     const size_t gpart = w4a4_gemm_part(M, N, K);
     uint16_t* Xv = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(workspace) + gpart);
     cudaError_t e = launch_act_expand(apacked, (long long)M * K, tables().f[afmt], Xv, stream);

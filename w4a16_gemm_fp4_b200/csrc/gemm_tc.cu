@@ -922,6 +922,23 @@ bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, int elem_bytes, const v
     return r == CUDA_SUCCESS;
 }
 
+// 4-bit codes, packed two per byte in rows of `elems` codes, copied as
+// 16 x U4 with 16-byte alignment: every 16 codes (8 bytes) land in a
+// 16-byte slot of shared memory, the operand layout of kind::f8f6f4 MMAs.
+// Boxes of 128 codes x box_rows rows under the 128-byte swizzle.
+bool encode_2d_u4(CUtensorMap* map, const void* base, uint64_t elems, uint64_t rows, uint32_t box_rows) {
+    EncodeTiledFn fn = get_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {elems, rows};
+    cuuint64_t strides[1] = {elems / 2};
+    cuuint32_t box[2] = {128, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // A 3-D view {inner, mid, outer} with byte strides {mid_stride, outer_stride},
 // no swizzle (used for L2 prefetches of several consecutive segments per row).
 bool encode_3d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t mid,
