@@ -18,6 +18,10 @@
 // fp32; fold warps then add s[n,g] * acc to fp32 totals, as in the W4A16
 // tensor engine, and the epilogue multiplies by s_a.
 //
+// Six shared-memory stages keep copies in flight across the ~1 us latency
+// of a TMA load; four TMEM accumulators (all 512 columns) decouple the
+// MMAs from the fold.
+//
 // Warp roles (2 + NF warps, one CTA per SM):
 //   warp 0   TMA producer: the first ring-full of weight codes before the
 //            dependency wait, activation codes after it;
@@ -48,14 +52,16 @@ struct W4Cfg {
     static constexpr int ABYTES = BW * KB;       // weight codes in shared memory (one byte per code)
     static constexpr int BBYTES = BT * KB;       // activation codes in shared memory
     static constexpr int TX = (BW + BT) * KB / 2;  // bytes the two copies deliver (packed codes)
-    static constexpr int STG = 4;                // stages == TMEM accumulators
+    static constexpr int SST = BT == 256 ? 4 : 6;  // shared-memory stages (copies in flight)
+    static constexpr int ACC = 512 / BT;         // TMEM accumulators (all 512 columns)
     static constexpr int FCOLS = 64;             // accumulator columns per fold thread
+    static constexpr int LDB = BT == 256 ? 16 : 64;  // TMEM columns loaded per wait (register budget)
     static constexpr int NF = 4 * (BT / FCOLS);  // fold warps
     static constexpr int FW0 = 2;
     static constexpr int THREADS = (FW0 + NF) * 32;
-    static constexpr int TMEM_COLS = STG * BT;
-    static constexpr int NBAR = 3 * STG;
-    static constexpr int SMEM = STG * (ABYTES + BBYTES) + 1024 + NBAR * 8 + 16;
+    static constexpr int TMEM_COLS = ACC * BT;
+    static constexpr int NBAR = 2 * SST + 2 * ACC;
+    static constexpr int SMEM = SST * (ABYTES + BBYTES) + 1024 + NBAR * 8 + 16;
     static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation is a power of two");
     static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 };
@@ -87,13 +93,14 @@ __global__ void __launch_bounds__(W4Cfg<BT>::THREADS, 1)
     using C = W4Cfg<BT>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* ws = smem;                      // STG x ABYTES: weight codes
-    uint8_t* xs = ws + C::STG * C::ABYTES;   // STG x BBYTES: activation codes
-    uint64_t* bars = reinterpret_cast<uint64_t*>(xs + C::STG * C::BBYTES);
-    uint64_t* full = bars;                   // both tiles of the stage landed
-    uint64_t* kdone = full + C::STG;         // the stage's MMAs completed (stage free, accumulator ready)
-    uint64_t* gempty = kdone + C::STG;       // accumulator folded
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gempty + C::STG);
+    uint8_t* ws = smem;                      // SST x ABYTES: weight codes
+    uint8_t* xs = ws + C::SST * C::ABYTES;   // SST x BBYTES: activation codes
+    uint64_t* bars = reinterpret_cast<uint64_t*>(xs + C::SST * C::BBYTES);
+    uint64_t* full = bars;                   // [SST] both tiles of the stage landed
+    uint64_t* sfree = full + C::SST;         // [SST] the stage's MMAs have read it
+    uint64_t* kdone = sfree + C::SST;        // [ACC] the accumulator's MMAs completed
+    uint64_t* gempty = kdone + C::ACC;       // [ACC] accumulator folded
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gempty + C::ACC);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = blockIdx.x * C::BW, m0 = blockIdx.y * BT;
@@ -101,10 +108,13 @@ __global__ void __launch_bounds__(W4Cfg<BT>::THREADS, 1)
     const uint64_t to = p.timeout_ns;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::STG; ++s) {
+        for (int s = 0; s < C::SST; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&kdone[s], 1);
-            mbar_init(&gempty[s], C::NF);
+            mbar_init(&sfree[s], 1);
+        }
+        for (int a = 0; a < C::ACC; ++a) {
+            mbar_init(&kdone[a], 1);
+            mbar_init(&gempty[a], C::NF);
         }
         fence_mbar_init();
         prefetch_tmap(&tmA);
@@ -121,7 +131,7 @@ __global__ void __launch_bounds__(W4Cfg<BT>::THREADS, 1)
     // weight codes are not written by a kernel still running (see the
     // stream-order rule of the interface), so the first ring-full of them
     // goes out before the dependency wait
-    const int pre = nkb < C::STG ? nkb : C::STG;
+    const int pre = nkb < C::SST ? nkb : C::SST;
     if (warp == 0 && elect_one()) {
         for (int j = 0; j < pre; ++j) {
             mbar_arrive_expect_tx(&full[j], C::TX);
@@ -138,9 +148,9 @@ __global__ void __launch_bounds__(W4Cfg<BT>::THREADS, 1)
             for (int j = 0; j < pre; ++j) tma_load_2d(xs + j * C::BBYTES, &tmA, j * C::KB, m0, &full[j]);
             int issued = pre;
             for (int i = pre; i < nkb; ++i) {
-                const int s = i % C::STG;
+                const int s = i % C::SST;
                 // the stage's previous MMAs have read it
-                if (!mbar_wait(&kdone[s], (uint32_t)((i / C::STG) - 1) & 1u, to)) {
+                if (!mbar_wait(&sfree[s], (uint32_t)((i / C::SST) - 1) & 1u, to)) {
                     raise_status(p.status, kStatusTimeout);
                     break;
                 }
@@ -150,8 +160,8 @@ __global__ void __launch_bounds__(W4Cfg<BT>::THREADS, 1)
                 issued = i + 1;
             }
             // no copy may still be in flight when the CTA leaves
-            for (int i = issued - C::STG < 0 ? 0 : issued - C::STG; i < issued; ++i)
-                if (!mbar_wait(&full[i % C::STG], (uint32_t)(i / C::STG) & 1u, to)) {
+            for (int i = issued - C::SST < 0 ? 0 : issued - C::SST; i < issued; ++i)
+                if (!mbar_wait(&full[i % C::SST], (uint32_t)(i / C::SST) & 1u, to)) {
                     raise_status(p.status, kStatusTimeout);
                     break;
                 }
@@ -165,27 +175,28 @@ __global__ void __launch_bounds__(W4Cfg<BT>::THREADS, 1)
             constexpr uint32_t kWStep = C::ABYTES >> 4, kXStep = C::BBYTES >> 4;
             int committed = 0;
             for (int i = 0; i < nkb; ++i) {
-                const int s = i % C::STG;
-                const uint32_t ph = (uint32_t)(i / C::STG) & 1u;
-                if (!mbar_wait(&full[s], ph, to) || !mbar_wait(&gempty[s], ph ^ 1u, to)) {
+                const int s = i % C::SST, a = i % C::ACC;
+                if (!mbar_wait(&full[s], (uint32_t)(i / C::SST) & 1u, to) ||
+                    !mbar_wait(&gempty[a], ((uint32_t)(i / C::ACC) & 1u) ^ 1u, to)) {
                     raise_status(p.status, kStatusTimeout);
                     break;
                 }
                 tc_fence_after();
                 const uint64_t wd = wdesc0 + (uint64_t)(s * kWStep);
                 const uint64_t xd = xdesc0 + (uint64_t)(s * kXStep);
-                const uint32_t d = tmem + (uint32_t)(s * BT);
+                const uint32_t d = tmem + (uint32_t)(a * BT);
                 // K = 32 codes = 32 bytes of each 128-byte row per MMA
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     tc_mma_f8f6f4(d, wd + (uint64_t)(2 * kk), xd + (uint64_t)(2 * kk), idesc, kk ? 1u : 0u);
-                tc_commit(&kdone[s]);
+                tc_commit(&sfree[s]);
+                tc_commit(&kdone[a]);
                 ++committed;
             }
             // TMEM is freed below: the last commit must have landed
             if (committed > 0) {
                 const int last = committed - 1;
-                if (!mbar_wait(&kdone[last % C::STG], (uint32_t)(last / C::STG) & 1u, to))
+                if (!mbar_wait(&kdone[last % C::ACC], (uint32_t)(last / C::ACC) & 1u, to))
                     raise_status(p.status, kStatusTimeout);
             }
         }
@@ -206,23 +217,25 @@ __global__ void __launch_bounds__(W4Cfg<BT>::THREADS, 1)
         bool ok = true;
         float s_next = (nvalid && nkb > 0) ? load_scale(p.scales, p.sdt, (size_t)n * nkb) : 0.f;
         for (int i = 0; i < nkb; ++i) {
-            const int s = i % C::STG;
+            const int s = i % C::ACC;
             const float sc = s_next;
             if (i + 1 < nkb) s_next = nvalid ? load_scale(p.scales, p.sdt, (size_t)n * nkb + i + 1) : 0.f;
             // the warp decides together: the TMEM loads are warp-collective
-            if (!__all_sync(0xffffffffu, mbar_wait(&kdone[s], (uint32_t)(i / C::STG) & 1u, to))) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&kdone[s], (uint32_t)(i / C::ACC) & 1u, to))) {
                 raise_status(p.status, kStatusTimeout);
                 ok = false;
                 break;
             }
             tc_fence_after();
+            // LDB columns in flight per wait
 #pragma unroll
-            for (int c = 0; c < C::FCOLS; c += 16) {
-                uint32_t v[16];
-                tmem_ld16(tlane + (uint32_t)(s * BT + cb + c), v);
+            for (int c0 = 0; c0 < C::FCOLS; c0 += C::LDB) {
+                uint32_t v[C::LDB];
+#pragma unroll
+                for (int c = 0; c < C::LDB; c += 16) tmem_ld16(tlane + (uint32_t)(s * BT + cb + c0 + c), v + c);
                 tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < 16; ++j) tot[c + j] = fmaf(sc, __uint_as_float(v[j]), tot[c + j]);
+                for (int j = 0; j < C::LDB; ++j) tot[c0 + j] = fmaf(sc, __uint_as_float(v[j]), tot[c0 + j]);
             }
             tc_fence_before();
             __syncwarp();
@@ -265,10 +278,10 @@ bool w4a4_native_fits(int afmt, int fmt, int M, int N, int K, int group, const v
            (reinterpret_cast<uintptr_t>(apacked) & 31) == 0 && (reinterpret_cast<uintptr_t>(packed) & 31) == 0;
 }
 
-cudaError_t launch_gemm_w4a4(const uint8_t* apacked, const float* a_scale, const uint8_t* packed, const void* scales,
-                             int sdt, int M, int N, int K, uint16_t* Y, int act, int* status,
-                             unsigned long long timeout_ns, cudaStream_t st) {
-    constexpr int BT = 128;
+template <int BT>
+static cudaError_t launch_w4a4_bt(const uint8_t* apacked, const float* a_scale, const uint8_t* packed,
+                                  const void* scales, int sdt, int M, int N, int K, uint16_t* Y, int act, int* status,
+                                  unsigned long long timeout_ns, cudaStream_t st) {
     using C = W4Cfg<BT>;
     CUtensorMap ma, mw;
     if (!encode_2d_u4(&ma, apacked, (uint64_t)K, (uint64_t)M, BT)) return cudaErrorInvalidValue;
@@ -307,6 +320,16 @@ cudaError_t launch_gemm_w4a4(const uint8_t* apacked, const float* a_scale, const
     e = cudaLaunchKernelEx(&cfg, gemm_w4a4_kernel<BT>, ma, mw, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
+}
+
+// 256-token tiles (N = 256 MMAs: half the shared-memory operand reads per
+// flop of the 128-token tile) once M fills them; 128 below.
+cudaError_t launch_gemm_w4a4(const uint8_t* apacked, const float* a_scale, const uint8_t* packed, const void* scales,
+                             int sdt, int M, int N, int K, uint16_t* Y, int act, int* status,
+                             unsigned long long timeout_ns, cudaStream_t st) {
+    if (M > 128)
+        return launch_w4a4_bt<256>(apacked, a_scale, packed, scales, sdt, M, N, K, Y, act, status, timeout_ns, st);
+    return launch_w4a4_bt<128>(apacked, a_scale, packed, scales, sdt, M, N, K, Y, act, status, timeout_ns, st);
 }
 
 }  // namespace fp4
