@@ -500,7 +500,13 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
 // Stage s and accumulator s are the same index (STG == NACC): the next use
 // of a stage needs its accumulator folded first, so a stage barrier can
 // never run two phases ahead of the fold warps that wait on it.
-template <int BT>
+// ATM (the f16 path of the 128-token tile): the dequant warps write the
+// weights into tensor memory, the A operand of `tcgen05.mma` taken from
+// TMEM, instead of shared memory.  A stage in shared memory then carries
+// only the activations, which removes a third of its traffic (the 32 KB of
+// dequantized codes written and read back per stage), the limit of the
+// stage period.  TMEM: 3 accumulators x 128 columns + 2 A stages x 64.
+template <int BT, bool ATM = false>
 struct TgCfg {
     static constexpr int BW = 128;              // weight rows per tile (MMA M)
     static constexpr int KB = 128;              // k per stage = one group
@@ -518,10 +524,12 @@ struct TgCfg {
     static constexpr int DQ0 = 2;
     static constexpr int FW0 = DQ0 + DQW;
     static constexpr int THREADS = (FW0 + NF) * 32;
-    static constexpr int TMEM_NEED = STG * BT < 32 ? 32 : STG * BT;
+    static constexpr int NA = 2;                // A stages in TMEM (ATM)
+    static constexpr int ACOL = STG * BT;       // first TMEM column of the A stages (ATM)
+    static constexpr int TMEM_NEED = ATM ? STG * BT + NA * 64 : (STG * BT < 32 ? 32 : STG * BT);
     static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
-    static constexpr int RING = STG * (ABYTES + XBYTES) + WST * WBYTES;
-    static constexpr int NBAR = 4 * STG + 2 * WST;
+    static constexpr int RING = STG * ((ATM ? 0 : ABYTES) + XBYTES) + WST * WBYTES;
+    static constexpr int NBAR = 4 * STG + 2 * WST + (ATM ? NA : 0);
     static constexpr int DEP = DQW * 32 * 4;  // per-dequant-thread scratch words (stage release)
     // per fold warp, the f16 path's row factors of its FCOLS tokens
     static constexpr int XFB = kPair ? 0 : NF * FCOLS * 4;
@@ -531,13 +539,15 @@ struct TgCfg {
     static constexpr int SMEM = RING + SLACK + NBAR * 8 + 16 + DEP + XFB;
     static_assert(!kPair || SMEM + 1024 <= 228 * 1024 / 2, "two CTAs per SM");
     static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
-    static_assert(BT * 128 * 4 <= STG * ABYTES, "split-K partials overlay the dequantized tiles");
+    static_assert(BT * 128 * 4 <= STG * (ATM ? XBYTES : ABYTES), "split-K partials overlay the first stages");
+    static_assert(!ATM || (BT == 128 && TMEM_NEED <= 512), "ATM layout");
 };
 
 template <int BT, bool F16, bool ACT>
-__global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
+__global__ void __launch_bounds__(TgCfg<BT, F16 && BT == 128>::THREADS, TgCfg<BT, F16 && BT == 128>::CTAS_PER_SM)
     gemm_tcg_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, TcParams p) {
-    using C = TgCfg<BT>;
+    constexpr bool ATM = F16 && BT == 128;  // A operand in tensor memory
+    using C = TgCfg<BT, ATM>;
     // The activation epilogues are a separate instantiation: compiled into
     // the plain kernel, they cost the 128-token tile its register budget.
     const int act = ACT ? p.act : kActNone;
@@ -547,8 +557,8 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
         if (threadIdx.x == 0) raise_status(p.status, kStatusLayout);
         return;  // before any barrier, copy or TMEM allocation
     }
-    uint8_t* as = smem;                         // STG x ABYTES: dequantized codes
-    uint8_t* xs = as + C::STG * C::ABYTES;      // STG x XBYTES: activations
+    uint8_t* as = smem;                         // STG x ABYTES: dequantized codes (not with ATM)
+    uint8_t* xs = ATM ? smem : as + C::STG * C::ABYTES;  // STG x XBYTES: activations
     uint8_t* wsr = xs + C::STG * C::XBYTES;     // WST x WBYTES: packed codes
     uint64_t* bars = reinterpret_cast<uint64_t*>(wsr + C::WST * C::WBYTES);
     uint64_t* xfull = bars;                 // activations landed
@@ -557,7 +567,8 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
     uint64_t* wfull = kdone + C::STG;       // packed codes landed
     uint64_t* wempty = wfull + C::WST;      // packed codes read
     uint64_t* gempty = wempty + C::WST;     // accumulator folded (kdone's one arrival is the commit)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gempty + C::STG);
+    uint64_t* aempty = gempty + C::STG;     // ATM: the MMAs have read the A stage
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(aempty + (ATM ? C::NA : 0));
     uint32_t* dep_slots = tmem_slot + 4;
     float* xf_slots = reinterpret_cast<float*>(dep_slots + C::DEP / 4);
     volatile int* wide_fail = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -576,10 +587,12 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STG; ++s) {
             mbar_init(&xfull[s], 1);
-            mbar_init(&afull[s], C::DQW * 32);
+            mbar_init(&afull[s], ATM ? C::DQW : C::DQW * 32);
             mbar_init(&kdone[s], 1);
             mbar_init(&gempty[s], C::NF);
         }
+        if constexpr (ATM)
+            for (int a = 0; a < C::NA; ++a) mbar_init(&aempty[a], 1);
         for (int s = 0; s < C::WST; ++s) {
             mbar_init(&wfull[s], 1);
             mbar_init(&wempty[s], C::DQW * 32);
@@ -658,7 +671,40 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
         __syncwarp();
     } else if (warp == 1) {
         // ----------------------------------------------------- MMA issuer
-        if (elect_one()) {
+        if (ATM && elect_one()) {
+            // A from TMEM: stage i's weights at columns ACOL + (i % NA) * 64
+            const uint32_t idesc = idesc_f16_f32(C::BW, BT);
+            const uint64_t xdesc0 = sw128_desc(smem_u32(xs));
+            constexpr uint32_t kXStep = C::XBYTES >> 4, kXAtom = C::XBOX >> 4;
+            int committed = 0;
+            bool ok = true;
+            for (int i = 0; i < nkb && ok; ++i) {
+                const int s = i % C::STG, a = i % C::NA;
+                if (!mbar_wait(&afull[a], (uint32_t)(i / C::NA) & 1u, to) ||
+                    !mbar_wait(&xfull[s], (uint32_t)(i / C::STG) & 1u, to) ||
+                    !mbar_wait(&gempty[s], ((uint32_t)(i / C::STG) & 1u) ^ 1u, to)) {
+                    raise_status(p.status, kStatusTimeout);
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint64_t xd = xdesc0 + (uint64_t)(s * kXStep);
+                const uint32_t ta = tmem + (uint32_t)(C::ACOL + a * 64);
+                const uint32_t d = tmem + (uint32_t)(s * BT);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    tc_mma_ts(d, ta + (uint32_t)(8 * kk), xd + (uint64_t)((kk >> 2) * kXAtom + 2 * (kk & 3)), idesc,
+                              kk ? 1u : 0u);
+                tc_commit(&aempty[a]);
+                tc_commit(&kdone[s]);
+                ++committed;
+            }
+            if (committed > 0) {
+                const int last = committed - 1;
+                if (!mbar_wait(&kdone[last % C::STG], (uint32_t)(last / C::STG) & 1u, to))
+                    raise_status(p.status, kStatusTimeout);
+            }
+        } else if (!ATM && elect_one()) {
             const uint32_t idesc = F16 ? idesc_f16_f32(C::BW, BT) : idesc_bf16_f32(C::BW, BT);
             const uint64_t adesc0 = sw128_desc(smem_u32(as)), xdesc0 = sw128_desc(smem_u32(xs));
             constexpr uint32_t kAStep = C::ABYTES >> 4, kXStep = C::XBYTES >> 4;
@@ -696,7 +742,48 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
             }
         }
         __syncwarp();
-    } else if (warp >= C::DQ0 && warp < C::FW0) {
+    } else if (ATM && warp >= C::DQ0 && warp < C::FW0) {
+        // ------------------------------------------- dequantize into TMEM
+        // thread = half hh (64 k) of weight row r (its TMEM lane, so the warp
+        // covers the lane quadrant it may access); 8 words -> 32 columns of
+        // f16 pairs (k, k+1), the A layout of kind::f16 from TMEM
+        const int dw = warp - C::DQ0;
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        const int hh = dw >> 2;
+        const int swp = (r >> 1) & 3;  // 64-byte swizzle of the packed stage
+        const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
+        for (int i = 0; i < nkb; ++i) {
+            const int ws = i % C::WST, a = i % C::NA;
+            if (!__all_sync(0xffffffffu, mbar_wait(&wfull[ws], (uint32_t)(i / C::WST) & 1u, to))) {
+                raise_status(p.status, kStatusTimeout);
+                break;
+            }
+            const uint8_t* prow = wsr + ws * C::WBYTES + r * 64;
+            uint32_t words[8];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const uint4 w = lds128_tc(prow + (((u + 2 * hh) ^ swp) << 4));
+                words[4 * u + 0] = w.x;
+                words[4 * u + 1] = w.y;
+                words[4 * u + 2] = w.z;
+                words[4 * u + 3] = w.w;
+            }
+            mbar_arrive_after(&wempty[ws], words[0] ^ words[4], dep_slots + dw * 32 + lane);
+            uint32_t o[32];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) e2m1_to_f16x8(words[c], o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+            if (!__all_sync(0xffffffffu, mbar_wait(&aempty[a], ((uint32_t)(i / C::NA) & 1u) ^ 1u, to))) {
+                raise_status(p.status, kStatusTimeout);
+                break;
+            }
+            tmem_st32(tl + (uint32_t)(C::ACOL + a * 64 + hh * 32), o);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&afull[a]);
+        }
+    } else if (!ATM && warp >= C::DQ0 && warp < C::FW0) {
         // ---------------------------------------------------- dequantize
         // DQW = 4: one thread per weight row (16 words = 128 k per stage);
         // DQW = 8: two threads per row, each one 64-k atom (8 words).
@@ -1114,7 +1201,7 @@ cudaError_t launch_x_rows_to_f16(const uint16_t* X, int M, int K, uint16_t* Xh, 
 
 template <int BT, bool F16>
 static cudaError_t launch_tcg_bt(const CUtensorMap& mx, const CUtensorMap& mw, const TcParams& p, cudaStream_t st) {
-    using C = TgCfg<BT>;
+    using C = TgCfg<BT, F16 && BT == 128>;
     static bool attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
