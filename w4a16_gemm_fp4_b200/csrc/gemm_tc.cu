@@ -500,12 +500,13 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
 // Stage s and accumulator s are the same index (STG == NACC): the next use
 // of a stage needs its accumulator folded first, so a stage barrier can
 // never run two phases ahead of the fold warps that wait on it.
-// ATM (the f16 path of the 128-token tile): the dequant warps write the
-// weights into tensor memory, the A operand of `tcgen05.mma` taken from
-// TMEM, instead of shared memory.  A stage in shared memory then carries
-// only the activations, which removes a third of its traffic (the 32 KB of
-// dequantized codes written and read back per stage), the limit of the
-// stage period.  TMEM: 3 accumulators x 128 columns + 2 A stages x 64.
+// ATM: the dequant warps write the weights into tensor memory, the A
+// operand of `tcgen05.mma` taken from TMEM, instead of shared memory.  A
+// stage in shared memory then carries only the activations, which removes
+// the 32 KB of dequantized codes written and read back per stage, the
+// shared-memory traffic that set the stage period.  TMEM per CTA: STG
+// accumulators x BT columns + 2 A stages x 64 (512 columns at BT = 128,
+// 256 for each of the two CTAs per SM of the smaller tiles).
 template <int BT, bool ATM = false>
 struct TgCfg {
     static constexpr int BW = 128;              // weight rows per tile (MMA M)
@@ -540,13 +541,13 @@ struct TgCfg {
     static_assert(!kPair || SMEM + 1024 <= 228 * 1024 / 2, "two CTAs per SM");
     static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
     static_assert(BT * 128 * 4 <= STG * (ATM ? XBYTES : ABYTES), "split-K partials overlay the first stages");
-    static_assert(!ATM || (BT == 128 && TMEM_NEED <= 512), "ATM layout");
+    static_assert(!ATM || TMEM_NEED <= (kPair ? 256 : 512), "ATM layout: TMEM per CTA");
 };
 
 template <int BT, bool F16, bool ACT>
-__global__ void __launch_bounds__(TgCfg<BT, F16 && BT == 128>::THREADS, TgCfg<BT, F16 && BT == 128>::CTAS_PER_SM)
+__global__ void __launch_bounds__(TgCfg<BT, true>::THREADS, TgCfg<BT, true>::CTAS_PER_SM)
     gemm_tcg_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, TcParams p) {
-    constexpr bool ATM = F16 && BT == 128;  // A operand in tensor memory
+    constexpr bool ATM = true;  // A operand in tensor memory
     using C = TgCfg<BT, ATM>;
     // The activation epilogues are a separate instantiation: compiled into
     // the plain kernel, they cost the 128-token tile its register budget.
@@ -673,7 +674,7 @@ __global__ void __launch_bounds__(TgCfg<BT, F16 && BT == 128>::THREADS, TgCfg<BT
         // ----------------------------------------------------- MMA issuer
         if (ATM && elect_one()) {
             // A from TMEM: stage i's weights at columns ACOL + (i % NA) * 64
-            const uint32_t idesc = idesc_f16_f32(C::BW, BT);
+            const uint32_t idesc = F16 ? idesc_f16_f32(C::BW, BT) : idesc_bf16_f32(C::BW, BT);
             const uint64_t xdesc0 = sw128_desc(smem_u32(xs));
             constexpr uint32_t kXStep = C::XBYTES >> 4, kXAtom = C::XBOX >> 4;
             int committed = 0;
@@ -744,9 +745,15 @@ __global__ void __launch_bounds__(TgCfg<BT, F16 && BT == 128>::THREADS, TgCfg<BT
         __syncwarp();
     } else if (ATM && warp >= C::DQ0 && warp < C::FW0) {
         // ------------------------------------------- dequantize into TMEM
-        // thread = half hh (64 k) of weight row r (its TMEM lane, so the warp
-        // covers the lane quadrant it may access); 8 words -> 32 columns of
-        // f16 pairs (k, k+1), the A layout of kind::f16 from TMEM
+        // DQW = 4: one thread per weight row (16 words = 128 k per stage);
+        // DQW = 8: two threads per row, each one 64-k half (8 words).  The
+        // row is the thread's TMEM lane, so each warp covers the lane
+        // quadrant it may access.  A word (8 codes) becomes 4 columns of
+        // 16-bit pairs (k, k+1), the A layout of kind::f16 from TMEM: f16
+        // by the hardware e2m1 convert, or bf16 by the byte-plane LUT.
+        constexpr int kHalves = C::DQW / 4;
+        constexpr int kWords = 16 / kHalves;
+        const Bf16Lut lut = make_lut(p.t.mag, 1.f);
         const int dw = warp - C::DQ0;
         const int q = warp & 3;
         const int r = q * 32 + lane;
@@ -759,25 +766,37 @@ __global__ void __launch_bounds__(TgCfg<BT, F16 && BT == 128>::THREADS, TgCfg<BT
                 raise_status(p.status, kStatusTimeout);
                 break;
             }
+            // 16-byte unit u of the row's 64 bytes sits at unit u ^ ((r >> 1) & 3)
             const uint8_t* prow = wsr + ws * C::WBYTES + r * 64;
-            uint32_t words[8];
+            uint32_t words[kWords];
+            uint32_t dep = 0;
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const uint4 w = lds128_tc(prow + (((u + 2 * hh) ^ swp) << 4));
+            for (int u = 0; u < kWords / 4; ++u) {
+                const uint4 w = lds128_tc(prow + (((u + (kWords / 4) * hh) ^ swp) << 4));
                 words[4 * u + 0] = w.x;
                 words[4 * u + 1] = w.y;
                 words[4 * u + 2] = w.z;
                 words[4 * u + 3] = w.w;
+                dep ^= w.x;
             }
-            mbar_arrive_after(&wempty[ws], words[0] ^ words[4], dep_slots + dw * 32 + lane);
-            uint32_t o[32];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) e2m1_to_f16x8(words[c], o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+            // release the packed-code stage once its words are in registers
+            mbar_arrive_after(&wempty[ws], dep, dep_slots + dw * 32 + lane);
             if (!__all_sync(0xffffffffu, mbar_wait(&aempty[a], ((uint32_t)(i / C::NA) & 1u) ^ 1u, to))) {
                 raise_status(p.status, kStatusTimeout);
                 break;
             }
-            tmem_st32(tl + (uint32_t)(C::ACOL + a * 64 + hh * 32), o);
+#pragma unroll
+            for (int h = 0; h < kWords / 8; ++h) {
+                uint32_t o[32];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    if constexpr (F16)
+                        e2m1_to_f16x8(words[8 * h + c], o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+                    else
+                        dequant8(words[8 * h + c], lut, o + 4 * c);
+                }
+                tmem_st32(tl + (uint32_t)(C::ACOL + a * 64 + (hh + h) * 32), o);
+            }
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
@@ -1201,7 +1220,7 @@ cudaError_t launch_x_rows_to_f16(const uint16_t* X, int M, int K, uint16_t* Xh, 
 
 template <int BT, bool F16>
 static cudaError_t launch_tcg_bt(const CUtensorMap& mx, const CUtensorMap& mw, const TcParams& p, cudaStream_t st) {
-    using C = TgCfg<BT, F16 && BT == 128>;
+    using C = TgCfg<BT, true>;
     static bool attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
