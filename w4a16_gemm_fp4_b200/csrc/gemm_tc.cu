@@ -23,11 +23,13 @@
 //   warp 0       TMA producer: activation tiles (128-byte swizzle) and the
 //                packed code tiles (uint8, 128 rows) into shared-memory rings;
 //   warp 1       TMEM allocator and MMA issuer: one thread issues tcgen05.mma
-//                (K = 16) into the group's TMEM accumulator and commits;
-//   DQW warps    dequantize codes into exact 16-bit values, K-major with the
-//                128-byte swizzle (byte-plane LUT to bf16, or for E2M1 on the
-//                f16 path the hardware e2m1x2 -> f16x2 convert; 16-byte
-//                stores);
+//                (K = 16; A from shared memory or, at group 128, from TMEM)
+//                into the group's TMEM accumulator and commits;
+//   DQW warps    dequantize codes into exact 16-bit values (byte-plane LUT
+//                to bf16, or for E2M1 on the f16 path the hardware
+//                e2m1x2 -> f16x2 convert): group 32/64 kernel into K-major
+//                128-byte-swizzled shared-memory tiles; group-128 kernel
+//                into tensor memory, the MMA's A operand (tcgen05.st);
 //   NF warps     fold: for each group, tcgen05.ld the group accumulator and
 //                add s[n,g] * it to fp32 totals held in registers, then
 //                release the accumulator; finally the epilogue: * rho (and
@@ -500,20 +502,19 @@ __global__ void __launch_bounds__(TcCfg<BT>::THREADS, TcCfg<BT>::CTAS_PER_SM)
 // Stage s and accumulator s are the same index (STG == NACC): the next use
 // of a stage needs its accumulator folded first, so a stage barrier can
 // never run two phases ahead of the fold warps that wait on it.
-// ATM: the dequant warps write the weights into tensor memory, the A
-// operand of `tcgen05.mma` taken from TMEM, instead of shared memory.  A
-// stage in shared memory then carries only the activations, which removes
-// the 32 KB of dequantized codes written and read back per stage, the
-// shared-memory traffic that set the stage period.  TMEM per CTA: STG
-// accumulators x BT columns + 2 A stages x 64 (512 columns at BT = 128,
-// 256 for each of the two CTAs per SM of the smaller tiles).
-template <int BT, bool ATM = false>
+// The dequant warps write the weights into tensor memory, the A operand
+// of `tcgen05.mma` taken from TMEM, not into shared memory: a stage in
+// shared memory carries only the activations.  (Dequantized tiles in shared
+// memory cost 32 KB written and read back per stage; that traffic set the
+// stage period: prefill 873 -> 969 TFLOP/s when they moved to TMEM.)  TMEM
+// per CTA: STG accumulators x BT columns + 2 A stages x 64 (512 columns at
+// BT = 128, 256 for each of the two CTAs per SM of the smaller tiles).
+template <int BT>
 struct TgCfg {
     static constexpr int BW = 128;              // weight rows per tile (MMA M)
     static constexpr int KB = 128;              // k per stage = one group
     static constexpr int XBOX = BT * 128;       // activation box: 64 k x BT rows, 128-byte swizzle
     static constexpr int XBYTES = 2 * XBOX;     // activations of one stage (128 k)
-    static constexpr int ABYTES = 2 * 16384;    // dequantized codes: two 128-row x 64-k SW128 atoms
     static constexpr int WBYTES = BW * 64;      // packed codes of one stage: 128 rows x 64 B, 64-byte swizzle
     static constexpr bool kPair = BT <= 64;     // two CTAs per SM for small token tiles
     static constexpr int CTAS_PER_SM = kPair ? 2 : 1;
@@ -525,12 +526,12 @@ struct TgCfg {
     static constexpr int DQ0 = 2;
     static constexpr int FW0 = DQ0 + DQW;
     static constexpr int THREADS = (FW0 + NF) * 32;
-    static constexpr int NA = 2;                // A stages in TMEM (ATM)
-    static constexpr int ACOL = STG * BT;       // first TMEM column of the A stages (ATM)
-    static constexpr int TMEM_NEED = ATM ? STG * BT + NA * 64 : (STG * BT < 32 ? 32 : STG * BT);
+    static constexpr int NA = 2;                // A stages in TMEM, 64 columns each
+    static constexpr int ACOL = STG * BT;       // first TMEM column of the A stages
+    static constexpr int TMEM_NEED = STG * BT + NA * 64;
     static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
-    static constexpr int RING = STG * ((ATM ? 0 : ABYTES) + XBYTES) + WST * WBYTES;
-    static constexpr int NBAR = 4 * STG + 2 * WST + (ATM ? NA : 0);
+    static constexpr int RING = STG * XBYTES + WST * WBYTES;
+    static constexpr int NBAR = 4 * STG + 2 * WST + NA;
     static constexpr int DEP = DQW * 32 * 4;  // per-dequant-thread scratch words (stage release)
     // per fold warp, the f16 path's row factors of its FCOLS tokens
     static constexpr int XFB = kPair ? 0 : NF * FCOLS * 4;
@@ -540,15 +541,14 @@ struct TgCfg {
     static constexpr int SMEM = RING + SLACK + NBAR * 8 + 16 + DEP + XFB;
     static_assert(!kPair || SMEM + 1024 <= 228 * 1024 / 2, "two CTAs per SM");
     static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
-    static_assert(BT * 128 * 4 <= STG * (ATM ? XBYTES : ABYTES), "split-K partials overlay the first stages");
-    static_assert(!ATM || TMEM_NEED <= (kPair ? 256 : 512), "ATM layout: TMEM per CTA");
+    static_assert(BT * 128 * 4 <= STG * XBYTES, "split-K partials overlay the activation stages");
+    static_assert(TMEM_NEED <= (kPair ? 256 : 512), "TMEM per CTA");
 };
 
 template <int BT, bool F16, bool ACT>
-__global__ void __launch_bounds__(TgCfg<BT, true>::THREADS, TgCfg<BT, true>::CTAS_PER_SM)
+__global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
     gemm_tcg_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, TcParams p) {
-    constexpr bool ATM = true;  // A operand in tensor memory
-    using C = TgCfg<BT, ATM>;
+    using C = TgCfg<BT>;
     // The activation epilogues are a separate instantiation: compiled into
     // the plain kernel, they cost the 128-token tile its register budget.
     const int act = ACT ? p.act : kActNone;
@@ -558,8 +558,7 @@ __global__ void __launch_bounds__(TgCfg<BT, true>::THREADS, TgCfg<BT, true>::CTA
         if (threadIdx.x == 0) raise_status(p.status, kStatusLayout);
         return;  // before any barrier, copy or TMEM allocation
     }
-    uint8_t* as = smem;                         // STG x ABYTES: dequantized codes (not with ATM)
-    uint8_t* xs = ATM ? smem : as + C::STG * C::ABYTES;  // STG x XBYTES: activations
+    uint8_t* xs = smem;                         // STG x XBYTES: activations
     uint8_t* wsr = xs + C::STG * C::XBYTES;     // WST x WBYTES: packed codes
     uint64_t* bars = reinterpret_cast<uint64_t*>(wsr + C::WST * C::WBYTES);
     uint64_t* xfull = bars;                 // activations landed
@@ -568,8 +567,8 @@ __global__ void __launch_bounds__(TgCfg<BT, true>::THREADS, TgCfg<BT, true>::CTA
     uint64_t* wfull = kdone + C::STG;       // packed codes landed
     uint64_t* wempty = wfull + C::WST;      // packed codes read
     uint64_t* gempty = wempty + C::WST;     // accumulator folded (kdone's one arrival is the commit)
-    uint64_t* aempty = gempty + C::STG;     // ATM: the MMAs have read the A stage
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(aempty + (ATM ? C::NA : 0));
+    uint64_t* aempty = gempty + C::STG;     // [NA] the MMAs have read the A stage
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(aempty + C::NA);
     uint32_t* dep_slots = tmem_slot + 4;
     float* xf_slots = reinterpret_cast<float*>(dep_slots + C::DEP / 4);
     volatile int* wide_fail = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -588,12 +587,11 @@ __global__ void __launch_bounds__(TgCfg<BT, true>::THREADS, TgCfg<BT, true>::CTA
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STG; ++s) {
             mbar_init(&xfull[s], 1);
-            mbar_init(&afull[s], ATM ? C::DQW : C::DQW * 32);
+            mbar_init(&afull[s], C::DQW);
             mbar_init(&kdone[s], 1);
             mbar_init(&gempty[s], C::NF);
         }
-        if constexpr (ATM)
-            for (int a = 0; a < C::NA; ++a) mbar_init(&aempty[a], 1);
+        for (int a = 0; a < C::NA; ++a) mbar_init(&aempty[a], 1);
         for (int s = 0; s < C::WST; ++s) {
             mbar_init(&wfull[s], 1);
             mbar_init(&wempty[s], C::DQW * 32);
@@ -672,7 +670,7 @@ __global__ void __launch_bounds__(TgCfg<BT, true>::THREADS, TgCfg<BT, true>::CTA
         __syncwarp();
     } else if (warp == 1) {
         // ----------------------------------------------------- MMA issuer
-        if (ATM && elect_one()) {
+        if (elect_one()) {
             // A from TMEM: stage i's weights at columns ACOL + (i % NA) * 64
             const uint32_t idesc = F16 ? idesc_f16_f32(C::BW, BT) : idesc_bf16_f32(C::BW, BT);
             const uint64_t xdesc0 = sw128_desc(smem_u32(xs));
@@ -705,45 +703,9 @@ __global__ void __launch_bounds__(TgCfg<BT, true>::THREADS, TgCfg<BT, true>::CTA
                 if (!mbar_wait(&kdone[last % C::STG], (uint32_t)(last / C::STG) & 1u, to))
                     raise_status(p.status, kStatusTimeout);
             }
-        } else if (!ATM && elect_one()) {
-            const uint32_t idesc = F16 ? idesc_f16_f32(C::BW, BT) : idesc_bf16_f32(C::BW, BT);
-            const uint64_t adesc0 = sw128_desc(smem_u32(as)), xdesc0 = sw128_desc(smem_u32(xs));
-            constexpr uint32_t kAStep = C::ABYTES >> 4, kXStep = C::XBYTES >> 4;
-            constexpr uint32_t kAAtom = 16384 >> 4, kXAtom = C::XBOX >> 4;
-            int s = 0, committed = 0;
-            uint32_t ph = 0;
-            bool ok = true;
-            for (int i = 0; i < nkb && ok; ++i) {
-                if (!mbar_wait(&afull[s], ph, to) || !mbar_wait(&xfull[s], ph, to) ||
-                    !mbar_wait(&gempty[s], ph ^ 1u, to)) {
-                    raise_status(p.status, kStatusTimeout);
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint64_t ad = adesc0 + (uint64_t)(s * kAStep);
-                const uint64_t xd = xdesc0 + (uint64_t)(s * kXStep);
-                const uint32_t d = tmem + (uint32_t)(s * BT);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    tc_mma_f16(d, ad + (uint64_t)((kk >> 2) * kAAtom + 2 * (kk & 3)),
-                               xd + (uint64_t)((kk >> 2) * kXAtom + 2 * (kk & 3)), idesc, kk ? 1u : 0u);
-                tc_commit(&kdone[s]);
-                ++committed;
-                if (++s == C::STG) {
-                    s = 0;
-                    ph ^= 1u;
-                }
-            }
-            // TMEM is freed below: the last commit must have landed
-            if (committed > 0) {
-                const int last = committed - 1;
-                if (!mbar_wait(&kdone[last % C::STG], (uint32_t)(last / C::STG) & 1u, to))
-                    raise_status(p.status, kStatusTimeout);
-            }
         }
         __syncwarp();
-    } else if (ATM && warp >= C::DQ0 && warp < C::FW0) {
+    } else if (warp >= C::DQ0 && warp < C::FW0) {
         // ------------------------------------------- dequantize into TMEM
         // DQW = 4: one thread per weight row (16 words = 128 k per stage);
         // DQW = 8: two threads per row, each one 64-k half (8 words).  The
@@ -801,60 +763,6 @@ __global__ void __launch_bounds__(TgCfg<BT, true>::THREADS, TgCfg<BT, true>::CTA
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&afull[a]);
-        }
-    } else if (!ATM && warp >= C::DQ0 && warp < C::FW0) {
-        // ---------------------------------------------------- dequantize
-        // DQW = 4: one thread per weight row (16 words = 128 k per stage);
-        // DQW = 8: two threads per row, each one 64-k atom (8 words).
-        constexpr int kHalves = C::DQW / 4;
-        constexpr int kWords = 16 / kHalves;
-        const Bf16Lut lut = make_lut(p.t.mag, 1.f);
-        const int tid = (warp - C::DQ0) * 32 + lane;
-        const int r = tid & 127;                    // weight row within the tile
-        const int hh = kHalves == 1 ? 0 : tid >> 7; // atom (64-k half) of this thread
-        const int sw = r & 7;                       // 128-byte swizzle of the dequantized atoms
-        const int swp = (r >> 1) & 3;               // 64-byte swizzle of the packed stage
-        for (int i = 0; i < nkb; ++i) {
-            const int ws = i % C::WST, s = i % C::STG;
-            if (!mbar_wait(&wfull[ws], (uint32_t)(i / C::WST) & 1u, to) ||
-                !mbar_wait(&kdone[s], ((uint32_t)(i / C::STG) & 1u) ^ 1u, to)) {
-                raise_status(p.status, kStatusTimeout);
-                break;
-            }
-            // 16-byte unit u of the row's 64 bytes sits at unit u ^ ((r >> 1) & 3);
-            // units 2 hh, 2 hh + 1 hold atom hh's 8 words
-            const uint8_t* prow = wsr + ws * C::WBYTES + r * 64;
-            uint32_t words[kWords];
-#pragma unroll
-            for (int u = 0; u < kWords / 4; ++u) {
-                const uint4 w = lds128_tc(prow + (((u + 2 * hh) ^ swp) << 4));
-                words[4 * u + 0] = w.x;
-                words[4 * u + 1] = w.y;
-                words[4 * u + 2] = w.z;
-                words[4 * u + 3] = w.w;
-            }
-            // release the packed-code stage as soon as its words are in registers
-            // (the dependency takes one word of every load)
-            uint32_t dep = 0;
-#pragma unroll
-            for (int u = 0; u < kWords / 4; ++u) dep ^= words[4 * u];
-            mbar_arrive_after(&wempty[ws], dep, dep_slots + tid);
-            // word c of this thread holds k = 8 (c + kWords hh) .. + 7:
-            // atom (c + kWords hh) >> 3, 16-byte unit c & 7 of row r
-            uint8_t* arow = as + s * C::ABYTES + r * 128;
-#pragma unroll
-            for (int c = 0; c < kWords; ++c) {
-                const int cc = c + kWords * hh;
-                uint32_t v[4];
-                if constexpr (F16)
-                    e2m1_to_f16x8(words[c], v[0], v[1], v[2], v[3]);
-                else
-                    dequant8(words[c], lut, v);
-                *reinterpret_cast<uint4*>(arow + (cc >> 3) * 16384 + (((cc & 7) ^ sw) << 4)) =
-                    make_uint4(v[0], v[1], v[2], v[3]);
-            }
-            fence_proxy_async_smem();
-            mbar_arrive(&afull[s]);
         }
     } else if (warp >= C::FW0) {
         // ---------------------------------------------- fold + epilogue
@@ -1220,7 +1128,7 @@ cudaError_t launch_x_rows_to_f16(const uint16_t* X, int M, int K, uint16_t* Xh, 
 
 template <int BT, bool F16>
 static cudaError_t launch_tcg_bt(const CUtensorMap& mx, const CUtensorMap& mw, const TcParams& p, cudaStream_t st) {
-    using C = TgCfg<BT, true>;
+    using C = TgCfg<BT>;
     static bool attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
