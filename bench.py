@@ -828,6 +828,20 @@ def profile_case(case):
         Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
         for _ in range(3):
             api.gemm(X, q["packed"], q["scales"], api.E2M1, GROUP, out=Y)
+    elif kind == "w4a4":
+        # the W4A4 product: outlier activations calibrated and coded to E2M1,
+        # weights quantized with the same channel shift
+        N, K, M = dims
+        W = torch.from_numpy(synth.lognormal_row_weights(rng, N, K)).cuda()
+        Xb, _ = synth.outlier_activations(rng, M, K)
+        X = torch.from_numpy(Xb.view(np.int16)).cuda().view(torch.bfloat16)
+        shift, rho = api.preshift_calibrate(X)
+        q = api.quantize(W, GROUP, api.E2M1, False, shift)
+        del W
+        ap, a_scale = api.act_quantize(X, rho, api.E2M1, 0, shift)
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        for _ in range(3):
+            api.gemm_w4a4(ap, a_scale, q["packed"], q["scales"], api.E2M1, api.E2M1, GROUP, out=Y)
     elif kind == "quantize":
         N, K = dims
         W = torch.from_numpy(synth.lognormal_row_weights(rng, N, K)).cuda()
@@ -913,7 +927,8 @@ def main():
                     help="seconds of untimed replays before the timed region (clock sampling)")
     ap.add_argument("--profile-case", metavar="CASE",
                     help="run one case a few times and exit, for ncu captures: gemm:N:K:M (E2M1 g128 fp16 "
-                         "scales, synthetic weights and activations) or quantize:N:K")
+                         "scales, synthetic weights and activations), w4a4:N:K:M (4-bit activations) or "
+                         "quantize:N:K")
     ap.add_argument("--cpu-configs", action="store_true",
                     help="time the CPU oracle on every configuration (1 thread and all cores), print JSON, exit")
     ap.add_argument("--record-traffic", metavar="CSV[,CSV]",
