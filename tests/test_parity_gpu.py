@@ -491,13 +491,15 @@ def row_rel_err(Y, Yref):
     return worst
 
 
-@pytest.mark.parametrize("M,splits", [(65, 0), (200, 0), (300, 0), (300, 1), (130, 3)])
+@pytest.mark.parametrize("M,splits", [(65, 0), (200, 0), (300, 0), (300, 1), (130, 3), (9, 0), (16, 4), (33, 0),
+                                      (64, 0), (64, 8)])
 def test_gemm_f16_activation_rows(fp4, oracle_mod, M, splits):
-    """The 128-token tile runs E2M1 weights in f16 when given the workspace:
-    each activation row is rescaled by a power of two into the f16 range and
-    the factor is undone in the epilogue.  Rows 2^120 apart in magnitude
-    must each meet the bound against their own magnitude, with and without
-    the workspace (bf16 path)."""
+    """The tensor engine runs E2M1 weights in f16 when given the workspace
+    (every token tile but the 64-token one, which stays bf16): each activation row is rescaled by a power of two
+    into the f16 range and the factor is undone in the epilogue (split-K:
+    in the cluster reduction).  Rows 2^120 apart in magnitude must each meet
+    the bound against their own magnitude, with and without the workspace
+    (bf16 path)."""
     N, K = 256, 1024
     W, _ = synth.random_case(40 + M, N, K, 1)
     X = wide_range_rows(41 + M, M, K)
@@ -508,8 +510,11 @@ def test_gemm_f16_activation_rows(fp4, oracle_mod, M, splits):
     assert need >= M * K * 2 + M * 4
     ws = torch.empty(need, dtype=torch.uint8, device="cuda")
     small = torch.empty(16, dtype=torch.uint8, device="cuda")
-    a = fp4.gemm(dev_bf16(X), res["packed"], res["scales"], 1, 128, x_scale=xs, splits=splits, workspace=ws)
-    b = fp4.gemm(dev_bf16(X), res["packed"], res["scales"], 1, 128, x_scale=xs, splits=splits, workspace=small)
+    eng = fp4.ENGINE_TENSOR
+    a = fp4.gemm(dev_bf16(X), res["packed"], res["scales"], 1, 128, x_scale=xs, splits=splits, workspace=ws,
+                 engine=eng)
+    b = fp4.gemm(dev_bf16(X), res["packed"], res["scales"], 1, 128, x_scale=xs, splits=splits, workspace=small,
+                 engine=eng)
     assert row_rel_err(a, Yref) <= TOL
     assert row_rel_err(b, Yref) <= TOL
 

@@ -534,7 +534,7 @@ struct TgCfg {
     static constexpr int NBAR = 4 * STG + 2 * WST + NA;
     static constexpr int DEP = DQW * 32 * 4;  // per-dequant-thread scratch words (stage release)
     // per fold warp, the f16 path's row factors of its FCOLS tokens
-    static constexpr int XFB = kPair ? 0 : NF * FCOLS * 4;
+    static constexpr int XFB = NF * FCOLS * 4;
     // the 64-token layout only fits two CTAs per SM without alignment slack:
     // it relies on the 1024-byte-aligned dynamic shared-memory base (checked)
     static constexpr int SLACK = BT == 64 ? 0 : 1024;
@@ -1189,9 +1189,11 @@ cudaError_t launch_gemm_tc(const uint16_t* X, const uint8_t* packed, const void*
         if (splits <= 0) splits = tcg_splits(M, N, K);
         if (splits > K / 128) splits = K / 128;
         if (splits > 8) splits = 8;
-        // E2M1 codes on the 128-token tile: hardware convert to f16 and f16
-        // activations (needs the workspace; without it the bf16 path runs)
-        const bool f16 = BTg == 128 && e2m1 && ws != nullptr && ws_bytes >= tc_f16_ws_bytes(M, K);
+        // E2M1 codes: hardware convert to f16 and f16 activations (needs the
+        // workspace; without it the bf16 path runs).  Not on the 64-token
+        // tile: there the row pre-pass costs what the convert saves (measured
+        // on 4096x11008: 17.3 us bf16, 17.9 us f16; at 16 tokens 14.5 -> 12.9)
+        const bool f16 = e2m1 && BTg != 64 && ws != nullptr && ws_bytes >= tc_f16_ws_bytes(M, K);
         uint16_t* Xh = f16 ? static_cast<uint16_t*>(ws) : nullptr;
         float* xrow = f16 ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + xh_bytes(M, K)) : nullptr;
         CUtensorMap mx, mw;
@@ -1219,7 +1221,11 @@ cudaError_t launch_gemm_tc(const uint16_t* X, const uint8_t* packed, const void*
         if (f16) {
             cudaError_t e = launch_x_rows_to_f16(X, M, K, Xh, xrow, nullptr, 0, st);
             if (e != cudaSuccess) return e;
-            return launch_tcg_bt<128, true>(mx, mw, p, st);
+            switch (BTg) {
+                case 16: return launch_tcg_bt<16, true>(mx, mw, p, st);
+                case 32: return launch_tcg_bt<32, true>(mx, mw, p, st);
+                default: return launch_tcg_bt<128, true>(mx, mw, p, st);
+            }
         }
         switch (BTg) {
             case 16: return launch_tcg_bt<16, false>(mx, mw, p, st);

@@ -18,9 +18,11 @@
 // fp32; fold warps then add s[n,g] * acc to fp32 totals, as in the W4A16
 // tensor engine, and the epilogue multiplies by s_a.
 //
-// Six shared-memory stages keep copies in flight across the ~1 us latency
-// of a TMA load; four TMEM accumulators (all 512 columns) decouple the
-// MMAs from the fold.
+// Tiles of 128 weight rows x 256 tokens (N = 256 MMAs read half the
+// shared-memory operand bytes per flop of a 128-token tile, whose operand
+// reads matched the MMA rate) with four copy stages and two 256-column
+// accumulators; 128-token tiles for M <= 128 with six stages and four.
+// The accumulators fill all 512 TMEM columns.
 //
 // Warp roles (2 + NF warps, one CTA per SM):
 //   warp 0   TMA producer: the first ring-full of weight codes before the
