@@ -239,9 +239,13 @@ FP4_API fp4_status fp4_preshift_calibrate_noalloc(const uint16_t *X, int M, int 
  * fp4_gemm_w4a4:
  *   Y[m,n] = bf16( act( s_a * sum_k v_a(a[m,k]) * v(w[n,k]) * s[n,k/group] ) )
  *   apacked [M][K/2] from fp4_act_quantize in format afmt, a_scale its s_a;
- *   the weights, act, Y and the engine choice as for fp4_gemm_act.  The
- *   activation values (exact in bf16) are expanded into the workspace and
- *   multiplied on the 16-bit tensor paths.
+ *   the weights, act and Y as for fp4_gemm_act.  E2M1 activations with
+ *   E2M1 weights at group 128, M > 64, with apacked and packed 32-byte
+ *   aligned, multiply as 4-bit codes on tcgen05.mma kind::f8f6f4 (no
+ *   dequantization; each group's code-product sum is exact in fp32, then
+ *   scaled by s[n,g] in fp32).  Every other case expands the activation
+ *   values (exact in bf16) into the workspace and runs fp4_gemm_act's
+ *   engines on them.
  *   workspace  fp4_gemm_w4a4_workspace_size(M, N, K) bytes, zero-filled
  *              once before first use (its first part is the GEMM
  *              workspace, with the same rules).
