@@ -102,3 +102,15 @@ def test_reference_arm_json_line():
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     assert line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_launches_per_call_counts_the_prepass():
+    """The bench's launch count: one kernel per decode-engine call and per
+    64-token call, two (f16 pre-pass + GEMM) for the other tensor tiles."""
+    from w4a16_gemm_fp4_b200 import api
+    calls = {(M, N, K): bench.launches_per_call(api, M, N, K) for M in bench.MS for (N, K) in bench.SHAPES}
+    for (M, N, K), n in calls.items():
+        decode = api.gemm_engine_for(M, N, K, bench.GROUP) == api.ENGINE_DECODE
+        assert n == (1 if decode or 32 < M <= 64 else 2), (M, N, K, n)
+    # the sweep: M = 16 on all three matrices takes the tensor engine's 16-token tile
+    assert sum(calls.values()) == 15
