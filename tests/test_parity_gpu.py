@@ -520,10 +520,12 @@ def test_gemm_f16_activation_rows(fp4, oracle_mod, M, splits):
 
 
 @pytest.mark.parametrize("K", [2176, 4224, 8320, 16512])
-def test_gemm_f16_row_lengths(fp4, oracle_mod, K):
+@pytest.mark.parametrize("M", [70, 1100])
+def test_gemm_f16_row_lengths(fp4, oracle_mod, K, M):
     """Row lengths that take each form of the f16 activation pre-pass (the
-    row held in 2, 4 or 8 registers per thread, or read twice)."""
-    M, N = 70, 128
+    row held in 2, 4, 8 or 16 registers per thread, or read twice; 256
+    threads per row, or 128 from 1024 rows)."""
+    N = 128 if M < 1024 else 32
     W, _ = synth.random_case(K, N, K, 1)
     X = wide_range_rows(K + 1, M, K)
     res = fp4.quantize(dev_f32(W), 128, 1)

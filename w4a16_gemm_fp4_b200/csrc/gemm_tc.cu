@@ -1041,12 +1041,14 @@ static cudaError_t launch_tc_bt(const CUtensorMap& mx, const CUtensorMap& mw, co
 // i.e. under 2^-39 of the row maximum); infinities and NaNs pass through.
 //
 // R = 16-byte vectors of the row each thread keeps in registers (one read
-// of X); R = 0 reads the row twice (any K).
-template <int R>
-__global__ void __launch_bounds__(256) x_rows_to_f16_kernel(const uint16_t* __restrict__ X, int K,
-                                                            uint16_t* __restrict__ Xh, float* __restrict__ xrow,
-                                                            int* zero, int nzero) {
-    __shared__ uint32_t wmax[8];
+// of X); R = 0 reads the row twice (any K).  T threads per row: 256, or 128
+// for many rows (twice the bytes in flight per thread, and all of a
+// 2048-row prefill resident in one wave).
+template <int R, int T>
+__global__ void __launch_bounds__(T) x_rows_to_f16_kernel(const uint16_t* __restrict__ X, int K,
+                                                          uint16_t* __restrict__ Xh, float* __restrict__ xrow,
+                                                          int* zero, int nzero) {
+    __shared__ uint32_t wmax[T / 32];
     const int m = blockIdx.x, nv = K >> 3;
     const uint4* src = reinterpret_cast<const uint4*>(X + (size_t)m * K);
     uint4* dst = reinterpret_cast<uint4*>(Xh + (size_t)m * K);
@@ -1056,13 +1058,13 @@ __global__ void __launch_bounds__(256) x_rows_to_f16_kernel(const uint16_t* __re
     pdl_wait();  // X may come from the previous kernel in the stream
     // the decode engine's tile counters start at zero
     if (zero && m == 0)
-        for (int i = threadIdx.x; i < nzero; i += 256) zero[i] = 0;
+        for (int i = threadIdx.x; i < nzero; i += T) zero[i] = 0;
     uint32_t mx2 = 0;  // per-half maxima of the finite magnitudes (bf16 bits order like the values)
     uint4 v[R > 0 ? R : 1];
     if constexpr (R > 0) {
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-            const int i = threadIdx.x + r * 256;
+            const int i = threadIdx.x + r * T;
             v[r] = i < nv ? src[i] : make_uint4(0u, 0u, 0u, 0u);
             mx2 = finite_mag_max2(mx2, v[r].x);
             mx2 = finite_mag_max2(mx2, v[r].y);
@@ -1070,7 +1072,7 @@ __global__ void __launch_bounds__(256) x_rows_to_f16_kernel(const uint16_t* __re
             mx2 = finite_mag_max2(mx2, v[r].w);
         }
     } else {
-        for (int i = threadIdx.x; i < nv; i += 256) {
+        for (int i = threadIdx.x; i < nv; i += T) {
             const uint4 u = src[i];
             mx2 = finite_mag_max2(finite_mag_max2(finite_mag_max2(finite_mag_max2(mx2, u.x), u.y), u.z), u.w);
         }
@@ -1082,7 +1084,7 @@ __global__ void __launch_bounds__(256) x_rows_to_f16_kernel(const uint16_t* __re
     __syncthreads();
     mx = wmax[0];
 #pragma unroll
-    for (int w = 1; w < 8; ++w) mx = max(mx, wmax[w]);
+    for (int w = 1; w < T / 32; ++w) mx = max(mx, wmax[w]);
     const int E = (int)(mx >> 7);  // biased exponent of the row maximum
     int sh = mx == 0 ? 0 : 141 - (E < 1 ? 1 : E);
     if (sh > 126) sh = 126;
@@ -1091,11 +1093,11 @@ __global__ void __launch_bounds__(256) x_rows_to_f16_kernel(const uint16_t* __re
     if constexpr (R > 0) {
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-            const int i = threadIdx.x + r * 256;
+            const int i = threadIdx.x + r * T;
             if (i < nv) dst[i] = bf16x8_to_f16x8(v[r], sc);
         }
     } else {
-        for (int i = threadIdx.x; i < nv; i += 256) dst[i] = bf16x8_to_f16x8(src[i], sc);
+        for (int i = threadIdx.x; i < nv; i += T) dst[i] = bf16x8_to_f16x8(src[i], sc);
     }
 }
 
@@ -1107,8 +1109,9 @@ size_t tc_f16_ws_bytes(int M, int K) { return xh_bytes(M, K) + (size_t)M * 4; }
 cudaError_t launch_x_rows_to_f16(const uint16_t* X, int M, int K, uint16_t* Xh, float* xrow, int* zero, int nzero,
                                  cudaStream_t st) {
     cudaLaunchConfig_t cfg = {};
+    const bool narrow = M >= 1024;  // 128 threads per row
     cfg.gridDim = dim3((unsigned)M, 1, 1);
-    cfg.blockDim = dim3(256, 1, 1);
+    cfg.blockDim = dim3(narrow ? 128 : 256, 1, 1);
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1117,11 +1120,20 @@ cudaError_t launch_x_rows_to_f16(const uint16_t* X, int M, int K, uint16_t* Xh, 
     cfg.numAttrs = 1;
     const int nv = K / 8;
     cudaError_t e;
-    if (nv <= 256) e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<1>, X, K, Xh, xrow, zero, nzero);
-    else if (nv <= 512) e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<2>, X, K, Xh, xrow, zero, nzero);
-    else if (nv <= 1024) e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<4>, X, K, Xh, xrow, zero, nzero);
-    else if (nv <= 2048) e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<8>, X, K, Xh, xrow, zero, nzero);
-    else e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<0>, X, K, Xh, xrow, zero, nzero);
+    if (narrow) {
+        if (nv <= 128) e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<1, 128>, X, K, Xh, xrow, zero, nzero);
+        else if (nv <= 256) e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<2, 128>, X, K, Xh, xrow, zero, nzero);
+        else if (nv <= 512) e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<4, 128>, X, K, Xh, xrow, zero, nzero);
+        else if (nv <= 1024) e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<8, 128>, X, K, Xh, xrow, zero, nzero);
+        else if (nv <= 2048) e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<16, 128>, X, K, Xh, xrow, zero, nzero);
+        else e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<0, 128>, X, K, Xh, xrow, zero, nzero);
+    } else {
+        if (nv <= 256) e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<1, 256>, X, K, Xh, xrow, zero, nzero);
+        else if (nv <= 512) e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<2, 256>, X, K, Xh, xrow, zero, nzero);
+        else if (nv <= 1024) e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<4, 256>, X, K, Xh, xrow, zero, nzero);
+        else if (nv <= 2048) e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<8, 256>, X, K, Xh, xrow, zero, nzero);
+        else e = cudaLaunchKernelEx(&cfg, x_rows_to_f16_kernel<0, 256>, X, K, Xh, xrow, zero, nzero);
+    }
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
