@@ -817,7 +817,7 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
         if (wide) {
             // every MMA, and so every copy and dequantization, has completed
             // once the last stage has been folded: the fp32 tile [128 tokens]
-            // [128 rows] * rho goes over the dequantized-code stages (row =
+            // [128 rows] * rho goes over the activation stages (row =
             // token: the lanes' consecutive weight rows are consecutive words)
             // and all dequant and fold warps store it below.  No loads here:
             // a load per element would serialise on its latency.
@@ -850,7 +850,7 @@ __global__ void __launch_bounds__(TgCfg<BT>::THREADS, TgCfg<BT>::CTAS_PER_SM)
         } else {
             // every MMA, and so every copy and dequantization, has completed
             // once the last stage has been folded: the partial tile
-            // [BT tokens][128 rows] overlays the dequantized-code stages
+            // [BT tokens][128 rows] overlays the activation stages
             float* part = reinterpret_cast<float*>(smem);
 #pragma unroll
             for (int j = 0; j < C::FCOLS; ++j) part[(cb + j) * 128 + r] = tot[j];
